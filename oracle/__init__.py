@@ -1,0 +1,170 @@
+"""CPU oracle for MLA decode and latent-condensed attention (LCA).
+
+TEST INFRASTRUCTURE ONLY.  The CUDA library and its Python binding never
+import this package.  Only the tests, the package smoke check and the
+benchmark's CPU-baseline / reference leg use it.
+
+The arithmetic lives in ``lca_oracle.c`` (plain fp64 loops, one function per
+definition of "Latent-Condensed Transformer for Efficient Long Context
+Modeling", sections 整体框架 / 关键设计 1-3).  This module compiles it with
+gcc (OpenMP over independent sequences, groups, heads or prefill blocks) and
+exposes numpy wrappers.  Inputs are the exact bf16 bit patterns (uint16
+arrays); outputs are fp64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lca_oracle.c")
+_LIB = os.path.join(_HERE, "liblca_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library (gcc -O2 -fopenmp, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        Lg = ctypes.c_long
+        Dd = ctypes.c_double
+        lib.ora_num_threads.restype = I
+        lib.ora_num_groups.restype = Lg
+        lib.ora_num_groups.argtypes = [Lg, I, I]
+        lib.ora_lca_condense.restype = I
+        lib.ora_lca_condense.argtypes = [P, P, I, Lg, I, I, I, I, I, Dd, P, P, P, P, P]
+        lib.ora_mla_decode.restype = I
+        lib.ora_mla_decode.argtypes = [P, P, P, I, Lg, I, I, I, I, Dd, P, P]
+        lib.ora_lca_decode.restype = I
+        lib.ora_lca_decode.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
+        lib.ora_lca_attend_reps.restype = I
+        lib.ora_lca_attend_reps.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P]
+        lib.ora_lca_prefill.restype = I
+        lib.ora_lca_prefill.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, P, Lg,
+                                        P, P, P]
+        _lib = lib
+    return _lib
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == np.uint16, a.dtype
+    return a
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return _load().ora_num_threads()
+
+
+def num_groups(L: int, g: int, w: int) -> int:
+    """m = max(0, floor((L - w) / g))."""
+    return int(_load().ora_num_groups(L, g, w))
+
+
+def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64):
+    """cache [B,L,dc+dr] u16, q_recent [B,g,H,dc+dr] u16 ->
+    dict(rep_c [B,m,dc], rep_k [B,m,dr], anchor [B,m] int32 (position in the
+    sequence), alpha [B,m,g], score [B,m,g])."""
+    cache, q_recent = _u16(cache), _u16(q_recent)
+    B, L, D = cache.shape
+    H = q_recent.shape[2]
+    dc = D - dr
+    m = num_groups(L, g, w)
+    out = dict(rep_c=np.zeros((B, m, dc)), rep_k=np.zeros((B, m, dr)),
+               anchor=np.zeros((B, m), np.int32), alpha=np.zeros((B, m, g)),
+               score=np.zeros((B, m, g)))
+    _load().ora_lca_condense(_ptr(cache), _ptr(q_recent), B, L, H, dc, dr, g, w, scale,
+                             _ptr(out["rep_c"]), _ptr(out["rep_k"]), _ptr(out["anchor"]),
+                             _ptr(out["alpha"]), _ptr(out["score"]))
+    return out
+
+
+def mla_decode(cache, q, w_uv, scale: float, dr: int = 64):
+    """-> (o_lat [B,H,dc], out [B,H,dv]) in fp64."""
+    cache, q, w_uv = _u16(cache), _u16(q), _u16(w_uv)
+    B, L, D = cache.shape
+    H = q.shape[1]
+    dc = D - dr
+    dv = w_uv.shape[2]
+    o_lat = np.zeros((B, H, dc))
+    out = np.zeros((B, H, dv))
+    _load().ora_mla_decode(_ptr(cache), _ptr(q), _ptr(w_uv), B, L, H, dc, dr, dv, scale,
+                           _ptr(o_lat), _ptr(out))
+    return o_lat, out
+
+
+def lca_decode(cache, q_recent, q, w_uv, g: int, w: int, scale: float, dr: int = 64):
+    """-> (o_lat [B,H,dc], out [B,H,dv], anchor [B,m])."""
+    cache, q_recent, q, w_uv = _u16(cache), _u16(q_recent), _u16(q), _u16(w_uv)
+    B, L, D = cache.shape
+    H = q.shape[1]
+    dc = D - dr
+    dv = w_uv.shape[2]
+    m = num_groups(L, g, w)
+    o_lat = np.zeros((B, H, dc))
+    out = np.zeros((B, H, dv))
+    anchor = np.zeros((B, max(m, 1)), np.int32)
+    _load().ora_lca_decode(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L, H, dc, dr,
+                           dv, g, w, scale, _ptr(o_lat), _ptr(out), _ptr(anchor))
+    return o_lat, out, anchor[:, :m]
+
+
+def lca_attend_reps(cache, rep, q, w_uv, g: int, w: int, scale: float, dr: int = 64):
+    """Attention over bf16 representative rows rep [B,m,dc+dr] + window.
+    -> (o_lat, out)."""
+    cache, rep, q, w_uv = _u16(cache), _u16(rep), _u16(q), _u16(w_uv)
+    B, L, D = cache.shape
+    H = q.shape[1]
+    dc = D - dr
+    dv = w_uv.shape[2]
+    o_lat = np.zeros((B, H, dc))
+    out = np.zeros((B, H, dv))
+    _load().ora_lca_attend_reps(_ptr(cache), _ptr(rep), _ptr(q), _ptr(w_uv), B, L, H, dc, dr,
+                                dv, g, w, scale, _ptr(o_lat), _ptr(out))
+    return o_lat, out
+
+
+def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, scale: float,
+                blocks=None, dr: int = 64, want_anchor: bool = False):
+    """Blockwise LCA prefill.  -> (o_lat [B,q_len,H,dc], out [B,q_len,H,dv], anchor|None).
+    `blocks` = absolute block indices to evaluate (others left as NaN)."""
+    cache, qpre, w_uv = _u16(cache), _u16(qpre), _u16(w_uv)
+    B, L, D = cache.shape
+    H = qpre.shape[2]
+    dc = D - dr
+    dv = w_uv.shape[2]
+    o_lat = np.full((B, q_len, H, dc), np.nan)
+    out = np.full((B, q_len, H, dv), np.nan)
+    bl = None
+    nbl = 0
+    if blocks is not None:
+        bl = np.ascontiguousarray(np.asarray(blocks, dtype=np.int64))
+        nbl = len(bl)
+    m_max = num_groups(q_start + q_len - g, g, w)
+    anchor = np.full((B, q_len // g, max(m_max, 1)), -1, np.int32) if want_anchor else None
+    rc = _load().ora_lca_prefill(_ptr(cache), _ptr(qpre), _ptr(w_uv), B, L, q_start, q_len, H,
+                                 dc, dr, dv, g, w, scale, _ptr(bl), nbl, _ptr(o_lat), _ptr(out),
+                                 _ptr(anchor))
+    if rc != 0:
+        raise ValueError("bad prefill range")
+    return o_lat, out, anchor
