@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""LCA decode benchmark: tokens/s and cache-read GB/s against the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+One step = one whole fused LCA decode step (summary query, importance,
+group softmax pooling, anchor pick, split-L attention over
+[representatives || window], log-sum-exp combine, W_UV up-projection) for
+every sequence of the batch, through the C ABI.  Inputs are synthetic and
+seeded (see mla_latent_space_lca_b200/inputs.py) and resident in HBM; the
+default workload's cache (1.2 GB) is ~10x the L2, so no flush is needed
+between steps.  Multi-GPU (torchrun): each rank decodes its own batch (weak
+scaling, no data-path collective); timing is the max over ranks.  Rank 0
+prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from mla_latent_space_lca_b200.inputs import WORKLOADS, make_decode_inputs  # noqa: E402
+
+ROW_BYTES = 576 * 2
+METRIC = "LCA decode tokens/s and cache-read GB/s (fraction of B200 HBM roofline)"
+PROFILE_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_b32_l32k")
+    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.rows = []
+        self.marks = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        t0, t1 = (self.marks + [0, 0])[:2] if len(self.marks) >= 2 else (0, 1e30)
+        inside = [r for t, r in self.rows if t0 <= t <= t1]
+        note = None
+        if not inside:
+            # timed region shorter than the sampling period: nearest sample
+            inside = [min(self.rows, key=lambda tr: abs(tr[0] - t0))[1]]
+            note = "timed region shorter than one 100 ms sample; nearest sample"
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in inside if len(r) > 8 and num(r[1]) is not None]
+        mx = [num(r[2]) for r in inside if len(r) > 8 and num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for k, nm in enumerate(names):
+                if len(r) > 5 + k and r[5 + k].lower().startswith("active"):
+                    reasons.add(nm)
+        out = {"sm_mhz": statistics.median(sm) if sm else None,
+               "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+               "samples": len(inside)}
+        if note:
+            out["note"] = note
+        return out
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in ("attn_decode.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "mla_latent_space_lca_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    try:
+        with open(PROFILE_FILE) as f:
+            d = json.load(f)
+        e = d[workload]
+        if e.get("source_hash") != source_hash():
+            return None
+        return e["dram_bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0):
+    """The oracle as it stands, on host cores, over a bounded sample of the
+    workload (whole sequences).  Returns (tokens/s, cores, sample text,
+    per-step seconds)."""
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits
+
+    B = inp.cache.shape[0]
+    # sample size: sequences whose oracle decode takes ~1-3 s
+    per_seq_guess = inp.L * 16 * 576 * 2 / 3e9
+    S = max(1, min(B, int(2.0 / max(per_seq_guess, 1e-6))))
+    sl = list(range(S))
+    c = bf16_bits(inp.cache[:S])
+    qr = bf16_bits(inp.q_recent[:S])
+    q = bf16_bits(inp.q[:S])
+    w = bf16_bits(inp.w_uv)
+    for _ in range(warmup):
+        oracle.lca_decode(c, qr, q, w, inp.g, inp.w, inp.scale)
+    times = []
+    t_start = time.time()
+    n = 0
+    while True:
+        t0 = time.perf_counter()
+        oracle.lca_decode(c, qr, q, w, inp.g, inp.w, inp.scale)
+        times.append(time.perf_counter() - t0)
+        n += 1
+        if (steps and n >= steps) or (not steps and time.time() - t_start >= budget_s):
+            break
+    tok_s = S * n / sum(times)
+    sample = (f"{S} of {B} sequences (L={inp.L}) per oracle call, {n} calls, "
+              f"{sum(times):.1f} s of CPU time")
+    del sl
+    return tok_s, oracle.num_threads(), sample, times
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    inp = make_decode_inputs(wl["B"], wl["L"], seed=0)
+    tok_s, cores, sample, times = cpu_baseline(inp, 0, steps=args.steps, warmup=args.warmup)
+    ms = 1e3 * statistics.mean(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": wl["B"], "L": wl["L"], "g": 16, "w": 1024},
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+
+    import mla_latent_space_lca_b200 as lca
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    assert wl["kind"] == "decode"
+    B, L = wl["B"], wl["L"]
+    inp = make_decode_inputs(B, L, seed=rank)
+    cache, q_recent, q, w_uv = (inp.cache.to(dev), inp.q_recent.to(dev), inp.q.to(dev),
+                                inp.w_uv.to(dev))
+    ws = lca.workspace(3, B, L, device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lca.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)
+    n0 = lca.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    launches = (lca.launch_count() - n0) / args.steps
+    barrier()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    if sampler:
+        sampler.stop()
+
+    # per-kernel durations (CUDA events around each launch, on its stream)
+    prof_steps = min(args.steps, 200)
+    lca.profile_enable(True)
+    for _ in range(prof_steps):
+        step()
+    torch.cuda.synchronize()
+    prof = lca.profile_collect()
+    lca.profile_enable(False)
+
+    # end to end through the public API: pinned host inputs -> device -> result -> host
+    pin = [t.pin_memory() for t in (inp.cache, inp.q_recent, inp.q)]
+    h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
+    dbuf = [torch.empty_like(t, device=dev) for t in pin]
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    d2h = h_out.numel() * 4
+    for _ in range(1):
+        for d, h in zip(dbuf, pin):
+            d.copy_(h, non_blocking=True)
+        lca.lca_decode(dbuf[0], dbuf[1], dbuf[2], w_uv, scale=inp.scale, out=out, ws=ws)
+        h_out.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        for d, h in zip(dbuf, pin):
+            d.copy_(h, non_blocking=True)
+        lca.lca_decode(dbuf[0], dbuf[1], dbuf[2], w_uv, scale=inp.scale, out=out, ws=ws)
+        h_out.copy_(out, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = x0.elapsed_time(x1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    rc, detail = lca.device_status(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+
+    if rank != 0:
+        return
+    tokens = B * world
+    value = tokens / (ms / 1e3)
+    gbs = B * L * ROW_BYTES * world / (ms / 1e3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    attn = prof.get("attn_decode")
+    attn_ms = attn[1] / attn[0] if attn else None
+    algo_bytes = B * L * ROW_BYTES
+    achieved = algo_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
+    traffic = ncu_traffic(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B_per_gpu": B, "L": L, "g": 16, "w": 1024,
+                   "heads": 16, "d_c": 512, "d_r": 64, "parallelism": f"replicas x{world}",
+                   "l2": "inputs (B*L*1152 B) larger than the 126 MB L2; no flush"},
+        "cache_gbps": gbs, "cache_frac_of_hbm": gbs / world / peak,
+        "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak if achieved else None, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": algo_bytes,
+                     "launch_ms": attn_ms},
+        "kernels_ms_per_step": {k: v[1] / v[0] for k, v in prof.items()},
+        "gpu_launches": launches,
+        "clocks": sampler.summary() if sampler else None,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        tok_s, cores, sample, _ = cpu_baseline(inp, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+/*
+ * lca.h -- C ABI of liblca_b200.so: multi-head latent attention (MLA) decode
+ * read straight from the compressed latent KV cache, and latent-condensed
+ * attention (LCA) on top of it, as hand-written sm_100a (B200) kernels.
+ *
+ * Method: "Latent-Condensed Transformer for Efficient Long Context Modeling"
+ * (papernotes.org notes on the ACL 2026 paper).  整体框架 (overall
+ * framework): history outside a local window of w recent tokens is cut into
+ * m = floor((L - w) / g) groups; each group is condensed into one
+ * representative; attention runs over [m representatives || window].
+ * 关键设计 1: the representative latent is c_j^rep = sum_i alpha_i c_i^KV with
+ * alpha = softmax of the tokens' importance under the summary query (mean of
+ * the last g queries).  关键设计 2: the representative RoPE key is the key of
+ * the group's most important token, k_j^{R_rep} = k^R_{I_j}.  关键设计 3: the
+ * window is kept uncompressed.
+ *
+ * Fixed model dimensions: H = 16 heads, latent d_c = 512, RoPE key d_r = 64,
+ * cache row D = 576 bf16 (1152 bytes: [c^KV | k^R]), value width d_v = 128.
+ * Queries come in the weight-absorbed form q = [q_lat (512) | q_rope (64)]
+ * per head, so logits are taken against the latent directly:
+ *   z = scale * (q_lat . c + q_rope . k^R),  o_lat = sum p c,
+ *   out_h = W_UV[h]^T o_lat,h  (W_UV laid out [16][512][128]).
+ * The importance of token i is s_i = (1/H) sum_h scale * (qbar_h . row_i);
+ * a representative carries no logit bias; the anchor is the first index of
+ * the group maximum; tokens left over by the floor join the window.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the
+ *    library allocates no device memory.  bf16 tensors are passed as
+ *    `const void*` holding IEEE bfloat16 values, row-major and contiguous.
+ *  - Every bf16 / fp32 tensor pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous on it and never synchronise the host.
+ *  - Return 0 (LCA_OK) or a negative lca_status.  Invalid arguments are
+ *    rejected before anything is launched.  A launch failure returns
+ *    LCA_ERR_CUDA with nothing further enqueued.
+ *  - `ws` is caller-owned device scratch of at least
+ *    lca_workspace_bytes(op, ...) bytes, 256-byte aligned.  Its contents on
+ *    entry do not matter; two calls in flight at once need separate ws.
+ *  - Every in-kernel wait is bounded; a kernel whose wait expires records
+ *    LCA_ERR_DEVICE_TIMEOUT in a device status word (read it with
+ *    lca_device_status) and returns early, leaving outputs undefined.
+ *  - The current token is already in the cache: the query of a decode step
+ *    sits at position L-1 of a cache of length L.
+ */
+#ifndef LCA_B200_H
+#define LCA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LCA_HEADS 16
+#define LCA_DC 512
+#define LCA_DR 64
+#define LCA_D 576
+#define LCA_DV 128
+
+/* Status codes. */
+#define LCA_OK 0
+#define LCA_ERR_INVALID_ARG (-1)   /* NULL pointer, bad size or range */
+#define LCA_ERR_MISALIGNED (-2)    /* a pointer is not 16-byte aligned (ws: 256) */
+#define LCA_ERR_WORKSPACE (-3)     /* ws NULL or smaller than lca_workspace_bytes */
+#define LCA_ERR_UNSUPPORTED (-4)   /* parameter outside what the kernels implement */
+#define LCA_ERR_CUDA (-5)          /* a CUDA runtime/driver call or launch failed */
+#define LCA_ERR_NO_DEVICE (-6)     /* the current device is not sm_100 */
+#define LCA_ERR_DEVICE_TIMEOUT (-7) /* a kernel's bounded wait expired */
+
+/* Condensation parameters.  g: group size (16; g = 1 makes every token its
+ * own representative, which is exactly MLA).  w: local window (>= 0).
+ * scale: logit scale (1/sqrt(192) for the 128+64 per-head MLA width). */
+typedef struct {
+    int g;
+    int w;
+    float scale;
+} lca_params;
+
+/* Operation ids for lca_workspace_bytes. */
+#define LCA_OP_MLA_DECODE 0
+#define LCA_OP_CONDENSE 1
+#define LCA_OP_DECODE_ATTN 2
+#define LCA_OP_DECODE 3
+#define LCA_OP_PREFILL 4
+
+/* m = max(0, floor((L - w) / g)); 0 for invalid parameters. */
+int64_t lca_num_groups(int64_t L, lca_params p);
+
+/* Device scratch an entry point needs for this problem size, in bytes
+ * (0 for invalid parameters).  q_len is used by LCA_OP_PREFILL only. */
+size_t lca_workspace_bytes(int op, int B, int64_t L, int64_t q_len, lca_params p);
+
+/* MLA decode (the uncondensed reference point, "MLA keeps all L tokens in
+ * attention", 研究背景与动机): each of B sequences' current query attends
+ * all L cached rows; split-L across the GPU, log-sum-exp combine, then the
+ * per-head W_UV up-projection.
+ *   cache [B][L][576] bf16, q [B][16][576] bf16, w_uv [16][512][128] bf16
+ *   out   [B][16][128] fp32            (required)
+ *   o_lat [B][16][512] fp32 or NULL    (attention output before W_UV)
+ * 1 <= B, 1 <= L < 2^31. */
+int mla_decode_attn(const void *cache, const void *q, const void *w_uv, int B, int64_t L,
+                    float scale, float *out, float *o_lat, void *ws, size_t ws_bytes,
+                    void *stream);
+
+/* LCA condensation (关键设计 1 and 2) of the m history groups of each
+ * sequence with the summary query qbar = mean of q_recent:
+ *   cache    [B][L][576] bf16
+ *   q_recent [B][g][16][576] bf16 (the last g queries, current one last)
+ *   rep      [B][m][576] bf16  out: [c_rep (512) | k^R of the anchor (64)],
+ *            the latent rounded to bf16 like a cache row, the key copied
+ *            bit for bit
+ *   anchor   [B][m] int32 out or NULL: absolute position of each anchor
+ *   alpha    [B][m][g] fp32 out or NULL: pooling weights
+ * Requires g == 16.  m == 0 is valid (nothing is written). */
+int lca_condense(const void *cache, const void *q_recent, int B, int64_t L, lca_params p,
+                 void *rep, int32_t *anchor, float *alpha, void *ws, size_t ws_bytes,
+                 void *stream);
+
+/* LCA decode attention over stored representatives (整体框架): the current
+ * query attends [rep rows 0..m-1 || cache rows m*g .. L-1], then W_UV.
+ *   rep [B][m][576] bf16 (as written by lca_condense); may be NULL if m == 0.
+ * Other arguments as mla_decode_attn.  Requires g == 16. */
+int lca_decode_attn(const void *cache, const void *rep, const void *q, const void *w_uv, int B,
+                    int64_t L, lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes,
+                    void *stream);
+
+/* One whole LCA decode step, fused: summary query, per-group importance,
+ * softmax pooling, anchor pick and attention over [representatives ||
+ * window] in one pass over the cache (representatives never leave the
+ * chip), log-sum-exp combine, W_UV.  Same results as lca_condense followed
+ * by lca_decode_attn, except that representatives are not rounded to bf16.
+ *   anchor [B][m] int32 out or NULL.
+ * g == 1 runs mla_decode_attn (every token is its own representative).
+ * Otherwise requires g == 16. */
+int lca_decode(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B,
+               int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor, void *ws,
+               size_t ws_bytes, void *stream);
+
+/* Blockwise LCA prefill of query positions [q_start, q_start + q_len) (both
+ * multiples of g).  Block k covers t0 = k*g .. t0+g-1; its summary query is
+ * the mean of its own g queries; history rows 0 .. m_k*g-1 with
+ * m_k = floor((t0 - w)/g) (0 when t0 <= w) are condensed with it; each query
+ * t of the block attends [m_k representatives || cache rows m_k*g .. t].
+ *   cache [B][L][576] bf16, q [B][L][16][576] bf16 (rows outside the range
+ *   are not read), w_uv [16][512][128] bf16
+ *   out   [B][q_len][16][128] fp32, o_lat [B][q_len][16][512] fp32 or NULL
+ * Requires g == 16. */
+int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L,
+                      int64_t q_start, int64_t q_len, lca_params p, float *out, float *o_lat,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* Text for a status code (static storage). */
+const char *lca_strerror(int status);
+
+/* Reads (and if clear != 0 resets) the device status word of the current
+ * device: LCA_OK or LCA_ERR_DEVICE_TIMEOUT with the kernel id in bits 8..15
+ * of *detail.  Synchronises the device. */
+int lca_device_status(int clear, int *detail);
+
+/* Kernel timing.  lca_profile_enable(1) makes every later call record a
+ * CUDA event pair around each kernel it launches (on the call's stream);
+ * lca_profile_collect() waits for them, fills up to `max` entries
+ * {name, launches, total_ms} and resets the record.  Returns the number of
+ * entries or a negative status. */
+typedef struct {
+    char name[32];
+    int launches;
+    double total_ms;
+} lca_kernel_time;
+int lca_profile_enable(int on);
+int lca_profile_collect(lca_kernel_time *out, int max);
+
+/* Number of kernels this library has launched since it was loaded. */
+int64_t lca_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LCA_B200_H */

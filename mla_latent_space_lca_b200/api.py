@@ -1,0 +1,164 @@
+"""PyTorch-facing wrappers of the C ABI (argument marshalling only).
+
+Every function takes CUDA tensors, checks dtype / shape / contiguity,
+allocates missing outputs and scratch with torch (device memory is the only
+thing PyTorch provides here), and calls the corresponding entry point of
+liblca_b200.so on the current stream.  All arithmetic runs in the library's
+kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import LcaParams, check
+
+H, D_C, D_R, D, D_V = 16, 512, 64, 576, 128
+
+
+def default_scale() -> float:
+    return 1.0 / math.sqrt(192.0)
+
+
+def _params(g: int, w: int, scale: float | None) -> LcaParams:
+    return LcaParams(int(g), int(w), float(default_scale() if scale is None else scale))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def num_groups(L: int, g: int = 16, w: int = 1024) -> int:
+    return int(_lib.lib().lca_num_groups(L, _params(g, w, None)))
+
+
+def workspace_bytes(op: int, B: int, L: int, q_len: int = 0, g: int = 16, w: int = 1024) -> int:
+    return int(_lib.lib().lca_workspace_bytes(op, B, L, q_len, _params(g, w, None)))
+
+
+def workspace(op: int, B: int, L: int, q_len: int = 0, g: int = 16, w: int = 1024,
+              device=None) -> torch.Tensor:
+    n = workspace_bytes(op, B, L, q_len, g, w)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def mla_decode_attn(cache, q, w_uv, scale=None, out=None, o_lat=None, ws=None, stream=None):
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    ws = workspace(_lib.OP_MLA_DECODE, B, L, device=cache.device) if ws is None else ws
+    rc = _lib.lib().mla_decode_attn(_ptr(cache), _ptr(q), _ptr(w_uv), B, L,
+                                    float(default_scale() if scale is None else scale), _ptr(out),
+                                    _ptr(o_lat), _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "mla_decode_attn")
+    return out
+
+
+def lca_condense(cache, q_recent, g=16, w=1024, scale=None, rep=None, anchor=None, alpha=None,
+                 ws=None, stream=None):
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
+    m = num_groups(L, g, w)
+    dev = cache.device
+    rep = torch.empty(B, m, D, dtype=torch.bfloat16, device=dev) if rep is None else rep
+    ws = workspace(_lib.OP_CONDENSE, B, L, g=g, w=w, device=dev) if ws is None else ws
+    rc = _lib.lib().lca_condense(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale),
+                                 _ptr(rep) if m > 0 else None, _ptr(anchor), _ptr(alpha), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    check(rc, "lca_condense")
+    return rep
+
+
+def lca_decode_attn(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None, ws=None,
+                    stream=None):
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    m = num_groups(L, g, w)
+    if m > 0:
+        _need(rep, "rep", torch.bfloat16, (B, m, D))
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_decode_attn(_ptr(cache), _ptr(rep) if m > 0 else None, _ptr(q), _ptr(w_uv),
+                                    B, L, _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(ws),
+                                    ws.numel(), _stream(stream))
+    check(rc, "lca_decode_attn")
+    return out
+
+
+def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None,
+               anchor=None, ws=None, stream=None):
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    if g != 1:
+        _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_decode(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
+                               _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(anchor), _ptr(ws),
+                               ws.numel(), _stream(stream))
+    check(rc, "lca_decode")
+    return out
+
+
+def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, out=None,
+                      o_lat=None, ws=None, stream=None):
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q, "q", torch.bfloat16, (B, L, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    out = (torch.empty(B, q_len, H, D_V, dtype=torch.float32, device=cache.device)
+           if out is None else out)
+    ws = workspace(_lib.OP_PREFILL, B, L, q_len, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_prefill_block(_ptr(cache), _ptr(q), _ptr(w_uv), B, L, q_start, q_len,
+                                      _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(ws),
+                                      ws.numel(), _stream(stream))
+    check(rc, "lca_prefill_block")
+    return out
+
+
+def device_status(clear: bool = True) -> tuple[int, int]:
+    d = ctypes.c_int(0)
+    rc = _lib.lib().lca_device_status(1 if clear else 0, ctypes.byref(d))
+    return rc, d.value
+
+
+def profile_enable(on: bool = True) -> None:
+    check(_lib.lib().lca_profile_enable(1 if on else 0), "lca_profile_enable")
+
+
+def profile_collect() -> dict:
+    arr = (_lib.KernelTime * 16)()
+    n = _lib.lib().lca_profile_collect(arr, 16)
+    if n < 0:
+        check(n, "lca_profile_collect")
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
+
+
+def launch_count() -> int:
+    return int(_lib.lib().lca_launch_count())

@@ -1,0 +1,493 @@
+// attn_decode.cuh -- split-L flash-decode attention on tcgen05 tensor cores,
+// read straight from the MLA latent cache, with the LCA condensation fused in.
+//
+// Row sources ("tiles" of 64 rows, 1152 B each, TMA-loaded as 9 boxes of
+// [64 rows x 64 columns] with 128-byte swizzle, 72 KB per stage, 3 stages):
+//   MODE_MLA : cache rows 0..L-1 (MLA decode, every token attends).
+//   MODE_REPS: stored representatives rep[b][0..m) then window rows m*g..L-1.
+//   MODE_LCA : raw history rows 0..m*16-1 (4 groups of 16 per tile), condensed
+//              on the fly, then window rows m*16..L-1.
+//
+// Tensor-core formulation (per tile, M=128):
+//   S  [128 x 64]  = A(TMEM, 128 lanes x 576) * rows^T     (tcgen05 TS MMA)
+//     The A operand holds per-lane query rows.  In warp quadrant q (lanes
+//     32q..32q+31) lane r holds:
+//       MLA/REPS: r<4: full q of head 4q+r
+//       LCA:      r<4: latent half of q (rope zeroed)  -> X = q_lat . c
+//                 4<=r<8: rope half of q (latent zeroed) -> Y = q_rope . k^R
+//                 r=8,9: hi and lo bf16 parts of the folded summary query u
+//                        -> importance s = u . row   (关键设计 1)
+//   O^T[512 x 16] += rows_lat^T * P^T                       (tcgen05 SS MMA,
+//     4 x M=128 over d, N = 16 heads, K = 64 rows; A is the same smem tile read
+//     MN-major, so the tile is read from HBM exactly once)
+// For an LCA history tile, with alpha the group softmax of s and I_j the
+// group argmax, the logit of representative j for head h is
+//   z_hj = scale * (sum_{i in G_j} alpha_i X_hi + Y_h,I_j)
+// = scale * (q_lat,h . c_j^rep + q_rope,h . k^R_{I_j}), exactly the
+// representative's logit (关键设计 1 and 2) without materialising c_j^rep, and
+// its value contribution p_hj c_j^rep = sum_i (p_hj alpha_i) c_i is the PV
+// MMA with per-token weights p_hj * alpha_i.
+//
+// Warp roles (192 threads): warps 0-3 softmax / epilogue (one TMEM lane
+// quadrant each), warp 4 MMA issuer, warp 5 TMA producer.  Online softmax
+// keeps a per-head reference max and rescales O only when the max grows by
+// more than 2^8 (the final normalisation uses the same reference, so the
+// result is exact either way).  Each CTA writes one (O, m, l) partial per
+// sequence piece it owns; combine_kernel merges them.
+#pragma once
+#include "common.cuh"
+
+namespace lca {
+
+constexpr int AT_TILE = 64;
+constexpr int AT_STAGES = 3;
+constexpr int AT_CHUNK = AT_TILE * 128;          // 8192 B: [64 rows x 64 cols] bf16
+constexpr int AT_STAGE = 9 * AT_CHUNK;           // 73728 B
+constexpr int AT_PBUF = LCA_HEADS * 128;         // 2048 B: P^T [16 heads x 64 rows] bf16
+constexpr uint32_t AT_TM_Q = 0;                  // 288 columns (bf16 pairs)
+constexpr uint32_t AT_TM_S0 = 288;               // 64 columns
+constexpr uint32_t AT_TM_S1 = 352;               // 64 columns
+constexpr uint32_t AT_TM_O = 416;                // 4 x 16 columns
+constexpr uint32_t AT_TM_COLS = 512;
+constexpr int AT_THREADS = 192;
+
+constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
+constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
+constexpr int AT_NBAR = 19;
+constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
+constexpr int AT_SMEM = AT_OFF_MISC + 256;              // 225792
+constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
+
+enum { MODE_MLA = 0, MODE_REPS = 1, MODE_LCA = 2 };
+
+struct AttnArgs {
+    const uint16_t *q;     // [B][16][576]
+    const uint16_t *uhl;   // [B][2][576] (LCA)
+    int64_t L;
+    int64_t m;             // representatives / groups per sequence (0 for MLA)
+    int64_t win0;          // first window row (m*g), 0 for MLA
+    int n_hist;            // tiles before the window per sequence
+    int n_tiles;           // tiles per sequence
+    int64_t T;             // B * n_tiles
+    int G;                 // CTAs
+    float sl2;             // scale * log2(e)
+    float *part_o;         // [G+B][16][512]
+    float *part_ml;        // [G+B][16][2]
+    int32_t *anchor;       // [B][m] or NULL (LCA)
+};
+
+struct TileInfo {
+    int from_rep;   // 1: rows come from the representative tensor
+    int hist;       // 1: LCA history tile (groups), 0: plain rows
+    int64_t row;    // first row
+    int valid;      // valid rows (plain) or valid groups (hist)
+};
+
+template <int MODE>
+__device__ __forceinline__ TileInfo tile_info(const AttnArgs &a, int k)
+{
+    TileInfo ti;
+    ti.from_rep = 0;
+    ti.hist = 0;
+    if (MODE != MODE_MLA && k < a.n_hist) {
+        if (MODE == MODE_REPS) {
+            ti.from_rep = 1;
+            ti.row = int64_t(k) * AT_TILE;
+            ti.valid = int(min64(AT_TILE, a.m - ti.row));
+        } else {
+            ti.hist = 1;
+            ti.row = int64_t(k) * AT_TILE;
+            ti.valid = int(min64(4, a.m - int64_t(k) * 4));
+        }
+        return ti;
+    }
+    const int kw = (MODE == MODE_MLA) ? k : k - a.n_hist;
+    ti.row = a.win0 + int64_t(kw) * AT_TILE;
+    ti.valid = int(min64(AT_TILE, a.L - ti.row));
+    return ti;
+}
+
+// Write this lane's 576-wide query row (or zeros) into TMEM columns
+// AT_TM_Q.. of its lane.  See the lane map in the file header.
+template <int MODE>
+__device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int quad, int lane,
+                                            uint32_t tmem)
+{
+    const uint16_t *src = nullptr;
+    int keep_lo = 0, keep_hi = 18;   // 16-column chunks [keep_lo, keep_hi) are kept
+    if (MODE == MODE_LCA) {
+        if (lane < 4) {
+            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane) * LCA_D;
+            keep_hi = 16;
+        } else if (lane < 8) {
+            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane - 4) * LCA_D;
+            keep_lo = 16;
+        } else if (lane < 10) {
+            src = a.uhl + (size_t(b) * 2 + (lane - 8)) * LCA_D;
+        }
+    } else {
+        if (lane < 4) src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane) * LCA_D;
+    }
+    const uint32_t base = tmem + (uint32_t(32 * quad) << 16) + AT_TM_Q;
+#pragma unroll 1
+    for (int cc = 0; cc < 18; ++cc) {
+        uint32_t r[16];
+        if (src && cc >= keep_lo && cc < keep_hi) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(src + 32 * cc);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 x = p[v];
+                r[4 * v + 0] = x.x;
+                r[4 * v + 1] = x.y;
+                r[4 * v + 2] = x.z;
+                r[4 * v + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int v = 0; v < 16; ++v) r[v] = 0u;
+        }
+        tmem_st16(base + 16 * cc, r);
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(AT_THREADS, 1)
+    attn_decode_kernel(const __grid_constant__ CUtensorMap map_cache,
+                       const __grid_constant__ CUtensorMap map_rep, const AttnArgs a)
+{
+    extern __shared__ uint8_t at_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // barrier ids
+    auto BAR = [&](int i) -> uint32_t { return sbase + AT_OFF_BAR + 8 * i; };
+    auto full = [&](int s) { return BAR(s); };
+    auto empty = [&](int s) { return BAR(3 + s); };
+    auto sfull = [&](int s) { return BAR(6 + s); };
+    auto sempty = [&](int s) { return BAR(8 + s); };
+    auto pfull = [&](int s) { return BAR(10 + s); };
+    auto pempty = [&](int s) { return BAR(12 + s); };
+    auto fex = [&](int s) { return BAR(17 + s); };
+    const uint32_t ofull = BAR(14), segready = BAR(15), drain = BAR(16);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
+    float *fsc = reinterpret_cast<float *>(smem + AT_OFF_MISC + 128);   // [2][16]
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 3; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(sfull(s), 1);
+            mbar_init(sempty(s), 4);
+            mbar_init(pfull(s), 4);
+            mbar_init(pempty(s), 1);
+        }
+        mbar_init(ofull, 1);
+        mbar_init(segready, 4);
+        mbar_init(drain, 1);
+        mbar_init(fex(0), 4);
+        mbar_init(fex(1), 4);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(sbase + AT_OFF_MISC, AT_TM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int c = blockIdx.x;
+    const int64_t t_begin = split_begin(c, a.T, a.G);
+    const int64_t t_end = split_begin(c + 1, a.T, a.G);
+    const int n_tiles = a.n_tiles;
+
+    if (warp == 5) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&map_cache);
+            if (MODE == MODE_REPS && a.m > 0) prefetch_tensormap(&map_rep);
+            const uint64_t pol = policy_evict_first();
+            int last[3] = {-1, -1, -1};
+            int i = 0;
+            for (int64_t t = t_begin; t < t_end; ++t, ++i) {
+                const int s = i % 3;
+                if (!mbar_wait(empty(s), ((i / 3) & 1) ^ 1, abort_flag, K_ATTN, 1)) break;
+                const int64_t b = t / n_tiles;
+                const TileInfo ti = tile_info<MODE>(a, int(t - b * n_tiles));
+                mbar_expect_tx(full(s), AT_STAGE);
+                const CUtensorMap *mp = ti.from_rep ? &map_rep : &map_cache;
+                const uint32_t dst = sbase + s * AT_STAGE;
+#pragma unroll 1
+                for (int ch = 0; ch < 9; ++ch)
+                    tma_load_3d(dst + ch * AT_CHUNK, mp, full(s), 64 * ch, int(ti.row), int(b), pol);
+                last[s] = i;
+            }
+            for (int s = 0; s < 3; ++s)
+                if (last[s] >= 0) mbar_wait(full(s), (last[s] / 3) & 1, nullptr, K_ATTN, 2);
+        }
+    } else if (warp == 4) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_S = idesc_bf16(128, AT_TILE, 0, 0);
+            constexpr uint32_t IDESC_PV = idesc_bf16(128, LCA_HEADS, 1, 0);
+            auto issue_pv = [&](int j, bool first_pv) -> bool {
+                if (!mbar_wait(pfull(j & 1), (j >> 1) & 1, abort_flag, K_ATTN, 7)) return false;
+                tc_fence_after();
+                const uint32_t stage = sbase + (j % 3) * AT_STAGE;
+                const uint32_t pbuf = sbase + AT_OFF_P + (j & 1) * AT_PBUF;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sdesc_sw128(stage + 2 * cc * AT_CHUNK + ks * 2048, AT_CHUNK, 1024);
+                        const uint64_t bd = sdesc_sw128(pbuf + ks * 32, 16, 1024);
+                        mma_ss(tmem + AT_TM_O + 16 * cc, ad, bd, IDESC_PV, (first_pv && ks == 0) ? 0u : 1u);
+                    }
+                }
+                tc_commit(empty(j % 3));
+                tc_commit(pempty(j & 1));
+                return true;
+            };
+            bool ok = true;
+            int i = 0, seg = 0;
+            int64_t t = t_begin;
+            while (ok && t < t_end) {
+                const int64_t b = t / n_tiles;
+                const int64_t seg_end = min64(t_end, (b + 1) * int64_t(n_tiles));
+                if (!mbar_wait(segready, seg & 1, abort_flag, K_ATTN, 3)) { ok = false; break; }
+                tc_fence_after();
+                const int first = i;
+                for (; t < seg_end; ++t, ++i) {
+                    const int s = i % 3, sb = i & 1;
+                    if (!mbar_wait(full(s), (i / 3) & 1, abort_flag, K_ATTN, 4)) { ok = false; break; }
+                    if (!mbar_wait(sempty(sb), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 5)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t stage = sbase + s * AT_STAGE;
+                    const uint32_t dS = tmem + (sb ? AT_TM_S1 : AT_TM_S0);
+#pragma unroll 4
+                    for (int ks = 0; ks < 36; ++ks) {
+                        const uint64_t bd = sdesc_sw128(stage + (ks >> 2) * AT_CHUNK + (ks & 3) * 32, 16, 1024);
+                        mma_ts(dS, tmem + AT_TM_Q + 8 * ks, bd, IDESC_S, ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(sfull(sb));
+                    if (i > first && !issue_pv(i - 1, i - 1 == first)) { ok = false; break; }
+                }
+                if (!ok) break;
+                if (!issue_pv(i - 1, i - 1 == first)) { ok = false; break; }
+                tc_commit(ofull);
+                ++seg;
+            }
+            tc_commit(drain);
+            mbar_wait(drain, 0, nullptr, K_ATTN, 6);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps
+        const int quad = warp;
+        const float NEG_INF = -INFINITY;
+        const uint32_t lane_base = uint32_t(32 * quad) << 16;
+        int i = 0, seg = 0;
+        int64_t t = t_begin;
+        bool ok = true;
+        float m_use = NEG_INF, l_run = 0.f;   // lanes 0..3: head 4*quad + lane
+        while (ok && t < t_end) {
+            const int64_t b = t / n_tiles;
+            const int64_t seg_end = min64(t_end, (b + 1) * int64_t(n_tiles));
+            load_q_rows<MODE>(a, b, quad, lane, tmem);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(segready);
+            m_use = NEG_INF;
+            l_run = 0.f;
+            const int first = i;
+            for (; t < seg_end; ++t, ++i) {
+                const int k = int(t - b * n_tiles);
+                const int sb = i & 1;
+                const TileInfo ti = tile_info<MODE>(a, k);
+                ok = mbar_wait(sfull(sb), (i >> 1) & 1, abort_flag, K_ATTN, 8);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                float v[64];
+                tmem_ld64(tmem + lane_base + (sb ? AT_TM_S1 : AT_TM_S0), v);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sempty(sb));
+
+                float w[64];        // P^T weights of this lane's head (lanes 0..3)
+                float tmax;
+                if (MODE == MODE_LCA && ti.hist) {
+                    // ---- fused condensation of 4 groups (lanes 8/9 = u hi/lo)
+                    float z[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float s[16];
+#pragma unroll
+                        for (int kk = 0; kk < 16; ++kk)
+                            s[kk] = v[16 * j + kk] + __shfl_down_sync(0xffffffffu, v[16 * j + kk], 1);
+                        float gm = s[0];
+                        int gi = 0;
+#pragma unroll
+                        for (int kk = 1; kk < 16; ++kk)
+                            if (s[kk] > gm) { gm = s[kk]; gi = kk; }
+                        float den = 0.f;
+#pragma unroll
+                        for (int kk = 0; kk < 16; ++kk) {
+                            s[kk] = fast_exp2((s[kk] - gm) * kLog2e);
+                            den += s[kk];
+                        }
+                        const float inv = 1.f / den;
+#pragma unroll
+                        for (int kk = 0; kk < 16; ++kk)
+                            w[16 * j + kk] = __shfl_sync(0xffffffffu, s[kk] * inv, 8);   // alpha
+                        const int anc = __shfl_sync(0xffffffffu, gi, 8);
+                        if (a.anchor && quad == 0 && lane == 8 && j < ti.valid)
+                            a.anchor[size_t(b) * a.m + size_t(k) * 4 + j] = int32_t((k * 4 + j) * 16 + gi);
+                        const bool is_y = (lane >= 4 && lane < 8);
+                        float rj = 0.f;
+#pragma unroll
+                        for (int kk = 0; kk < 16; ++kk) {
+                            const float cf = is_y ? (kk == anc ? 1.f : 0.f) : w[16 * j + kk];
+                            rj = fmaf(cf, v[16 * j + kk], rj);
+                        }
+                        const float yj = __shfl_down_sync(0xffffffffu, rj, 4);
+                        z[j] = (j < ti.valid) ? (rj + yj) * a.sl2 : NEG_INF;
+                    }
+                    tmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
+                    // reference max update (lanes 0..3 own heads)
+                    float f = 1.f;
+                    if (i == first) {
+                        m_use = tmax;
+                    } else if (tmax > m_use + 8.f) {
+                        f = fast_exp2(m_use - tmax);
+                        m_use = tmax;
+                        l_run *= f;
+                    }
+                    if (lane < 4) fsc[(i & 1) * 16 + 4 * quad + lane] = f;
+                    float psum = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float p = (j < ti.valid) ? fast_exp2(z[j] - m_use) : 0.f;
+                        psum += p;
+#pragma unroll
+                        for (int kk = 0; kk < 16; ++kk) w[16 * j + kk] *= p;
+                    }
+                    l_run += psum;
+                } else {
+                    // ---- plain rows (MLA, stored reps, window)
+                    if (MODE == MODE_LCA) {
+#pragma unroll
+                        for (int e = 0; e < 64; ++e) v[e] += __shfl_down_sync(0xffffffffu, v[e], 4);
+                    }
+                    tmax = NEG_INF;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) {
+                        v[e] = (e < ti.valid) ? v[e] * a.sl2 : NEG_INF;
+                        tmax = fmaxf(tmax, v[e]);
+                    }
+                    float f = 1.f;
+                    if (i == first) {
+                        m_use = tmax;
+                    } else if (tmax > m_use + 8.f) {
+                        f = fast_exp2(m_use - tmax);
+                        m_use = tmax;
+                        l_run *= f;
+                    }
+                    if (lane < 4) fsc[(i & 1) * 16 + 4 * quad + lane] = f;
+                    float psum = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 64; ++e) {
+                        w[e] = (e < ti.valid) ? fast_exp2(v[e] - m_use) : 0.f;
+                        psum += w[e];
+                    }
+                    l_run += psum;
+                }
+
+                // ---- P^T row of this lane's head into the swizzled buffer
+                ok = mbar_wait(pempty(sb), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 9);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                if (lane < 4) {
+                    const int h = 4 * quad + lane;
+                    uint8_t *prow = smem + AT_OFF_P + sb * AT_PBUF + (h >> 3) * 1024 + (h & 7) * 128;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint4 o;
+                        o.x = pack_bf16(w[8 * ch + 0], w[8 * ch + 1]);
+                        o.y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
+                        o.z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
+                        o.w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
+                        *reinterpret_cast<uint4 *>(prow + ((ch ^ (h & 7)) << 4)) = o;
+                    }
+                }
+                fence_proxy_async();
+
+                // ---- rescale O^T columns whose reference max moved (the
+                // factors of all 16 heads are exchanged through fsc)
+                __syncwarp();
+                if (lane == 0) mbar_arrive(fex(i & 1));
+                ok = mbar_wait(fex(i & 1), (i >> 1) & 1, abort_flag, K_ATTN, 12);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                bool any = false;
+                float fs[16];
+#pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    fs[h] = fsc[(i & 1) * 16 + h];
+                    any |= (fs[h] != 1.f);
+                }
+                if (any) {
+                    // PV(i-1) must have landed before O is touched
+                    ok = mbar_wait(pempty((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, K_ATTN, 11);
+                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float o[16];
+                        const uint32_t ta = tmem + lane_base + AT_TM_O + 16 * cc;
+                        tmem_ld16(ta, o);
+                        uint32_t r[16];
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) r[h] = __float_as_uint(o[h] * fs[h]);
+                        tmem_st16(ta, r);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pfull(sb));
+            }
+            if (!ok) break;
+
+            // ---- segment done: write the partial (O, m, l) of sequence b
+            ok = mbar_wait(ofull, seg & 1, abort_flag, K_ATTN, 10);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            const size_t slot = size_t(c) + size_t(b);
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                float o[16];
+                tmem_ld16(tmem + lane_base + AT_TM_O + 16 * cc, o);
+                const int d = 128 * cc + 32 * quad + lane;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) a.part_o[(slot * LCA_HEADS + h) * LCA_DC + d] = o[h];
+            }
+            if (lane < 4) {
+                const size_t hh = slot * LCA_HEADS + 4 * quad + lane;
+                a.part_ml[hh * 2 + 0] = m_use;
+                a.part_ml[hh * 2 + 1] = l_run;
+            }
+            tc_fence_before();
+            ++seg;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, AT_TM_COLS);
+}
+
+}  // namespace lca

@@ -1,0 +1,224 @@
+// condense.cuh -- streaming LCA condensation (关键设计 1 and 2) that writes
+// representatives to memory in cache-row format.
+//
+// One warp condenses one group of 16 tokens at a time.  The group is one
+// contiguous 18 KB span of the cache ([16 rows x 1152 B]); each warp keeps a
+// 3-slot ring of such spans in shared memory, filled by cp.async.bulk with an
+// L2 evict-first hint, so the cache streams through once with ~54 KB per warp
+// in flight.  Per group, from shared memory:
+//   s_i   = u . row_i           (u = folded summary query, fp32 FMA; lanes
+//                                own 16-byte column slices, a halving
+//                                shuffle transpose sums the 16 dots so that
+//                                lanes 2t, 2t+1 end up with token t)
+//   alpha = softmax(s)          (shuffle max / sum over the 16 tokens)
+//   I     = first argmax s      (shuffle reduction on (s, index))
+//   rep   = [sum_i alpha_i c_i (fp32 accumulate, bf16 store) | k^R_I (bit copy)]
+#pragma once
+#include "common.cuh"
+
+namespace lca {
+
+constexpr int CD_WARPS = 4;
+constexpr int CD_SLOTS = 3;
+constexpr int CD_GROUP_BYTES = 16 * LCA_D * 2;                      // 18432
+constexpr int CD_SMEM = CD_WARPS * CD_SLOTS * CD_GROUP_BYTES + CD_WARPS * CD_SLOTS * 8;
+
+struct CondenseArgs {
+    const uint16_t *cache;   // [B][L][576]
+    const float *u;          // [B][576]
+    int64_t L;
+    int64_t m;               // groups per sequence
+    int64_t total;           // B * m
+    uint16_t *rep;           // [B][m][576]
+    int32_t *anchor;         // [B][m] or NULL
+    float *alpha;            // [B][m][16] or NULL
+};
+
+__device__ __forceinline__ float dot8(const uint4 x, const float *u)
+{
+    float a = bf_lo(x.x) * u[0];
+    a = fmaf(bf_hi(x.x), u[1], a);
+    a = fmaf(bf_lo(x.y), u[2], a);
+    a = fmaf(bf_hi(x.y), u[3], a);
+    a = fmaf(bf_lo(x.z), u[4], a);
+    a = fmaf(bf_hi(x.z), u[5], a);
+    a = fmaf(bf_lo(x.w), u[6], a);
+    a = fmaf(bf_hi(x.w), u[7], a);
+    return a;
+}
+
+__global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const CondenseArgs a)
+{
+    extern __shared__ __align__(128) uint8_t cd_smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *ring = cd_smem + size_t(warp) * CD_SLOTS * CD_GROUP_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(cd_smem + CD_WARPS * CD_SLOTS * CD_GROUP_BYTES) +
+                     warp * CD_SLOTS;
+    if (lane == 0) {
+        for (int s = 0; s < CD_SLOTS; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    const int64_t nw = int64_t(gridDim.x) * CD_WARPS;
+    const int64_t gw = int64_t(blockIdx.x) * CD_WARPS + warp;
+    const uint64_t pol = policy_evict_first();
+
+    auto issue = [&](int64_t gi, int s) {
+        const int64_t b = gi / a.m, j = gi - b * a.m;
+        const uint16_t *src = a.cache + (size_t(b) * a.L + size_t(j) * 16) * LCA_D;
+        const uint32_t bar = smem_u32(&bars[s]);
+        mbar_expect_tx(bar, CD_GROUP_BYTES);
+        bulk_load(smem_u32(ring + s * CD_GROUP_BYTES), src, CD_GROUP_BYTES, bar, pol);
+    };
+
+    int issued_last[CD_SLOTS] = {-1, -1, -1};
+    if (lane == 0) {
+        for (int s = 0; s < CD_SLOTS; ++s) {
+            const int64_t gi = gw + s * nw;
+            if (gi < a.total) {
+                issue(gi, s);
+                issued_last[s] = s;
+            }
+        }
+    }
+
+    bool ok = true;
+    int it = 0;
+    for (int64_t gi = gw; gi < a.total; gi += nw, ++it) {
+        const int s = it % CD_SLOTS;
+        ok = mbar_wait(smem_u32(&bars[s]), (it / CD_SLOTS) & 1, nullptr, K_CONDENSE, 1);
+        if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+        }
+        const int64_t b = gi / a.m, j = gi - b * a.m;
+        const uint8_t *tile = ring + s * CD_GROUP_BYTES;
+
+        // importance: partial dots over this lane's 16-byte column slices
+        // (lane, lane+32 and, for lanes < 8, lane+64 of the 72 slices)
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll 1
+        for (int r = 0; r < 3; ++r) {
+            const int v = lane + 32 * r;
+            if (v < 72) {
+                const float4 *up = reinterpret_cast<const float4 *>(a.u + size_t(b) * LCA_D + 8 * v);
+                const float4 x0 = __ldg(up), x1 = __ldg(up + 1);
+                const float uu[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    acc[i] += dot8(*reinterpret_cast<const uint4 *>(tile + i * (LCA_D * 2) + v * 16), uu);
+            }
+        }
+        // halving transpose-reduce: after it lanes 2t and 2t+1 hold token t
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const bool up = lane & 16;
+            const float send = up ? acc[k] : acc[k + 8];
+            const float keep = up ? acc[k + 8] : acc[k];
+            acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const bool up = lane & 8;
+            const float send = up ? acc[k] : acc[k + 4];
+            const float keep = up ? acc[k + 4] : acc[k];
+            acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const bool up = lane & 4;
+            const float send = up ? acc[k] : acc[k + 2];
+            const float keep = up ? acc[k + 2] : acc[k];
+            acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        }
+        {
+            const bool up = lane & 2;
+            const float send = up ? acc[0] : acc[1];
+            const float keep = up ? acc[1] : acc[0];
+            acc[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        }
+        const float sc = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 1);
+        const int tok = lane >> 1;
+
+        // group max and first-index argmax
+        float best = sc;
+        int bi = tok;
+#pragma unroll
+        for (int off = 2; off <= 16; off <<= 1) {
+            const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ob > best || (ob == best && oi < bi)) {
+                best = ob;
+                bi = oi;
+            }
+        }
+        const float e = fast_exp2((sc - best) * kLog2e);
+        float den = e;
+#pragma unroll
+        for (int off = 2; off <= 16; off <<= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+        const float al = e / den;
+
+        // pooled latent: lane owns 16-byte slices lane and lane+32 of c
+        float pa[2][8];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) pa[r][k] = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const float ai = __shfl_sync(0xffffffffu, al, 2 * i);
+            const uint8_t *row = tile + i * (LCA_D * 2);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(row + (lane + 32 * r) * 16);
+                pa[r][0] = fmaf(ai, bf_lo(x.x), pa[r][0]);
+                pa[r][1] = fmaf(ai, bf_hi(x.x), pa[r][1]);
+                pa[r][2] = fmaf(ai, bf_lo(x.y), pa[r][2]);
+                pa[r][3] = fmaf(ai, bf_hi(x.y), pa[r][3]);
+                pa[r][4] = fmaf(ai, bf_lo(x.z), pa[r][4]);
+                pa[r][5] = fmaf(ai, bf_hi(x.z), pa[r][5]);
+                pa[r][6] = fmaf(ai, bf_lo(x.w), pa[r][6]);
+                pa[r][7] = fmaf(ai, bf_hi(x.w), pa[r][7]);
+            }
+        }
+        uint16_t *dst = a.rep + (size_t(b) * a.m + size_t(j)) * LCA_D;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            uint4 o;
+            o.x = pack_bf16(pa[r][0], pa[r][1]);
+            o.y = pack_bf16(pa[r][2], pa[r][3]);
+            o.z = pack_bf16(pa[r][4], pa[r][5]);
+            o.w = pack_bf16(pa[r][6], pa[r][7]);
+            reinterpret_cast<uint4 *>(dst)[lane + 32 * r] = o;
+        }
+        if (lane < 8) {
+            const uint4 k = *reinterpret_cast<const uint4 *>(tile + bi * (LCA_D * 2) + LCA_DC * 2 + lane * 16);
+            reinterpret_cast<uint4 *>(dst + LCA_DC)[lane] = k;
+        }
+        const size_t gidx = size_t(b) * a.m + size_t(j);
+        if (a.anchor && lane == 0) a.anchor[gidx] = int32_t(j * 16 + bi);
+        if (a.alpha && (lane & 1) == 0) a.alpha[gidx * 16 + tok] = al;
+
+        // release the slot and refill it
+        __syncwarp();
+        if (lane == 0) {
+            const int64_t nxt = gi + CD_SLOTS * nw;
+            if (nxt < a.total) {
+                fence_proxy_async();
+                issue(nxt, s);
+                issued_last[s] = it + CD_SLOTS;
+            }
+        }
+    }
+    if (!ok && lane == 0) {
+        // a wait expired: let every copy already issued land before exiting
+        for (int s = 0; s < CD_SLOTS; ++s)
+            if (issued_last[s] >= 0)
+                mbar_wait(smem_u32(&bars[s]), (issued_last[s] / CD_SLOTS) & 1, nullptr, K_CONDENSE, 2);
+    }
+}
+
+}  // namespace lca

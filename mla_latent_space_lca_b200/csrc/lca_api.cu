@@ -1,0 +1,470 @@
+// lca_api.cu -- the C ABI declared in include/lca.h: argument checks,
+// workspace layout, TMA tensor maps and kernel launches.  All kernels are in
+// this one translation unit (the .cuh files it includes).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lca.h"
+#include "common.cuh"
+#include "prep_combine.cuh"
+#include "condense.cuh"
+#include "attn_decode.cuh"
+#include "wuv_gemm.cuh"
+
+using namespace lca;
+
+namespace {
+
+constexpr int kMaxCtas = 256;      // split-L grid cap; sizes the partial buffers
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ device
+struct DeviceInfo {
+    int sms = 0;
+    bool ok = false;
+    bool attrs_set = false;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+int current_device(DeviceInfo **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LCA_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ok) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return LCA_ERR_NO_DEVICE;
+        if (major != 10 || minor != 0) return LCA_ERR_NO_DEVICE;
+        d.sms = sms;
+        d.ok = true;
+    }
+    if (!d.attrs_set) {
+        bool good = true;
+        good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_MLA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_REPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
+        good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
+        if (!good) return LCA_ERR_CUDA;
+        d.attrs_set = true;
+    }
+    *out = &d;
+    return LCA_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return LCA_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return LCA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return LCA_OK;
+}
+
+// 3-D bf16 map, dims {d0, d1, d2} (d0 innermost), byte strides {s1, s2},
+// box {b0, b1, b2}, 128-byte swizzle, zero fill out of bounds.
+int make_map3(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+              uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2)
+{
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1, s2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LCA_OK : LCA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ timing / counting
+struct ProfRec {
+    cudaEvent_t a, b;
+    int kid;
+};
+const char *kKernelNames[] = {"", "prep_summary", "condense", "attn_decode", "combine", "wuv_gemm", "prefill"};
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof_used;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
+int64_t g_launches = 0;
+
+struct Launch {
+    cudaStream_t st;
+    int kid;
+    ProfRec rec{};
+    bool timed = false;
+    Launch(cudaStream_t s, int k) : st(s), kid(k)
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        ++g_launches;
+        if (!g_prof_on) return;
+        if (g_prof_pool.empty()) {
+            cudaEvent_t x, y;
+            if (cudaEventCreate(&x) != cudaSuccess) return;
+            if (cudaEventCreate(&y) != cudaSuccess) { cudaEventDestroy(x); return; }
+            g_prof_pool.push_back({x, y});
+        }
+        rec.a = g_prof_pool.back().first;
+        rec.b = g_prof_pool.back().second;
+        g_prof_pool.pop_back();
+        rec.kid = k;
+        timed = cudaEventRecord(rec.a, st) == cudaSuccess;
+    }
+    int done()
+    {
+        const cudaError_t e = cudaGetLastError();
+        if (timed) {
+            cudaEventRecord(rec.b, st);
+            std::lock_guard<std::mutex> lk(g_mu);
+            g_prof_used.push_back(rec);
+        }
+        return e == cudaSuccess ? LCA_OK : LCA_ERR_CUDA;
+    }
+};
+
+// ------------------------------------------------------------------ workspace
+struct DecodeWs {
+    float *u;
+    uint16_t *uhl;
+    float *part_o;
+    float *part_ml;
+    uint16_t *o_bf16;
+    size_t bytes;
+};
+
+DecodeWs decode_ws_layout(void *ws, int B)
+{
+    DecodeWs w{};
+    const size_t slots = size_t(kMaxCtas) + size_t(B);
+    size_t off[6];
+    off[0] = 0;
+    off[1] = off[0] + align_up(size_t(B) * LCA_D * 4);                 // u
+    off[2] = off[1] + align_up(size_t(B) * 2 * LCA_D * 2);             // uhl
+    off[3] = off[2] + align_up(slots * LCA_HEADS * LCA_DC * 4);         // part_o
+    off[4] = off[3] + align_up(slots * LCA_HEADS * 2 * 4);              // part_ml
+    off[5] = off[4] + align_up(size_t(B) * LCA_HEADS * LCA_DC * 2);     // o_bf16
+    w.bytes = off[5];
+    if (ws) {
+        uint8_t *p = static_cast<uint8_t *>(ws);
+        w.u = reinterpret_cast<float *>(p + off[0]);
+        w.uhl = reinterpret_cast<uint16_t *>(p + off[1]);
+        w.part_o = reinterpret_cast<float *>(p + off[2]);
+        w.part_ml = reinterpret_cast<float *>(p + off[3]);
+        w.o_bf16 = reinterpret_cast<uint16_t *>(p + off[4]);
+    }
+    return w;
+}
+
+bool params_ok(const lca_params &p) { return p.g >= 1 && p.w >= 0 && std::isfinite(p.scale) && p.scale > 0.f; }
+
+int64_t num_groups(int64_t L, const lca_params &p)
+{
+    if (!params_ok(p) || L <= p.w) return 0;
+    return (L - p.w) / p.g;
+}
+
+int check_common(const void *cache, const void *q, const void *w_uv, int B, int64_t L, float *out)
+{
+    if (!cache || !q || !w_uv || !out) return LCA_ERR_INVALID_ARG;
+    if (B < 1 || L < 1 || L >= (int64_t(1) << 31) || int64_t(B) * L >= (int64_t(1) << 40)) return LCA_ERR_INVALID_ARG;
+    if (!aligned16(cache) || !aligned16(q) || !aligned16(w_uv) || !aligned16(out)) return LCA_ERR_MISALIGNED;
+    return LCA_OK;
+}
+
+int check_ws(void *ws, size_t ws_bytes, size_t need)
+{
+    if (!ws || ws_bytes < need) return LCA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return LCA_ERR_MISALIGNED;
+    return LCA_OK;
+}
+
+// Shared tail of the decode paths: split-L attention, combine, W_UV GEMM.
+template <int MODE>
+int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const void *q, const void *w_uv, int B,
+                  int64_t L, int64_t m, int64_t win0, float scale, float *out, float *o_lat, int32_t *anchor,
+                  const DecodeWs &w, cudaStream_t st)
+{
+    int rc = get_encode();
+    if (rc) return rc;
+    AttnArgs a{};
+    a.q = static_cast<const uint16_t *>(q);
+    a.uhl = w.uhl;
+    a.L = L;
+    a.m = m;
+    a.win0 = win0;
+    if (MODE == MODE_MLA) a.n_hist = 0;
+    else if (MODE == MODE_REPS) a.n_hist = int((m + AT_TILE - 1) / AT_TILE);
+    else a.n_hist = int((m + 3) / 4);
+    a.n_tiles = a.n_hist + int((L - win0 + AT_TILE - 1) / AT_TILE);
+    a.T = int64_t(B) * a.n_tiles;
+    a.G = int(std::min<int64_t>(std::min<int64_t>(dev->sms, kMaxCtas), a.T));
+    a.sl2 = scale * 1.4426950408889634f;
+    a.part_o = w.part_o;
+    a.part_ml = w.part_ml;
+    a.anchor = anchor;
+
+    CUtensorMap map_cache, map_rep;
+    rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
+                   uint64_t(L) * LCA_D * 2, 64, AT_TILE, 1);
+    if (rc) return rc;
+    if (MODE == MODE_REPS && m > 0) {
+        rc = make_map3(&map_rep, rep, LCA_D, uint64_t(m), uint64_t(B), uint64_t(LCA_D) * 2,
+                       uint64_t(m) * LCA_D * 2, 64, AT_TILE, 1);
+        if (rc) return rc;
+    } else {
+        map_rep = map_cache;
+    }
+    {
+        Launch l(st, K_ATTN);
+        attn_decode_kernel<MODE><<<a.G, AT_THREADS, AT_SMEM_ALLOC, st>>>(map_cache, map_rep, a);
+        if ((rc = l.done())) return rc;
+    }
+    {
+        Launch l(st, K_COMBINE);
+        combine_kernel<<<dim3(B, LCA_HEADS), 128, 0, st>>>(w.part_o, w.part_ml, a.n_tiles, a.T, a.G, o_lat, w.o_bf16);
+        if ((rc = l.done())) return rc;
+    }
+    CUtensorMap map_a, map_b;
+    rc = make_map3(&map_a, w.o_bf16, LCA_DC, LCA_HEADS, uint64_t(B), LCA_DC * 2, LCA_HEADS * LCA_DC * 2, 64, 1, 128);
+    if (rc) return rc;
+    rc = make_map3(&map_b, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
+    if (rc) return rc;
+    {
+        Launch l(st, K_GEMM);
+        wuv_gemm_kernel<<<dim3((B + 127) / 128, LCA_HEADS), 128, GM_SMEM_ALLOC, st>>>(map_a, map_b, out, B);
+        if ((rc = l.done())) return rc;
+    }
+    return LCA_OK;
+}
+
+int launch_prep(const void *q_recent, int B, const lca_params &p, const DecodeWs &w, cudaStream_t st)
+{
+    Launch l(st, K_PREP);
+    const float coef = p.scale / float(LCA_HEADS * p.g);
+    prep_summary_kernel<<<B, 192, 0, st>>>(static_cast<const uint16_t *>(q_recent), p.g, coef, w.u, w.uhl);
+    return l.done();
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int64_t lca_num_groups(int64_t L, lca_params p) { return num_groups(L, p); }
+
+size_t lca_workspace_bytes(int op, int B, int64_t L, int64_t q_len, lca_params p)
+{
+    (void)L;
+    (void)q_len;
+    if (B < 1) return 0;
+    switch (op) {
+    case LCA_OP_MLA_DECODE:
+    case LCA_OP_DECODE_ATTN:
+    case LCA_OP_DECODE:
+    case LCA_OP_CONDENSE:
+        if (op != LCA_OP_MLA_DECODE && !params_ok(p)) return 0;
+        return decode_ws_layout(nullptr, B).bytes;
+    case LCA_OP_PREFILL:
+        return 0;
+    default:
+        return 0;
+    }
+}
+
+int mla_decode_attn(const void *cache, const void *q, const void *w_uv, int B, int64_t L, float scale, float *out,
+                    float *o_lat, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!std::isfinite(scale) || scale <= 0.f) return LCA_ERR_INVALID_ARG;
+    if (o_lat && !aligned16(o_lat)) return LCA_ERR_MISALIGNED;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, 0, 0, scale, out, o_lat, nullptr, w,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int lca_condense(const void *cache, const void *q_recent, int B, int64_t L, lca_params p, void *rep,
+                 int32_t *anchor, float *alpha, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!cache || !q_recent) return LCA_ERR_INVALID_ARG;
+    if (B < 1 || L < 1 || L >= (int64_t(1) << 31)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    const int64_t m = num_groups(L, p);
+    if (m > 0 && !rep) return LCA_ERR_INVALID_ARG;
+    if (!aligned16(cache) || !aligned16(q_recent) || (rep && !aligned16(rep)) || (alpha && !aligned16(alpha)) ||
+        (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+        return LCA_ERR_MISALIGNED;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    int rc = check_ws(ws, ws_bytes, w.bytes);
+    if (rc) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m == 0) return LCA_OK;
+    if ((rc = launch_prep(q_recent, B, p, w, st))) return rc;
+    CondenseArgs a{};
+    a.cache = static_cast<const uint16_t *>(cache);
+    a.u = w.u;
+    a.L = L;
+    a.m = m;
+    a.total = int64_t(B) * m;
+    a.rep = static_cast<uint16_t *>(rep);
+    a.anchor = anchor;
+    a.alpha = alpha;
+    const int64_t want = (a.total + CD_WARPS - 1) / CD_WARPS;
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(dev->sms, want)));
+    Launch l(st, K_CONDENSE);
+    condense_kernel<<<grid, CD_WARPS * 32, CD_SMEM, st>>>(a);
+    return l.done();
+}
+
+int lca_decode_attn(const void *cache, const void *rep, const void *q, const void *w_uv, int B, int64_t L,
+                    lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    const int64_t m = num_groups(L, p);
+    if (m > 0 && !rep) return LCA_ERR_INVALID_ARG;
+    if ((rep && !aligned16(rep)) || (o_lat && !aligned16(o_lat))) return LCA_ERR_MISALIGNED;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, nullptr, w,
+                                    static_cast<cudaStream_t>(stream));
+}
+
+int lca_decode(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B, int64_t L,
+               lca_params p, float *out, float *o_lat, int32_t *anchor, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.g == 1) return mla_decode_attn(cache, q, w_uv, B, L, p.scale, out, o_lat, ws, ws_bytes, stream);
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    if (!q_recent) return LCA_ERR_INVALID_ARG;
+    if (!aligned16(q_recent) || (o_lat && !aligned16(o_lat)) || (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+        return LCA_ERR_MISALIGNED;
+    const int64_t m = num_groups(L, p);
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m > 0 && (rc = launch_prep(q_recent, B, p, w, st))) return rc;
+    return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, anchor, w, st);
+}
+
+int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L, int64_t q_start,
+                      int64_t q_len, lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes,
+                      void *stream)
+{
+    (void)cache; (void)q; (void)w_uv; (void)B; (void)L; (void)q_start; (void)q_len; (void)p; (void)out;
+    (void)o_lat; (void)ws; (void)ws_bytes; (void)stream;
+    return LCA_ERR_UNSUPPORTED;
+}
+
+const char *lca_strerror(int status)
+{
+    switch (status) {
+    case LCA_OK: return "ok";
+    case LCA_ERR_INVALID_ARG: return "invalid argument";
+    case LCA_ERR_MISALIGNED: return "pointer not aligned (16 bytes; workspace 256)";
+    case LCA_ERR_WORKSPACE: return "workspace missing or too small";
+    case LCA_ERR_UNSUPPORTED: return "parameter not supported by these kernels";
+    case LCA_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case LCA_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    case LCA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    default: return "unknown status";
+    }
+}
+
+int lca_device_status(int clear, int *detail)
+{
+    int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return LCA_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, lca::g_status, sizeof v) != cudaSuccess) return LCA_ERR_CUDA;
+    if (clear) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(lca::g_status, &z, sizeof z) != cudaSuccess) return LCA_ERR_CUDA;
+    }
+    if (detail) *detail = v;
+    return v == 0 ? LCA_OK : LCA_ERR_DEVICE_TIMEOUT;
+}
+
+int lca_profile_enable(int on)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_prof_on = on != 0;
+    return LCA_OK;
+}
+
+int lca_profile_collect(lca_kernel_time *out, int max)
+{
+    std::vector<ProfRec> recs;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        recs.swap(g_prof_used);
+    }
+    lca_kernel_time acc[8];
+    std::memset(acc, 0, sizeof acc);
+    int rc = LCA_OK;
+    for (const ProfRec &r : recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            rc = LCA_ERR_CUDA;
+        acc[r.kid].launches += 1;
+        acc[r.kid].total_ms += ms;
+    }
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        for (const ProfRec &r : recs) g_prof_pool.push_back({r.a, r.b});
+    }
+    if (rc) return rc;
+    int n = 0;
+    for (int k = 1; k < 7 && n < max; ++k) {
+        if (!acc[k].launches) continue;
+        std::snprintf(out[n].name, sizeof out[n].name, "%s", kKernelNames[k]);
+        out[n].launches = acc[k].launches;
+        out[n].total_ms = acc[k].total_ms;
+        ++n;
+    }
+    return n;
+}
+
+int64_t lca_launch_count(void)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_launches;
+}
+
+}  // extern "C"

@@ -17,3 +17,11 @@ def ora():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def lcalib():
+    """The built C-ABI library (compiled here if missing; nvcc cross-compiles)."""
+    from mla_latent_space_lca_b200 import _lib, build
+    build.build()
+    return _lib.lib()

@@ -1,0 +1,103 @@
+"""The C-ABI library loads, exports every entry point include/lca.h declares,
+and rejects invalid arguments on the host before touching the GPU (these
+tests run without a GPU: only argument checks are exercised)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_latent_space_lca_b200 import _lib
+from mla_latent_space_lca_b200._lib import LcaParams
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "lca.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", src)) - {"sizeof"})
+
+
+def test_exports_every_declared_symbol(lcalib):
+    declared = header_functions()
+    assert set(declared) == set(_lib.EXPORTS)
+    for name in declared:
+        assert hasattr(lcalib, name), name
+
+
+def test_num_groups(lcalib, ora):
+    for L, g, w in [(4096, 16, 1024), (32768, 16, 1024), (1039, 16, 1024), (1040, 16, 1024),
+                    (100, 16, 1024), (1 << 20, 16, 1024), (77, 1, 5), (1, 16, 0)]:
+        assert lcalib.lca_num_groups(L, LcaParams(g, w, 0.1)) == ora.num_groups(L, g, w)
+    assert lcalib.lca_num_groups(100, LcaParams(0, 1, 0.1)) == 0
+
+
+def test_workspace_bytes(lcalib):
+    p = LcaParams(16, 1024, 0.07)
+    for op in range(4):
+        n = lcalib.lca_workspace_bytes(op, 32, 32768, 0, p)
+        assert n > 0 and n % 256 == 0
+    assert lcalib.lca_workspace_bytes(0, 0, 32768, 0, p) == 0
+    assert lcalib.lca_workspace_bytes(99, 1, 10, 0, p) == 0
+
+
+def test_strerror(lcalib):
+    for s in range(0, -8, -1):
+        assert _lib.strerror(s)
+    assert "unknown" in _lib.strerror(-100)
+
+
+# fake, never-dereferenced device addresses: argument checks fail first
+A = 0x7F0000000000
+
+
+def call_decode(lcalib, **kw):
+    args = dict(cache=A, q_recent=A, q=A, w_uv=A, B=2, L=4096, p=LcaParams(16, 1024, 0.07),
+                out=A, o_lat=None, anchor=None, ws=A, ws_bytes=1 << 30, stream=None)
+    args.update(kw)
+    return lcalib.lca_decode(args["cache"], args["q_recent"], args["q"], args["w_uv"], args["B"],
+                             args["L"], args["p"], args["out"], args["o_lat"], args["anchor"],
+                             args["ws"], args["ws_bytes"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cache=None), _lib.LCA_ERR_INVALID_ARG),
+    (dict(out=None), _lib.LCA_ERR_INVALID_ARG),
+    (dict(q_recent=None), _lib.LCA_ERR_INVALID_ARG),
+    (dict(B=0), _lib.LCA_ERR_INVALID_ARG),
+    (dict(L=0), _lib.LCA_ERR_INVALID_ARG),
+    (dict(L=1 << 31), _lib.LCA_ERR_INVALID_ARG),
+    (dict(p=LcaParams(16, -1, 0.07)), _lib.LCA_ERR_INVALID_ARG),
+    (dict(p=LcaParams(16, 1024, 0.0)), _lib.LCA_ERR_INVALID_ARG),
+    (dict(p=LcaParams(16, 1024, float("nan"))), _lib.LCA_ERR_INVALID_ARG),
+    (dict(p=LcaParams(8, 1024, 0.07)), _lib.LCA_ERR_UNSUPPORTED),
+    (dict(cache=A + 8), _lib.LCA_ERR_MISALIGNED),
+    (dict(o_lat=A + 4), _lib.LCA_ERR_MISALIGNED),
+    (dict(anchor=A + 2), _lib.LCA_ERR_MISALIGNED),
+    (dict(ws=None), _lib.LCA_ERR_WORKSPACE),
+    (dict(ws_bytes=1024), _lib.LCA_ERR_WORKSPACE),
+    (dict(ws=A + 64), _lib.LCA_ERR_MISALIGNED),
+])
+def test_decode_rejects_bad_arguments(lcalib, kw, status):
+    assert call_decode(lcalib, **kw) == status
+
+
+def test_other_entry_points_reject_bad_arguments(lcalib):
+    p = LcaParams(16, 1024, 0.07)
+    big = 1 << 30
+    assert lcalib.mla_decode_attn(None, A, A, 1, 10, 0.1, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.mla_decode_attn(A, A, A, 1, 10, -1.0, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.mla_decode_attn(A, A, A, 1, 10, 0.1, A, None, A, 10, None) == _lib.LCA_ERR_WORKSPACE
+    assert lcalib.lca_condense(A, A, 1, 4096, LcaParams(4, 1024, 0.1), A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
+    assert lcalib.lca_condense(A, A, 1, 4096, p, None, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.lca_condense(A, A, 1, 4096, p, A + 2, None, None, A, big, None) == _lib.LCA_ERR_MISALIGNED
+    assert lcalib.lca_decode_attn(A, None, A, A, 1, 4096, p, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.lca_decode_attn(A, A, A, A, 1, 4096, p, A, None, A, 16, None) == _lib.LCA_ERR_WORKSPACE
+
+
+def test_valid_call_without_gpu_reports_no_device(lcalib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert call_decode(lcalib) == _lib.LCA_ERR_NO_DEVICE
