@@ -11,12 +11,16 @@
 // Tensor-core formulation (per tile, M=128):
 //   S  [128 x 64]  = A(TMEM, 128 lanes x 576) * rows^T     (tcgen05 TS MMA)
 //     The A operand holds per-lane query rows.  In warp quadrant q (lanes
-//     32q..32q+31) lane r holds:
+//     32q..32q+31) row r (lane 32q+r) holds:
 //       MLA/REPS: r<4: full q of head 4q+r
-//       LCA:      r<4: latent half of q (rope zeroed)  -> X = q_lat . c
-//                 4<=r<8: rope half of q (latent zeroed) -> Y = q_rope . k^R
-//                 r=8,9: hi and lo bf16 parts of the folded summary query u
-//                        -> importance s = u . row   (关键设计 1)
+//       LCA:      r<4:     latent part of q of head 4q+r (rope zeroed) -> X = q_lat . c
+//                 8<=r<12: rope part of q of head 4q+r-8 (latent zeroed) -> Y = q_rope . k^R
+//                 r=4, r=12: hi and lo bf16 parts of the folded summary
+//                        query u -> importance s = u . row   (关键设计 1)
+//       all other rows zero.  S is read back with the 16x256b shape, which
+//       hands thread T rows T/4 and T/4+8 for 16 of the 64 tokens
+//       (8j + 2(T%4) + {0,1}), so X and Y of a head, and u_hi and u_lo, meet
+//       in one thread and every row's tokens are spread over 4 threads.
 //   O^T[512 x 16] += rows_lat^T * P^T                       (tcgen05 SS MMA,
 //     4 x M=128 over d, N = 16 heads, K = 64 rows; A is the same smem tile read
 //     MN-major, so the tile is read from HBM exactly once)
@@ -119,11 +123,11 @@ __device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int qu
         if (lane < 4) {
             src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane) * LCA_D;
             keep_hi = 16;
-        } else if (lane < 8) {
-            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane - 4) * LCA_D;
+        } else if (lane >= 8 && lane < 12) {
+            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane - 8) * LCA_D;
             keep_lo = 16;
-        } else if (lane < 10) {
-            src = a.uhl + (size_t(b) * 2 + (lane - 8)) * LCA_D;
+        } else if (lane == 4 || lane == 12) {
+            src = a.uhl + (size_t(b) * 2 + (lane == 4 ? 0 : 1)) * LCA_D;
         }
     } else {
         if (lane < 4) src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane) * LCA_D;
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         int i = 0, seg = 0;
         int64_t t = t_begin;
         bool ok = true;
-        float m_use = NEG_INF, l_run = 0.f;   // lanes 0..3: head 4*quad + lane
+        float m_use = NEG_INF, l_run = 0.f;   // threads with lane/4 < 4: head 4*quad + lane/4
         while (ok && t < t_end) {
             const int64_t b = t / n_tiles;
             const int64_t seg_end = min64(t_end, (b + 1) * int64_t(n_tiles));
@@ -313,54 +317,90 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 ok = mbar_wait(sfull(sb), (i >> 1) & 1, abort_flag, K_ATTN, 8);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
-                float v[64];
-                tmem_ld64(tmem + lane_base + (sb ? AT_TM_S1 : AT_TM_S0), v);
+                // thread T: rows g = T/4 (lo) and g+8 (hi), tokens
+                // tok(x) = 8*(x>>1) + 2*sub + (x&1), x = 0..15; group of x = x>>2
+                const int g = lane >> 2, sub = lane & 3;
+                float lo[16], hi[16];
+                {
+                    float r[32];
+                    tmem_ld_16x256b_x8(tmem + lane_base + (sb ? AT_TM_S1 : AT_TM_S0), r);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        lo[2 * j] = r[4 * j];
+                        lo[2 * j + 1] = r[4 * j + 1];
+                        hi[2 * j] = r[4 * j + 2];
+                        hi[2 * j + 1] = r[4 * j + 3];
+                    }
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sempty(sb));
 
-                float w[64];        // P^T weights of this lane's head (lanes 0..3)
-                float tmax;
+                float w[16];        // P^T weights of this thread's head and tokens (g < 4)
+                float f = 1.f;      // reference-max rescale factor of this head
                 if (MODE == MODE_LCA && ti.hist) {
-                    // ---- fused condensation of 4 groups (lanes 8/9 = u hi/lo)
-                    float z[4];
+                    // ---- fused condensation of 4 groups; threads g == 4 own u
+                    float al[16];
+                    int anc[4];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float s[16];
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        float sc[4];
 #pragma unroll
-                        for (int kk = 0; kk < 16; ++kk)
-                            s[kk] = v[16 * j + kk] + __shfl_down_sync(0xffffffffu, v[16 * j + kk], 1);
-                        float gm = s[0];
-                        int gi = 0;
+                        for (int e = 0; e < 4; ++e) sc[e] = lo[4 * k4 + e] + hi[4 * k4 + e];
+                        // group max and first-index argmax (token order)
+                        float gm = sc[0];
+                        int gi = 2 * sub;
 #pragma unroll
-                        for (int kk = 1; kk < 16; ++kk)
-                            if (s[kk] > gm) { gm = s[kk]; gi = kk; }
+                        for (int e = 1; e < 4; ++e) {
+                            const int te = 8 * (e >> 1) + 2 * sub + (e & 1);
+                            if (sc[e] > gm) { gm = sc[e]; gi = te; }
+                        }
+#pragma unroll
+                        for (int off = 1; off <= 2; off <<= 1) {
+                            const float og = __shfl_xor_sync(0xffffffffu, gm, off);
+                            const int oi = __shfl_xor_sync(0xffffffffu, gi, off);
+                            if (og > gm || (og == gm && oi < gi)) { gm = og; gi = oi; }
+                        }
                         float den = 0.f;
 #pragma unroll
-                        for (int kk = 0; kk < 16; ++kk) {
-                            s[kk] = fast_exp2((s[kk] - gm) * kLog2e);
-                            den += s[kk];
+                        for (int e = 0; e < 4; ++e) {
+                            sc[e] = fast_exp2((sc[e] - gm) * kLog2e);
+                            den += sc[e];
                         }
+                        den += __shfl_xor_sync(0xffffffffu, den, 1);
+                        den += __shfl_xor_sync(0xffffffffu, den, 2);
                         const float inv = 1.f / den;
 #pragma unroll
-                        for (int kk = 0; kk < 16; ++kk)
-                            w[16 * j + kk] = __shfl_sync(0xffffffffu, s[kk] * inv, 8);   // alpha
-                        const int anc = __shfl_sync(0xffffffffu, gi, 8);
-                        if (a.anchor && quad == 0 && lane == 8 && j < ti.valid)
-                            a.anchor[size_t(b) * a.m + size_t(k) * 4 + j] = int32_t((k * 4 + j) * 16 + gi);
-                        const bool is_y = (lane >= 4 && lane < 8);
-                        float rj = 0.f;
-#pragma unroll
-                        for (int kk = 0; kk < 16; ++kk) {
-                            const float cf = is_y ? (kk == anc ? 1.f : 0.f) : w[16 * j + kk];
-                            rj = fmaf(cf, v[16 * j + kk], rj);
-                        }
-                        const float yj = __shfl_down_sync(0xffffffffu, rj, 4);
-                        z[j] = (j < ti.valid) ? (rj + yj) * a.sl2 : NEG_INF;
+                        for (int e = 0; e < 4; ++e) al[4 * k4 + e] = sc[e] * inv;
+                        anc[k4] = gi;
                     }
-                    tmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
-                    // reference max update (lanes 0..3 own heads)
-                    float f = 1.f;
+                    // alpha of my tokens lives in thread (g=4, same sub)
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) al[x] = __shfl_sync(0xffffffffu, al[x], 16 + sub);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) anc[k4] = __shfl_sync(0xffffffffu, anc[k4], 16);
+                    if (a.anchor && quad == 0 && lane == 0) {
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4)
+                            if (k4 < ti.valid)
+                                a.anchor[size_t(b) * a.m + size_t(k) * 4 + k4] = int32_t((k * 4 + k4) * 16 + anc[k4]);
+                    }
+                    // z_j = scale * (sum_i alpha_i X_i + Y_anchor), summed over the 4 threads of the head
+                    float z[4];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int te = 8 * (e >> 1) + 2 * sub + (e & 1);
+                            acc = fmaf(al[4 * k4 + e], lo[4 * k4 + e], acc);
+                            if (te == anc[k4]) acc += hi[4 * k4 + e];
+                        }
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                        z[k4] = (k4 < ti.valid) ? acc * a.sl2 : NEG_INF;
+                    }
+                    const float tmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
                     if (i == first) {
                         m_use = tmax;
                     } else if (tmax > m_use + 8.f) {
@@ -368,29 +408,27 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         m_use = tmax;
                         l_run *= f;
                     }
-                    if (lane < 4) fsc[(i & 1) * 16 + 4 * quad + lane] = f;
                     float psum = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float p = (j < ti.valid) ? fast_exp2(z[j] - m_use) : 0.f;
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float p = (k4 < ti.valid) ? fast_exp2(z[k4] - m_use) : 0.f;
                         psum += p;
 #pragma unroll
-                        for (int kk = 0; kk < 16; ++kk) w[16 * j + kk] *= p;
+                        for (int e = 0; e < 4; ++e) w[4 * k4 + e] = p * al[4 * k4 + e];
                     }
                     l_run += psum;
                 } else {
-                    // ---- plain rows (MLA, stored reps, window)
-                    if (MODE == MODE_LCA) {
+                    // ---- plain rows (MLA, stored reps, window; LCA adds Y)
+                    float tmax = NEG_INF;
 #pragma unroll
-                        for (int e = 0; e < 64; ++e) v[e] += __shfl_down_sync(0xffffffffu, v[e], 4);
+                    for (int x = 0; x < 16; ++x) {
+                        const int tok = 8 * (x >> 1) + 2 * sub + (x & 1);
+                        const float zz = (MODE == MODE_LCA) ? lo[x] + hi[x] : lo[x];
+                        w[x] = (tok < ti.valid) ? zz * a.sl2 : NEG_INF;
+                        tmax = fmaxf(tmax, w[x]);
                     }
-                    tmax = NEG_INF;
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        v[e] = (e < ti.valid) ? v[e] * a.sl2 : NEG_INF;
-                        tmax = fmaxf(tmax, v[e]);
-                    }
-                    float f = 1.f;
+                    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+                    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
                     if (i == first) {
                         m_use = tmax;
                     } else if (tmax > m_use + 8.f) {
@@ -398,31 +436,28 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         m_use = tmax;
                         l_run *= f;
                     }
-                    if (lane < 4) fsc[(i & 1) * 16 + 4 * quad + lane] = f;
                     float psum = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        w[e] = (e < ti.valid) ? fast_exp2(v[e] - m_use) : 0.f;
-                        psum += w[e];
+                    for (int x = 0; x < 16; ++x) {
+                        w[x] = fast_exp2(w[x] - m_use);   // exp2(-inf) = 0 for masked rows
+                        psum += w[x];
                     }
+                    psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+                    psum += __shfl_xor_sync(0xffffffffu, psum, 2);
                     l_run += psum;
                 }
+                if (g < 4 && sub == 0) fsc[(i & 1) * 16 + 4 * quad + g] = f;
 
-                // ---- P^T row of this lane's head into the swizzled buffer
+                // ---- P^T row of this thread's head: token pairs (8j+2sub, +1)
                 ok = mbar_wait(pempty(sb), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 9);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                if (lane < 4) {
-                    const int h = 4 * quad + lane;
+                if (g < 4) {
+                    const int h = 4 * quad + g;
                     uint8_t *prow = smem + AT_OFF_P + sb * AT_PBUF + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint4 o;
-                        o.x = pack_bf16(w[8 * ch + 0], w[8 * ch + 1]);
-                        o.y = pack_bf16(w[8 * ch + 2], w[8 * ch + 3]);
-                        o.z = pack_bf16(w[8 * ch + 4], w[8 * ch + 5]);
-                        o.w = pack_bf16(w[8 * ch + 6], w[8 * ch + 7]);
-                        *reinterpret_cast<uint4 *>(prow + ((ch ^ (h & 7)) << 4)) = o;
-                    }
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint32_t *>(prow + ((j ^ (h & 7)) << 4) + 4 * sub) =
+                            pack_bf16(w[2 * j], w[2 * j + 1]);
                 }
                 fence_proxy_async();
 
@@ -474,8 +509,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 #pragma unroll
                 for (int h = 0; h < 16; ++h) a.part_o[(slot * LCA_HEADS + h) * LCA_DC + d] = o[h];
             }
-            if (lane < 4) {
-                const size_t hh = slot * LCA_HEADS + 4 * quad + lane;
+            if ((lane & 3) == 0 && lane < 16) {
+                const size_t hh = slot * LCA_HEADS + 4 * quad + (lane >> 2);
                 a.part_ml[hh * 2 + 0] = m_use;
                 a.part_ml[hh * 2 + 1] = l_run;
             }

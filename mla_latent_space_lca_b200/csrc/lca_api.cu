@@ -62,6 +62,7 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
         good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(combine_wuv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CW_SMEM_ALLOC) == cudaSuccess;
         if (!good) return LCA_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -105,7 +106,7 @@ struct ProfRec {
     cudaEvent_t a, b;
     int kid;
 };
-const char *kKernelNames[] = {"", "prep_summary", "condense", "attn_decode", "combine", "wuv_gemm", "prefill"};
+const char *kKernelNames[] = {"", "prep_summary", "condense", "attn_decode", "combine_wuv", "wuv_gemm", "prefill"};
 bool g_prof_on = false;
 std::vector<ProfRec> g_prof_used;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
@@ -242,19 +243,13 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
         attn_decode_kernel<MODE><<<a.G, AT_THREADS, AT_SMEM_ALLOC, st>>>(map_cache, map_rep, a);
         if ((rc = l.done())) return rc;
     }
+    CUtensorMap map_w;
+    rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
+    if (rc) return rc;
     {
         Launch l(st, K_COMBINE);
-        combine_kernel<<<dim3(B, LCA_HEADS), 128, 0, st>>>(w.part_o, w.part_ml, a.n_tiles, a.T, a.G, o_lat, w.o_bf16);
-        if ((rc = l.done())) return rc;
-    }
-    CUtensorMap map_a, map_b;
-    rc = make_map3(&map_a, w.o_bf16, LCA_DC, LCA_HEADS, uint64_t(B), LCA_DC * 2, LCA_HEADS * LCA_DC * 2, 64, 1, 128);
-    if (rc) return rc;
-    rc = make_map3(&map_b, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
-    if (rc) return rc;
-    {
-        Launch l(st, K_GEMM);
-        wuv_gemm_kernel<<<dim3((B + 127) / 128, LCA_HEADS), 128, GM_SMEM_ALLOC, st>>>(map_a, map_b, out, B);
+        combine_wuv_kernel<<<dim3(LCA_HEADS, (B + CW_ROWS - 1) / CW_ROWS), 128, CW_SMEM_ALLOC, st>>>(
+            map_w, w.part_o, w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out);
         if ((rc = l.done())) return rc;
     }
     return LCA_OK;
@@ -264,7 +259,7 @@ int launch_prep(const void *q_recent, int B, const lca_params &p, const DecodeWs
 {
     Launch l(st, K_PREP);
     const float coef = p.scale / float(LCA_HEADS * p.g);
-    prep_summary_kernel<<<B, 192, 0, st>>>(static_cast<const uint16_t *>(q_recent), p.g, coef, w.u, w.uhl);
+    prep_summary_kernel<<<dim3(B, LCA_D / 64), 256, 0, st>>>(static_cast<const uint16_t *>(q_recent), p.g, coef, w.u, w.uhl);
     return l.done();
 }
 

@@ -121,4 +121,150 @@ __global__ void __launch_bounds__(128, 1)
     if (warp == 0) tmem_dealloc(tmem, GM_TM_COLS);
 }
 
+
+// ------------------------------------------------------------------------
+// Decode tail, fused: log-sum-exp combine of the split-L partials and the
+// W_UV up-projection in one kernel, swap-AB so the tensor-core M dimension is
+// the 128 output columns:  out^T[128 x nb] = W_UV[h]^T[128 x 512] * o^T[512 x nb].
+// Grid (16 heads, ceil(B/64)); 128 threads.  W_UV[h] (128 KB, MN-major A) is
+// TMA-loaded at entry while the warps combine the partials of their batch
+// rows straight into the K-major B operand in shared memory (bf16).
+constexpr int CW_ROWS = 64;                       // batch rows per CTA
+constexpr int CW_A = LCA_DC * LCA_DV * 2;         // 131072 B: W_UV[h]
+constexpr int CW_BCHUNK = CW_ROWS * 128;          // 8192 B per 64-k chunk
+constexpr int CW_OFF_B = CW_A;
+constexpr int CW_OFF_BAR = CW_OFF_B + 8 * CW_BCHUNK;      // 196608
+constexpr int CW_SMEM = CW_OFF_BAR + 256;
+constexpr int CW_SMEM_ALLOC = CW_SMEM + 1024;
+
+__global__ void __launch_bounds__(128, 1)
+    combine_wuv_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
+                       const float *__restrict__ part_ml, int B, int n_tiles, int64_t T, int G,
+                       float *__restrict__ o_lat, float *__restrict__ out)
+{
+    extern __shared__ uint8_t cw_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(cw_smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x;
+    const int b0 = blockIdx.y * CW_ROWS;
+    const int nb = min(CW_ROWS, B - b0);
+    const int nb16 = (nb + 15) & ~15;
+    const uint32_t wfull = sbase + CW_OFF_BAR, accf = wfull + 8, drain = wfull + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CW_OFF_BAR + 64);
+
+    if (threadIdx.x == 0) {
+        mbar_init(wfull, 1);
+        mbar_init(accf, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&map_w);
+        const uint64_t pol = policy_evict_last();
+        mbar_expect_tx(wfull, CW_A);
+        for (int kc = 0; kc < 8; ++kc)
+            for (int nh = 0; nh < 2; ++nh)
+                tma_load_3d(sbase + kc * 16384 + nh * 8192, &map_w, wfull, 64 * nh, 64 * kc, h, pol);
+    }
+
+    // combine: warp w handles rows w, w+4, ...; lane owns k = 16*lane .. 16*lane+15
+    for (int r = warp; r < nb16; r += 4) {
+        float o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = 0.f;
+        if (r < nb) {
+            const int b = b0 + r;
+            const int c0 = split_owner(int64_t(b) * n_tiles, T, G);
+            const int c1 = split_owner(int64_t(b + 1) * n_tiles - 1, T, G);
+            float M = -INFINITY;
+            for (int c = c0; c <= c1; ++c) M = fmaxf(M, part_ml[(size_t(c + b) * LCA_HEADS + h) * 2]);
+            float den = 0.f;
+            for (int c = c0; c <= c1; ++c) {
+                const size_t sl = size_t(c + b) * LCA_HEADS + h;
+                const float wgt = exp2f(part_ml[sl * 2] - M);
+                den += wgt * part_ml[sl * 2 + 1];
+                const float4 *po = reinterpret_cast<const float4 *>(part_o + sl * LCA_DC + 16 * lane);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 x = po[v];
+                    o[4 * v + 0] = fmaf(wgt, x.x, o[4 * v + 0]);
+                    o[4 * v + 1] = fmaf(wgt, x.y, o[4 * v + 1]);
+                    o[4 * v + 2] = fmaf(wgt, x.z, o[4 * v + 2]);
+                    o[4 * v + 3] = fmaf(wgt, x.w, o[4 * v + 3]);
+                }
+            }
+            const float inv = 1.f / den;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] *= inv;
+            if (o_lat) {
+                float4 *dst = reinterpret_cast<float4 *>(o_lat + (size_t(b) * LCA_HEADS + h) * LCA_DC + 16 * lane);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            }
+        }
+        // K-major SW128 row r of chunk lane/4, 16-byte units 2*(lane%4) and +1
+        uint8_t *rowp = smem + CW_OFF_B + (lane >> 2) * CW_BCHUNK + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+            const int unit = 2 * (lane & 3) + hlf;
+            uint4 pk;
+            pk.x = pack_bf16(o[8 * hlf + 0], o[8 * hlf + 1]);
+            pk.y = pack_bf16(o[8 * hlf + 2], o[8 * hlf + 3]);
+            pk.z = pack_bf16(o[8 * hlf + 4], o[8 * hlf + 5]);
+            pk.w = pack_bf16(o[8 * hlf + 6], o[8 * hlf + 7]);
+            *reinterpret_cast<uint4 *>(rowp + ((unit ^ (r & 7)) << 4)) = pk;
+        }
+    }
+    fence_proxy_async();
+    __syncthreads();
+
+    if (threadIdx.x == 0) {
+        bool ok = mbar_wait(wfull, 0, nullptr, K_GEMM, 11);
+        if (ok) {
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16(128, nb16, 1, 0);
+#pragma unroll 1
+            for (int ks = 0; ks < 32; ++ks) {
+                const int kc = ks >> 2, kk = ks & 3;
+                const uint64_t ad = sdesc_sw128(sbase + kc * 16384 + kk * 2048, 8192, 1024);
+                const uint64_t bd = sdesc_sw128(sbase + CW_OFF_B + kc * CW_BCHUNK + kk * 32, 16, 1024);
+                mma_ss(tmem, ad, bd, idesc, ks ? 1u : 0u);
+            }
+            tc_commit(accf);
+        }
+        tc_commit(drain);
+        mbar_wait(drain, 0, nullptr, K_GEMM, 12);
+    }
+    __syncwarp();
+    bool ok = mbar_wait(accf, 0, nullptr, K_GEMM, 13);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+        tc_fence_after();
+        const int n = 32 * warp + lane;
+        const uint32_t ta = tmem + (uint32_t(32 * warp) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < nb16; c0 += 16) {
+            float v[16];
+            tmem_ld16(ta + c0, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                if (c0 + e < nb) out[(size_t(b0 + c0 + e) * LCA_HEADS + h) * LCA_DV + n] = v[e];
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
 }  // namespace lca
