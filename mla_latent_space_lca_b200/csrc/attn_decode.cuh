@@ -8,8 +8,8 @@
 //   MODE_LCA : raw history rows 0..m*16-1 (4 groups of 16 per tile), condensed
 //              on the fly, then window rows m*16..L-1.
 //
-// Tensor-core formulation (per tile, M=128):
-//   S  [128 x 64]  = A(TMEM, 128 lanes x 576) * rows^T     (tcgen05 TS MMA)
+// Tensor-core formulation (per tile):
+//   S  [64 x 64]  = A(TMEM, 64 lanes x 576) * rows^T        (tcgen05 TS MMA, M=64)
 //     The A operand holds per-lane query rows.  In warp quadrant q (lanes
 //     32q..32q+31) row r (lane 32q+r) holds:
 //       MLA/REPS: r<4: full q of head 4q+r
@@ -32,8 +32,9 @@
 // its value contribution p_hj c_j^rep = sum_i (p_hj alpha_i) c_i is the PV
 // MMA with per-token weights p_hj * alpha_i.
 //
-// Warp roles (192 threads): warps 0-3 softmax / epilogue (one TMEM lane
-// quadrant each), warp 4 MMA issuer, warp 5 TMA producer.  Online softmax
+// Warp roles (224 threads): warps 0-3 softmax / epilogue (one TMEM lane
+// quadrant each), warp 4 issues the S MMAs, warp 5 is the TMA producer,
+// warp 6 issues the PV MMAs.  Online softmax
 // keeps a per-head reference max and rescales O only when the max grows by
 // more than 2^8 (the final normalisation uses the same reference, so the
 // result is exact either way).  Each CTA writes one (O, m, l) partial per
@@ -53,11 +54,11 @@ constexpr uint32_t AT_TM_S0 = 288;               // 64 columns
 constexpr uint32_t AT_TM_S1 = 352;               // 64 columns
 constexpr uint32_t AT_TM_O = 416;                // 4 x 16 columns
 constexpr uint32_t AT_TM_COLS = 512;
-constexpr int AT_THREADS = 192;
+constexpr int AT_THREADS = 224;
 
 constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
-constexpr int AT_NBAR = 19;
+constexpr int AT_NBAR = 20;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
 constexpr int AT_SMEM = AT_OFF_MISC + 256;              // 225792
 constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     auto pfull = [&](int s) { return BAR(10 + s); };
     auto pempty = [&](int s) { return BAR(12 + s); };
     auto fex = [&](int s) { return BAR(17 + s); };
+    const uint32_t drain2 = BAR(19);
     const uint32_t ofull = BAR(14), segready = BAR(15), drain = BAR(16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
@@ -193,6 +195,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         mbar_init(ofull, 1);
         mbar_init(segready, 4);
         mbar_init(drain, 1);
+        mbar_init(drain2, 1);
         mbar_init(fex(0), 4);
         mbar_init(fex(1), 4);
         *abort_flag = 0;
@@ -237,12 +240,40 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 if (last[s] >= 0) mbar_wait(full(s), (last[s] / 3) & 1, nullptr, K_ATTN, 2);
         }
     } else if (warp == 4) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ S issuer
+        // S is M=64: the query rows live in TMEM lanes 0-15 of each quadrant.
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16(128, AT_TILE, 0, 0);
+            constexpr uint32_t IDESC_S = idesc_bf16(64, AT_TILE, 0, 0);
+            int i = 0, seg = 0;
+            for (int64_t t = t_begin; t < t_end; ++t, ++i) {
+                const bool first = (i == 0) || (t % n_tiles == 0);
+                if (first && !mbar_wait(segready, seg++ & 1, abort_flag, K_ATTN, 3)) break;
+                if (!mbar_wait(full(i % 3), (i / 3) & 1, abort_flag, K_ATTN, 4)) break;
+                if (!mbar_wait(sempty(i & 1), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 5)) break;
+                tc_fence_after();
+                const uint32_t stage = sbase + (i % 3) * AT_STAGE;
+                const uint32_t dS = tmem + ((i & 1) ? AT_TM_S1 : AT_TM_S0);
+#pragma unroll 4
+                for (int ks = 0; ks < 36; ++ks) {
+                    const uint64_t bd = sdesc_sw128(stage + (ks >> 2) * AT_CHUNK + (ks & 3) * 32, 16, 1024);
+                    mma_ts(dS, tmem + AT_TM_Q + 8 * ks, bd, IDESC_S, ks > 0 ? 1u : 0u);
+                }
+                tc_commit(sfull(i & 1));
+            }
+            tc_commit(drain);
+            mbar_wait(drain, 0, nullptr, K_ATTN, 6);
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ PV issuer
+        // A separate thread, so its commits track only PV MMAs: a stage is
+        // released as soon as its own PV completes.
+        if (lane == 0) {
             constexpr uint32_t IDESC_PV = idesc_bf16(128, LCA_HEADS, 1, 0);
-            auto issue_pv = [&](int j, bool first_pv) -> bool {
-                if (!mbar_wait(pfull(j & 1), (j >> 1) & 1, abort_flag, K_ATTN, 7)) return false;
+            int j = 0, first_j = 0;
+            for (int64_t t = t_begin; t < t_end; ++t, ++j) {
+                if (j == 0 || t % n_tiles == 0) first_j = j;
+                const bool last = (t + 1 == t_end) || ((t + 1) % n_tiles == 0);
+                if (!mbar_wait(pfull(j & 1), (j >> 1) & 1, abort_flag, K_ATTN, 7)) break;
                 tc_fence_after();
                 const uint32_t stage = sbase + (j % 3) * AT_STAGE;
                 const uint32_t pbuf = sbase + AT_OFF_P + (j & 1) * AT_PBUF;
@@ -252,44 +283,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = sdesc_sw128(stage + 2 * cc * AT_CHUNK + ks * 2048, AT_CHUNK, 1024);
                         const uint64_t bd = sdesc_sw128(pbuf + ks * 32, 16, 1024);
-                        mma_ss(tmem + AT_TM_O + 16 * cc, ad, bd, IDESC_PV, (first_pv && ks == 0) ? 0u : 1u);
+                        mma_ss(tmem + AT_TM_O + 16 * cc, ad, bd, IDESC_PV, (j == first_j && ks == 0) ? 0u : 1u);
                     }
                 }
                 tc_commit(empty(j % 3));
                 tc_commit(pempty(j & 1));
-                return true;
-            };
-            bool ok = true;
-            int i = 0, seg = 0;
-            int64_t t = t_begin;
-            while (ok && t < t_end) {
-                const int64_t b = t / n_tiles;
-                const int64_t seg_end = min64(t_end, (b + 1) * int64_t(n_tiles));
-                if (!mbar_wait(segready, seg & 1, abort_flag, K_ATTN, 3)) { ok = false; break; }
-                tc_fence_after();
-                const int first = i;
-                for (; t < seg_end; ++t, ++i) {
-                    const int s = i % 3, sb = i & 1;
-                    if (!mbar_wait(full(s), (i / 3) & 1, abort_flag, K_ATTN, 4)) { ok = false; break; }
-                    if (!mbar_wait(sempty(sb), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 5)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t stage = sbase + s * AT_STAGE;
-                    const uint32_t dS = tmem + (sb ? AT_TM_S1 : AT_TM_S0);
-#pragma unroll 4
-                    for (int ks = 0; ks < 36; ++ks) {
-                        const uint64_t bd = sdesc_sw128(stage + (ks >> 2) * AT_CHUNK + (ks & 3) * 32, 16, 1024);
-                        mma_ts(dS, tmem + AT_TM_Q + 8 * ks, bd, IDESC_S, ks > 0 ? 1u : 0u);
-                    }
-                    tc_commit(sfull(sb));
-                    if (i > first && !issue_pv(i - 1, i - 1 == first)) { ok = false; break; }
-                }
-                if (!ok) break;
-                if (!issue_pv(i - 1, i - 1 == first)) { ok = false; break; }
-                tc_commit(ofull);
-                ++seg;
+                if (last) tc_commit(ofull);
             }
-            tc_commit(drain);
-            mbar_wait(drain, 0, nullptr, K_ATTN, 6);
+            tc_commit(drain2);
+            mbar_wait(drain2, 0, nullptr, K_ATTN, 13);
         }
     } else {
         // ------------------------------------------------------------ softmax warps

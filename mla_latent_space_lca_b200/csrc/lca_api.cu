@@ -248,7 +248,7 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     if (rc) return rc;
     {
         Launch l(st, K_COMBINE);
-        combine_wuv_kernel<<<dim3(LCA_HEADS, (B + CW_ROWS - 1) / CW_ROWS), 128, CW_SMEM_ALLOC, st>>>(
+        combine_wuv_kernel<<<dim3(LCA_HEADS, (B + CW_ROWS - 1) / CW_ROWS), CW_THREADS, CW_SMEM_ALLOC, st>>>(
             map_w, w.part_o, w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out);
         if ((rc = l.done())) return rc;
     }

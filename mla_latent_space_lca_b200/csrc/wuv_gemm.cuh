@@ -125,19 +125,26 @@ __global__ void __launch_bounds__(128, 1)
 // ------------------------------------------------------------------------
 // Decode tail, fused: log-sum-exp combine of the split-L partials and the
 // W_UV up-projection in one kernel, swap-AB so the tensor-core M dimension is
-// the 128 output columns:  out^T[128 x nb] = W_UV[h]^T[128 x 512] * o^T[512 x nb].
-// Grid (16 heads, ceil(B/64)); 128 threads.  W_UV[h] (128 KB, MN-major A) is
-// TMA-loaded at entry while the warps combine the partials of their batch
-// rows straight into the K-major B operand in shared memory (bf16).
-constexpr int CW_ROWS = 64;                       // batch rows per CTA
+// the 128 output columns:  out^T[128 x 16] = W_UV[h]^T[128 x 512] * o^T[512 x 16]
+// (N = 16: up to 8 batch rows per CTA, the rest zero).  Grid (16 heads,
+// ceil(B/8)); 256 threads.  W_UV[h] (128 KB, MN-major A) is TMA-loaded at
+// entry.  Meanwhile, per batch row, the 8 warps split that row's partial
+// slots (online max/rescale merge inside a warp, then across warps through
+// shared memory) and write the normalised o row as bf16 straight into the
+// K-major B operand.
+constexpr int CW_ROWS = 8;                        // batch rows per CTA
+constexpr int CW_N = 16;                          // MMA N (rows padded)
+constexpr int CW_THREADS = 256;
 constexpr int CW_A = LCA_DC * LCA_DV * 2;         // 131072 B: W_UV[h]
-constexpr int CW_BCHUNK = CW_ROWS * 128;          // 8192 B per 64-k chunk
-constexpr int CW_OFF_B = CW_A;
-constexpr int CW_OFF_BAR = CW_OFF_B + 8 * CW_BCHUNK;      // 196608
+constexpr int CW_BCHUNK = CW_N * 128;             // 2048 B per 64-k chunk
+constexpr int CW_OFF_B = CW_A;                    // 8 chunks = 16 KB
+constexpr int CW_OFF_SCR = CW_OFF_B + 8 * CW_BCHUNK;          // 147456
+constexpr int CW_SCR = 8 * (LCA_DC + 2) * 4;                  // per-warp (o, M, den)
+constexpr int CW_OFF_BAR = CW_OFF_SCR + CW_SCR;
 constexpr int CW_SMEM = CW_OFF_BAR + 256;
 constexpr int CW_SMEM_ALLOC = CW_SMEM + 1024;
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(CW_THREADS, 1)
     combine_wuv_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
                        const float *__restrict__ part_ml, int B, int n_tiles, int64_t T, int G,
                        float *__restrict__ o_lat, float *__restrict__ out)
@@ -150,9 +157,9 @@ __global__ void __launch_bounds__(128, 1)
     const int h = blockIdx.x;
     const int b0 = blockIdx.y * CW_ROWS;
     const int nb = min(CW_ROWS, B - b0);
-    const int nb16 = (nb + 15) & ~15;
     const uint32_t wfull = sbase + CW_OFF_BAR, accf = wfull + 8, drain = wfull + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CW_OFF_BAR + 64);
+    float *scr = reinterpret_cast<float *>(smem + CW_OFF_SCR);   // [8][512 + 2]
 
     if (threadIdx.x == 0) {
         mbar_init(wfull, 1);
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(128, 1)
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(tmem_slot), 64);
+        tmem_alloc(smem_u32(tmem_slot), 32);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -177,62 +184,78 @@ __global__ void __launch_bounds__(128, 1)
                 tma_load_3d(sbase + kc * 16384 + nh * 8192, &map_w, wfull, 64 * nh, 64 * kc, h, pol);
     }
 
-    // combine: warp w handles rows w, w+4, ...; lane owns k = 16*lane .. 16*lane+15
-    for (int r = warp; r < nb16; r += 4) {
-        float o[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] = 0.f;
+    for (int r = 0; r < CW_N; ++r) {
+        float o[2] = {0.f, 0.f};   // merged o for k = 2*threadIdx.x, +1
         if (r < nb) {
             const int b = b0 + r;
             const int c0 = split_owner(int64_t(b) * n_tiles, T, G);
-            const int c1 = split_owner(int64_t(b + 1) * n_tiles - 1, T, G);
-            float M = -INFINITY;
-            for (int c = c0; c <= c1; ++c) M = fmaxf(M, part_ml[(size_t(c + b) * LCA_HEADS + h) * 2]);
-            float den = 0.f;
-            for (int c = c0; c <= c1; ++c) {
-                const size_t sl = size_t(c + b) * LCA_HEADS + h;
-                const float wgt = exp2f(part_ml[sl * 2] - M);
-                den += wgt * part_ml[sl * 2 + 1];
+            const int ns = split_owner(int64_t(b + 1) * n_tiles - 1, T, G) - c0 + 1;
+            float M = -INFINITY, den = 0.f, acc[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+            for (int sidx = warp; sidx < ns; sidx += 8) {
+                const size_t sl = size_t(c0 + sidx + b) * LCA_HEADS + h;
+                const float m = part_ml[sl * 2], l = part_ml[sl * 2 + 1];
                 const float4 *po = reinterpret_cast<const float4 *>(part_o + sl * LCA_DC + 16 * lane);
+                const float4 x0 = po[0], x1 = po[1], x2 = po[2], x3 = po[3];
+                if (m > M) {
+                    const float sc = exp2f(M - m);   // 0 on the first slot
+                    den *= sc;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float4 x = po[v];
-                    o[4 * v + 0] = fmaf(wgt, x.x, o[4 * v + 0]);
-                    o[4 * v + 1] = fmaf(wgt, x.y, o[4 * v + 1]);
-                    o[4 * v + 2] = fmaf(wgt, x.z, o[4 * v + 2]);
-                    o[4 * v + 3] = fmaf(wgt, x.w, o[4 * v + 3]);
+                    for (int e = 0; e < 16; ++e) acc[e] *= sc;
+                    M = m;
                 }
+                const float wgt = exp2f(m - M);
+                den = fmaf(wgt, l, den);
+                const float xs[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                      x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] = fmaf(wgt, xs[e], acc[e]);
             }
-            const float inv = 1.f / den;
+            float *my = scr + warp * (LCA_DC + 2);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] *= inv;
-            if (o_lat) {
-                float4 *dst = reinterpret_cast<float4 *>(o_lat + (size_t(b) * LCA_HEADS + h) * LCA_DC + 16 * lane);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) dst[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+            for (int e = 0; e < 16; ++e) my[16 * lane + e] = acc[e];
+            if (lane == 0) {
+                my[LCA_DC] = M;
+                my[LCA_DC + 1] = den;
             }
-        }
-        // K-major SW128 row r of chunk lane/4, 16-byte units 2*(lane%4) and +1
-        uint8_t *rowp = smem + CW_OFF_B + (lane >> 2) * CW_BCHUNK + (r >> 3) * 1024 + (r & 7) * 128;
+            __syncthreads();
+            float Mt = -INFINITY;
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-            const int unit = 2 * (lane & 3) + hlf;
-            uint4 pk;
-            pk.x = pack_bf16(o[8 * hlf + 0], o[8 * hlf + 1]);
-            pk.y = pack_bf16(o[8 * hlf + 2], o[8 * hlf + 3]);
-            pk.z = pack_bf16(o[8 * hlf + 4], o[8 * hlf + 5]);
-            pk.w = pack_bf16(o[8 * hlf + 6], o[8 * hlf + 7]);
-            *reinterpret_cast<uint4 *>(rowp + ((unit ^ (r & 7)) << 4)) = pk;
+            for (int w8 = 0; w8 < 8; ++w8) Mt = fmaxf(Mt, scr[w8 * (LCA_DC + 2) + LCA_DC]);
+            float dt = 0.f;
+#pragma unroll
+            for (int w8 = 0; w8 < 8; ++w8) {
+                const float *wp = scr + w8 * (LCA_DC + 2);
+                const float Mw = wp[LCA_DC];
+                const float f = (Mw == -INFINITY) ? 0.f : exp2f(Mw - Mt);
+                dt = fmaf(f, wp[LCA_DC + 1], dt);
+                o[0] = fmaf(f, wp[2 * threadIdx.x], o[0]);
+                o[1] = fmaf(f, wp[2 * threadIdx.x + 1], o[1]);
+            }
+            const float inv = 1.f / dt;
+            o[0] *= inv;
+            o[1] *= inv;
+            if (o_lat)
+                *reinterpret_cast<float2 *>(o_lat + (size_t(b) * LCA_HEADS + h) * LCA_DC + 2 * threadIdx.x) =
+                    make_float2(o[0], o[1]);
         }
+        // row r of the K-major SW128 B operand: k = 2*tid -> chunk k/64, byte (k%64)*2
+        {
+            const int k = 2 * threadIdx.x;
+            const int unit = (k & 63) >> 3, within = (k & 7) * 2;
+            uint8_t *rowp = smem + CW_OFF_B + (k >> 6) * CW_BCHUNK + (r >> 3) * 1024 + (r & 7) * 128;
+            *reinterpret_cast<uint32_t *>(rowp + ((unit ^ (r & 7)) << 4) + within) = pack_bf16(o[0], o[1]);
+        }
+        __syncthreads();
     }
     fence_proxy_async();
     __syncthreads();
 
     if (threadIdx.x == 0) {
-        bool ok = mbar_wait(wfull, 0, nullptr, K_GEMM, 11);
-        if (ok) {
+        if (mbar_wait(wfull, 0, nullptr, K_GEMM, 11)) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, nb16, 1, 0);
+            const uint32_t idesc = idesc_bf16(128, CW_N, 1, 0);
 #pragma unroll 1
             for (int ks = 0; ks < 32; ++ks) {
                 const int kc = ks >> 2, kk = ks & 3;
@@ -246,25 +269,23 @@ __global__ void __launch_bounds__(128, 1)
         mbar_wait(drain, 0, nullptr, K_GEMM, 12);
     }
     __syncwarp();
-    bool ok = mbar_wait(accf, 0, nullptr, K_GEMM, 13);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-        tc_fence_after();
-        const int n = 32 * warp + lane;
-        const uint32_t ta = tmem + (uint32_t(32 * warp) << 16);
-#pragma unroll 1
-        for (int c0 = 0; c0 < nb16; c0 += 16) {
+    if (warp < 4) {
+        bool ok = mbar_wait(accf, 0, nullptr, K_GEMM, 13);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            const int n = 32 * warp + lane;
             float v[16];
-            tmem_ld16(ta + c0, v);
+            tmem_ld16(tmem + (uint32_t(32 * warp) << 16), v);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                if (c0 + e < nb) out[(size_t(b0 + c0 + e) * LCA_HEADS + h) * LCA_DV + n] = v[e];
+            for (int e = 0; e < CW_ROWS; ++e)
+                if (e < nb) out[(size_t(b0 + e) * LCA_HEADS + h) * LCA_DV + n] = v[e];
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (warp == 0) tmem_dealloc(tmem, 32);
 }
 
 }  // namespace lca
