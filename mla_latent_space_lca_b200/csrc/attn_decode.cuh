@@ -8,22 +8,28 @@
 //   MODE_LCA : raw history rows 0..m*16-1 (4 groups of 16 per tile), condensed
 //              on the fly, then window rows m*16..L-1.
 //
-// Tensor-core formulation (per tile):
-//   S  [64 x 64]  = A(TMEM, 64 lanes x 576) * rows^T        (tcgen05 TS MMA, M=64)
-//     The A operand holds per-lane query rows.  In warp quadrant q (lanes
-//     32q..32q+31) row r (lane 32q+r) holds:
-//       MLA/REPS: r<4: full q of head 4q+r
-//       LCA:      r<4:     latent part of q of head 4q+r (rope zeroed) -> X = q_lat . c
-//                 8<=r<12: rope part of q of head 4q+r-8 (latent zeroed) -> Y = q_rope . k^R
-//                 r=4, r=12: hi and lo bf16 parts of the folded summary
-//                        query u -> importance s = u . row   (关键设计 1)
-//       all other rows zero.  S is read back with the 16x256b shape, which
-//       hands thread T rows T/4 and T/4+8 for 16 of the 64 tokens
-//       (8j + 2(T%4) + {0,1}), so X and Y of a head, and u_hi and u_lo, meet
-//       in one thread and every row's tokens are spread over 4 threads.
-//   O^T[512 x 16] += rows_lat^T * P^T                       (tcgen05 SS MMA,
-//     4 x M=128 over d, N = 16 heads, K = 64 rows; A is the same smem tile read
-//     MN-major, so the tile is read from HBM exactly once)
+// Tensor-core formulation (per tile).  A tcgen05.mma chain issued by one
+// thread runs at ~one instruction per ~120 cycles whatever its shape, while
+// chains issued by different threads overlap, so the work is split into
+// independent chains, each with its own issuing thread and accumulator:
+//   S_j [128 x 64] = A_j(TMEM) * rows[:, 288j : 288j+288]^T,  j = 0, 1
+//     (two K-halves of the 576-wide row, 18 k-steps each, TS MMA)
+//   O^T[128c..128c+127, 16] += rows_lat[:, 128c..]^T * P^T,  c = 0..3
+//     (two PV issuers, two d-chunks each; A is the same smem tile read
+//     MN-major, so each tile is read from HBM exactly once)
+// The A operand (TMEM, 144 columns = 288 bf16) holds per-lane query rows.
+// In warp quadrant q (lanes 32q..32q+31), row r (h = 4q + r%8):
+//   MLA/REPS: r<4: q_h[0:288]        8<=r<12: q_h[288:576]
+//   LCA:      r<4: q_h[0:288]        8<=r<12: [q_h[288:512] | 0]     -> X = q_lat . c
+//             24<=r<28: [0 | q_h[512:576]]                           -> Y = q_rope . k^R
+//             r=4, 12: u_hi halves   r=20, 28: u_lo halves  (folded summary
+//             query u = hi + lo in bf16)                   -> s = u . row  (关键设计 1)
+//   all other rows zero.  S_0 and S_1 are read back with the 16x256b shape
+//   at lane offsets 0 and 16; thread T (g = T/4) receives rows g, g+8,
+//   16+g, 24+g for 16 of the 64 tokens (8j + 2(T%4) + {0,1}), so
+//     lo = S_0[g] + S_1[8+g]     (X, the full MLA logit, or u_hi . row)
+//     hi = S_0[16+g] + S_1[24+g] (Y, 0, or u_lo . row)
+//   land in one thread, and every row's tokens are spread over 4 threads.
 // For an LCA history tile, with alpha the group softmax of s and I_j the
 // group argmax, the logit of representative j for head h is
 //   z_hj = scale * (sum_{i in G_j} alpha_i X_hi + Y_h,I_j)
@@ -32,9 +38,9 @@
 // its value contribution p_hj c_j^rep = sum_i (p_hj alpha_i) c_i is the PV
 // MMA with per-token weights p_hj * alpha_i.
 //
-// Warp roles (224 threads): warps 0-3 softmax / epilogue (one TMEM lane
-// quadrant each), warp 4 issues the S MMAs, warp 5 is the TMA producer,
-// warp 6 issues the PV MMAs.  Online softmax
+// Warp roles (288 threads): warps 0-3 softmax / epilogue (one TMEM lane
+// quadrant each), warps 4 and 7 issue the two S chains, warp 5 is the TMA
+// producer, warps 6 and 8 issue the PV chains for d-chunks {0,1} and {2,3}.  Online softmax
 // keeps a per-head reference max and rescales O only when the max grows by
 // more than 2^8 (the final normalisation uses the same reference, so the
 // result is exact either way).  Each CTA writes one (O, m, l) partial per
@@ -49,16 +55,15 @@ constexpr int AT_STAGES = 3;
 constexpr int AT_CHUNK = AT_TILE * 128;          // 8192 B: [64 rows x 64 cols] bf16
 constexpr int AT_STAGE = 9 * AT_CHUNK;           // 73728 B
 constexpr int AT_PBUF = LCA_HEADS * 128;         // 2048 B: P^T [16 heads x 64 rows] bf16
-constexpr uint32_t AT_TM_Q = 0;                  // 288 columns (bf16 pairs)
-constexpr uint32_t AT_TM_S0 = 288;               // 64 columns
-constexpr uint32_t AT_TM_S1 = 352;               // 64 columns
+constexpr uint32_t AT_TM_Q = 0;                  // 144 columns (288 bf16 per lane)
+constexpr uint32_t AT_TM_S = 160;                // S[buf][half]: 4 x 64 columns
 constexpr uint32_t AT_TM_O = 416;                // 4 x 16 columns
 constexpr uint32_t AT_TM_COLS = 512;
-constexpr int AT_THREADS = 224;
+constexpr int AT_THREADS = 288;
 
 constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
-constexpr int AT_NBAR = 20;
+constexpr int AT_NBAR = 22;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
 constexpr int AT_SMEM = AT_OFF_MISC + 256;              // 225792
 constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
@@ -112,33 +117,46 @@ __device__ __forceinline__ TileInfo tile_info(const AttnArgs &a, int k)
     return ti;
 }
 
-// Write this lane's 576-wide query row (or zeros) into TMEM columns
-// AT_TM_Q.. of its lane.  See the lane map in the file header.
+// Write this lane's 288-wide query-row half (or zeros) into TMEM columns
+// AT_TM_Q.. of its lane.  See the row map in the file header.
 template <int MODE>
 __device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int quad, int lane,
                                             uint32_t tmem)
 {
-    const uint16_t *src = nullptr;
-    int keep_lo = 0, keep_hi = 18;   // 16-column chunks [keep_lo, keep_hi) are kept
+    const uint16_t *src = nullptr;   // a 576-wide vector
+    int off = 0;                     // first element of the half (0 or 288)
+    int z0 = 0, z1 = 0;              // elements [z0, z1) are zeroed (32-aligned)
+    const int h = 4 * quad + (lane & 3);
     if (MODE == MODE_LCA) {
         if (lane < 4) {
-            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane) * LCA_D;
-            keep_hi = 16;
+            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
         } else if (lane >= 8 && lane < 12) {
-            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane - 8) * LCA_D;
-            keep_lo = 16;
-        } else if (lane == 4 || lane == 12) {
-            src = a.uhl + (size_t(b) * 2 + (lane == 4 ? 0 : 1)) * LCA_D;
+            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
+            off = 288;
+            z0 = LCA_DC; z1 = LCA_D;
+        } else if (lane >= 24 && lane < 28) {
+            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
+            off = 288;
+            z0 = 288; z1 = LCA_DC;
+        } else if (lane == 4 || lane == 12 || lane == 20 || lane == 28) {
+            src = a.uhl + (size_t(b) * 2 + (lane >= 16 ? 1 : 0)) * LCA_D;
+            off = (lane & 8) ? 288 : 0;
         }
     } else {
-        if (lane < 4) src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + lane) * LCA_D;
+        if (lane < 4) {
+            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
+        } else if (lane >= 8 && lane < 12) {
+            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
+            off = 288;
+        }
     }
     const uint32_t base = tmem + (uint32_t(32 * quad) << 16) + AT_TM_Q;
 #pragma unroll 1
-    for (int cc = 0; cc < 18; ++cc) {
+    for (int cc = 0; cc < 9; ++cc) {
         uint32_t r[16];
-        if (src && cc >= keep_lo && cc < keep_hi) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(src + 32 * cc);
+        const int e0 = off + 32 * cc;
+        if (src && !(e0 >= z0 && e0 < z1)) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(src + e0);
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
                 const uint4 x = p[v];
@@ -175,7 +193,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     auto pfull = [&](int s) { return BAR(10 + s); };
     auto pempty = [&](int s) { return BAR(12 + s); };
     auto fex = [&](int s) { return BAR(17 + s); };
-    const uint32_t drain2 = BAR(19);
+    const uint32_t drain2 = BAR(19), drain3 = BAR(20), drain4 = BAR(21);
     const uint32_t ofull = BAR(14), segready = BAR(15), drain = BAR(16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
@@ -184,18 +202,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 3; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(empty(s), 1);
+            mbar_init(empty(s), 2);      // both PV issuers
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(sfull(s), 1);
+            mbar_init(sfull(s), 2);      // both S issuers
             mbar_init(sempty(s), 4);
             mbar_init(pfull(s), 4);
-            mbar_init(pempty(s), 1);
+            mbar_init(pempty(s), 2);     // both PV issuers
         }
-        mbar_init(ofull, 1);
+        mbar_init(ofull, 2);
         mbar_init(segready, 4);
         mbar_init(drain, 1);
         mbar_init(drain2, 1);
+        mbar_init(drain3, 1);
+        mbar_init(drain4, 1);
         mbar_init(fex(0), 4);
         mbar_init(fex(1), 4);
         *abort_flag = 0;
@@ -239,11 +259,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             for (int s = 0; s < 3; ++s)
                 if (last[s] >= 0) mbar_wait(full(s), (last[s] / 3) & 1, nullptr, K_ATTN, 2);
         }
-    } else if (warp == 4) {
-        // ------------------------------------------------------------ S issuer
-        // S is M=64: the query rows live in TMEM lanes 0-15 of each quadrant.
+    } else if (warp == 4 || warp == 7) {
+        // ------------------------------------------------------------ S issuers
+        // warp 4: K-half 0 (row columns 0..287), warp 7: K-half 1 (288..575)
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = idesc_bf16(64, AT_TILE, 0, 0);
+            const int half = (warp == 7) ? 1 : 0;
+            constexpr uint32_t IDESC_S = idesc_bf16(128, AT_TILE, 0, 0);
             int i = 0, seg = 0;
             for (int64_t t = t_begin; t < t_end; ++t, ++i) {
                 const bool first = (i == 0) || (t % n_tiles == 0);
@@ -252,22 +273,25 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 if (!mbar_wait(sempty(i & 1), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 5)) break;
                 tc_fence_after();
                 const uint32_t stage = sbase + (i % 3) * AT_STAGE;
-                const uint32_t dS = tmem + ((i & 1) ? AT_TM_S1 : AT_TM_S0);
-#pragma unroll 4
-                for (int ks = 0; ks < 36; ++ks) {
-                    const uint64_t bd = sdesc_sw128(stage + (ks >> 2) * AT_CHUNK + (ks & 3) * 32, 16, 1024);
+                const uint32_t dS = tmem + AT_TM_S + 64 * (2 * (i & 1) + half);
+#pragma unroll 6
+                for (int ks = 0; ks < 18; ++ks) {
+                    const int kg = 18 * half + ks;
+                    const uint64_t bd = sdesc_sw128(stage + (kg >> 2) * AT_CHUNK + (kg & 3) * 32, 16, 1024);
                     mma_ts(dS, tmem + AT_TM_Q + 8 * ks, bd, IDESC_S, ks > 0 ? 1u : 0u);
                 }
                 tc_commit(sfull(i & 1));
             }
-            tc_commit(drain);
-            mbar_wait(drain, 0, nullptr, K_ATTN, 6);
+            const uint32_t dr = half ? drain3 : drain;
+            tc_commit(dr);
+            mbar_wait(dr, 0, nullptr, K_ATTN, 6);
         }
-    } else if (warp == 6) {
-        // ------------------------------------------------------------ PV issuer
-        // A separate thread, so its commits track only PV MMAs: a stage is
-        // released as soon as its own PV completes.
+    } else if (warp == 6 || warp == 8) {
+        // ------------------------------------------------------------ PV issuers
+        // Separate threads, so their commits track only PV MMAs: a stage is
+        // released as soon as both halves of its PV complete.
         if (lane == 0) {
+            const int c0 = (warp == 8) ? 2 : 0;
             constexpr uint32_t IDESC_PV = idesc_bf16(128, LCA_HEADS, 1, 0);
             int j = 0, first_j = 0;
             for (int64_t t = t_begin; t < t_end; ++t, ++j) {
@@ -278,7 +302,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 const uint32_t stage = sbase + (j % 3) * AT_STAGE;
                 const uint32_t pbuf = sbase + AT_OFF_P + (j & 1) * AT_PBUF;
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
+                for (int cc = c0; cc < c0 + 2; ++cc) {
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = sdesc_sw128(stage + 2 * cc * AT_CHUNK + ks * 2048, AT_CHUNK, 1024);
@@ -290,8 +314,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 tc_commit(pempty(j & 1));
                 if (last) tc_commit(ofull);
             }
-            tc_commit(drain2);
-            mbar_wait(drain2, 0, nullptr, K_ATTN, 13);
+            const uint32_t dr = (warp == 8) ? drain4 : drain2;
+            tc_commit(dr);
+            mbar_wait(dr, 0, nullptr, K_ATTN, 13);
         }
     } else {
         // ------------------------------------------------------------ softmax warps
@@ -324,14 +349,32 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 const int g = lane >> 2, sub = lane & 3;
                 float lo[16], hi[16];
                 {
+                    const uint32_t s0 = tmem + AT_TM_S + 64 * (2 * sb);
+                    const uint32_t s1 = s0 + 64;
                     float r[32];
-                    tmem_ld_16x256b_x8(tmem + lane_base + (sb ? AT_TM_S1 : AT_TM_S0), r);
+                    tmem_ld_16x256b_x8(s0 + lane_base, r);                    // rows g, 8+g of S_0
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         lo[2 * j] = r[4 * j];
                         lo[2 * j + 1] = r[4 * j + 1];
-                        hi[2 * j] = r[4 * j + 2];
-                        hi[2 * j + 1] = r[4 * j + 3];
+                    }
+                    tmem_ld_16x256b_x8(s1 + lane_base, r);                    // rows g, 8+g of S_1
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        lo[2 * j] += r[4 * j + 2];
+                        lo[2 * j + 1] += r[4 * j + 3];
+                    }
+                    tmem_ld_16x256b_x8(s0 + lane_base + (16u << 16), r);      // rows 16+g, 24+g of S_0
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        hi[2 * j] = r[4 * j];
+                        hi[2 * j + 1] = r[4 * j + 1];
+                    }
+                    tmem_ld_16x256b_x8(s1 + lane_base + (16u << 16), r);      // rows 16+g, 24+g of S_1
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        hi[2 * j] += r[4 * j + 2];
+                        hi[2 * j + 1] += r[4 * j + 3];
                     }
                 }
                 tc_fence_before();
