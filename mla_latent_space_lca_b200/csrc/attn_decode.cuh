@@ -44,7 +44,7 @@
 // keeps a per-head reference max and rescales O only when the max grows by
 // more than 2^8 (the final normalisation uses the same reference, so the
 // result is exact either way).  Each CTA writes one (O, m, l) partial per
-// sequence piece it owns; combine_kernel merges them.
+// sequence piece it owns; tail_decode_kernel merges them.
 #pragma once
 #include "common.cuh"
 
@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    griddep_launch_dependents();
 
     const int c = blockIdx.x;
     const int64_t t_begin = split_begin(c, a.T, a.G);
@@ -327,6 +328,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         int64_t t = t_begin;
         bool ok = true;
         float m_use = NEG_INF, l_run = 0.f;   // threads with lane/4 < 4: head 4*quad + lane/4
+        griddep_wait();   // the folded summary query comes from the previous kernel
         while (ok && t < t_end) {
             const int64_t b = t / n_tiles;
             const int64_t seg_end = min64(t_end, (b + 1) * int64_t(n_tiles));

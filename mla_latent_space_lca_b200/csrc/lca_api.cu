@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/lca.h"
@@ -62,7 +63,7 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
         good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
-        good &= cudaFuncSetAttribute(combine_wuv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CW_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(tail_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TD_SMEM_ALLOC) == cudaSuccess;
         if (!good) return LCA_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -145,6 +146,26 @@ struct Launch {
         return e == cudaSuccess ? LCA_OK : LCA_ERR_CUDA;
     }
 };
+
+// Launch with programmatic dependent launch allowed (the kernel may start
+// its prologue while the previous kernel in the stream finishes; it calls
+// griddepcontrol.wait before touching that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                      Args &&...args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ workspace
 struct DecodeWs {
@@ -240,17 +261,21 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     }
     {
         Launch l(st, K_ATTN);
-        attn_decode_kernel<MODE><<<a.G, AT_THREADS, AT_SMEM_ALLOC, st>>>(map_cache, map_rep, a);
-        if ((rc = l.done())) return rc;
+        // after the summary-query kernel (LCA) the attention prologue and its
+        // first cache loads overlap it
+        const cudaError_t e = launch_ex(attn_decode_kernel<MODE>, dim3(a.G), dim3(AT_THREADS), AT_SMEM_ALLOC, st,
+                                        MODE == MODE_LCA && m > 0, map_cache, map_rep, a);
+        if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     CUtensorMap map_w;
     rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
     if (rc) return rc;
     {
         Launch l(st, K_COMBINE);
-        combine_wuv_kernel<<<dim3(LCA_HEADS, (B + CW_ROWS - 1) / CW_ROWS), CW_THREADS, CW_SMEM_ALLOC, st>>>(
-            map_w, w.part_o, w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out);
-        if ((rc = l.done())) return rc;
+        const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + TD_ROWS - 1) / TD_ROWS), dim3(256),
+                                        TD_SMEM_ALLOC, st, true, map_w, (const float *)w.part_o,
+                                        (const float *)w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out);
+        if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     return LCA_OK;
 }
@@ -259,7 +284,9 @@ int launch_prep(const void *q_recent, int B, const lca_params &p, const DecodeWs
 {
     Launch l(st, K_PREP);
     const float coef = p.scale / float(LCA_HEADS * p.g);
-    prep_summary_kernel<<<dim3(B, LCA_D / 64), 256, 0, st>>>(static_cast<const uint16_t *>(q_recent), p.g, coef, w.u, w.uhl);
+    const cudaError_t e = launch_ex(prep_summary_kernel, dim3(B, LCA_D / 64), dim3(PREP_THREADS), 0, st, true,
+                                    static_cast<const uint16_t *>(q_recent), p.g, coef, w.u, w.uhl);
+    if (e != cudaSuccess) return LCA_ERR_CUDA;
     return l.done();
 }
 

@@ -11,37 +11,60 @@ namespace lca {
 
 // u[b][576] fp32 and its bf16 hi/lo split uhl[b][2][576] (u = hi + lo to
 // ~2^-17 relative), used by the tensor-core importance pass.
-// Grid (B, 9): a block sums 64 columns over the g*16 (t, h) query rows with
-// 4 row-slices per column, then combines the slices through shared memory.
-__global__ void __launch_bounds__(256) prep_summary_kernel(const uint16_t *__restrict__ q_recent,
-                                                           int g, float coef, float *__restrict__ u,
-                                                           uint16_t *__restrict__ uhl)
+// Grid (B, 9): a block owns 64 columns of one sequence; its 256 threads are
+// 8 column groups (16-byte loads) x 32 row slices of the g*16 (t, h) query
+// rows, combined through shared memory.
+constexpr int PREP_THREADS = 256;
+
+__global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16_t *__restrict__ q_recent,
+                                                                    int g, float coef, float *__restrict__ u,
+                                                                    uint16_t *__restrict__ uhl)
 {
-    __shared__ float part[4][64];
+    __shared__ float part[32][64 + 1];
     const int b = blockIdx.x;
-    const int col = blockIdx.y * 64 + (threadIdx.x & 63);
-    const int slice = threadIdx.x >> 6;
+    const int cg = threadIdx.x & 7, sl = threadIdx.x >> 3;
+    const int col0 = blockIdx.y * 64 + 8 * cg;
     const int rows = g * LCA_HEADS;
-    const uint16_t *base = q_recent + size_t(b) * rows * LCA_D + col;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int r = slice;
-    for (; r + 12 < rows; r += 16) {
+    const uint16_t *base = q_recent + size_t(b) * rows * LCA_D + col0;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int r0 = sl; r0 < rows; r0 += 32 * 8) {
+        uint4 x[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            acc[e] += __uint_as_float(uint32_t(__ldg(base + size_t(r + 4 * e) * LCA_D)) << 16);
+        for (int e = 0; e < 8; ++e) {
+            const int r = r0 + 32 * e;
+            x[e] = (r < rows) ? __ldg(reinterpret_cast<const uint4 *>(base + size_t(r) * LCA_D))
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            acc[0] += bf_lo(x[e].x); acc[1] += bf_hi(x[e].x);
+            acc[2] += bf_lo(x[e].y); acc[3] += bf_hi(x[e].y);
+            acc[4] += bf_lo(x[e].z); acc[5] += bf_hi(x[e].z);
+            acc[6] += bf_lo(x[e].w); acc[7] += bf_hi(x[e].w);
+        }
     }
-    for (; r < rows; r += 4) acc[0] += __uint_as_float(uint32_t(__ldg(base + size_t(r) * LCA_D)) << 16);
-    part[slice][threadIdx.x & 63] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[sl][8 * cg + e] = acc[e];
     __syncthreads();
-    if (slice == 0) {
+    if (threadIdx.x < 64) {
         const int c = threadIdx.x;
-        const float uu = ((part[0][c] + part[1][c]) + (part[2][c] + part[3][c])) * coef;
+        float t = 0.f;
+#pragma unroll 8
+        for (int k = 0; k < 32; ++k) t += part[k][c];
+        const int col = blockIdx.y * 64 + c;
+        const float uu = t * coef;
         u[size_t(b) * LCA_D + col] = uu;
         const __nv_bfloat16 hi = __float2bfloat16_rn(uu);
         const __nv_bfloat16 lo = __float2bfloat16_rn(uu - __bfloat162float(hi));
         uhl[(size_t(b) * 2 + 0) * LCA_D + col] = __bfloat16_as_ushort(hi);
         uhl[(size_t(b) * 2 + 1) * LCA_D + col] = __bfloat16_as_ushort(lo);
     }
+    // This kernel may overlap the previous step's tail (it reads only its
+    // own inputs); the attention kernel that follows must not start before
+    // that tail has finished reading the split-L partials.
+    griddep_wait();
+    __syncthreads();
+    griddep_launch_dependents();
 }
 
 }  // namespace lca

@@ -124,51 +124,54 @@ __global__ void __launch_bounds__(128, 1)
 
 // ------------------------------------------------------------------------
 // Decode tail, fused: log-sum-exp combine of the split-L partials and the
-// W_UV up-projection in one kernel, swap-AB so the tensor-core M dimension is
-// the 128 output columns:  out^T[128 x 16] = W_UV[h]^T[128 x 512] * o^T[512 x 16]
+// per-head W_UV up-projection, swap-AB so the tensor-core M dimension is the
+// 128 output columns:
+//   out^T[128 x 16] = W_UV[h]^T[128 x 512] * o^T[512 x 16]
 // (N = 16: up to 8 batch rows per CTA, the rest zero).  Grid (16 heads,
-// ceil(B/8)); 256 threads.  W_UV[h] (128 KB, MN-major A) is TMA-loaded at
-// entry.  Meanwhile, per batch row, the 8 warps split that row's partial
-// slots (online max/rescale merge inside a warp, then across warps through
-// shared memory) and write the normalised o row as bf16 straight into the
-// K-major B operand.
-constexpr int CW_ROWS = 8;                        // batch rows per CTA
-constexpr int CW_N = 16;                          // MMA N (rows padded)
-constexpr int CW_THREADS = 256;
-constexpr int CW_A = LCA_DC * LCA_DV * 2;         // 131072 B: W_UV[h]
-constexpr int CW_BCHUNK = CW_N * 128;             // 2048 B per 64-k chunk
-constexpr int CW_OFF_B = CW_A;                    // 8 chunks = 16 KB
-constexpr int CW_OFF_SCR = CW_OFF_B + 8 * CW_BCHUNK;          // 147456
-constexpr int CW_SCR = 8 * (LCA_DC + 2) * 4;                  // per-warp (o, M, den)
-constexpr int CW_OFF_BAR = CW_OFF_SCR + CW_SCR;
-constexpr int CW_SMEM = CW_OFF_BAR + 256;
-constexpr int CW_SMEM_ALLOC = CW_SMEM + 1024;
+// ceil(B/8)), 256 threads.  W_UV[h] (128 KB, MN-major A) is TMA-loaded before
+// waiting on the attention kernel.  Combine: with nb rows, each row gets
+// 8/nb warps (at least one); a warp merges its share of the row's partial
+// slots online (rescaling on a new maximum, lanes own 16 of the 512 columns),
+// and the warps of a row are merged through shared memory into the bf16
+// K-major B operand.  K = 512 runs as four MMA chains of 8 k-steps, each on
+// its own issuing thread and TMEM accumulator; the epilogue sums them.
+constexpr int TD_ROWS = 8;
+constexpr int TD_N = 16;
+constexpr int TD_A = LCA_DC * LCA_DV * 2;               // 131072
+constexpr int TD_BCHUNK = TD_N * 128;                   // 2048 per 64-k chunk
+constexpr int TD_OFF_B = TD_A;                          // 8 chunks = 16 KB
+constexpr int TD_OFF_SCR = TD_OFF_B + 8 * TD_BCHUNK;    // 147456
+constexpr int TD_SCR_STRIDE = LCA_DC + 4;               // floats per warp state
+constexpr int TD_OFF_BAR = TD_OFF_SCR + 8 * TD_SCR_STRIDE * 4;
+constexpr int TD_SMEM = TD_OFF_BAR + 256;
+constexpr int TD_SMEM_ALLOC = TD_SMEM + 1024;
 
-__global__ void __launch_bounds__(CW_THREADS, 1)
-    combine_wuv_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
+__global__ void __launch_bounds__(256, 1)
+    tail_decode_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
                        const float *__restrict__ part_ml, int B, int n_tiles, int64_t T, int G,
                        float *__restrict__ o_lat, float *__restrict__ out)
 {
-    extern __shared__ uint8_t cw_smem_raw[];
+    extern __shared__ uint8_t td_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(cw_smem_raw) + 1023) & ~uintptr_t(1023));
+        (reinterpret_cast<uintptr_t>(td_smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x;
-    const int b0 = blockIdx.y * CW_ROWS;
-    const int nb = min(CW_ROWS, B - b0);
-    const uint32_t wfull = sbase + CW_OFF_BAR, accf = wfull + 8, drain = wfull + 16;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CW_OFF_BAR + 64);
-    float *scr = reinterpret_cast<float *>(smem + CW_OFF_SCR);   // [8][512 + 2]
+    const int b0 = blockIdx.y * TD_ROWS;
+    const int nb = min(TD_ROWS, B - b0);
+    const int wpr = max(1, TD_ROWS / nb);     // warps per row
+    const uint32_t wbar = sbase + TD_OFF_BAR, accf = wbar + 8, drain0 = wbar + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TD_OFF_BAR + 128);
+    float *scr = reinterpret_cast<float *>(smem + TD_OFF_SCR);
 
     if (threadIdx.x == 0) {
-        mbar_init(wfull, 1);
-        mbar_init(accf, 1);
-        mbar_init(drain, 1);
+        mbar_init(wbar, 1);
+        mbar_init(accf, 4);
+        for (int k = 0; k < 4; ++k) mbar_init(drain0 + 8 * k, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(tmem_slot), 32);
+        tmem_alloc(smem_u32(tmem_slot), 64);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -178,114 +181,152 @@ __global__ void __launch_bounds__(CW_THREADS, 1)
     if (threadIdx.x == 0) {
         prefetch_tensormap(&map_w);
         const uint64_t pol = policy_evict_last();
-        mbar_expect_tx(wfull, CW_A);
+        mbar_expect_tx(wbar, TD_A);
         for (int kc = 0; kc < 8; ++kc)
             for (int nh = 0; nh < 2; ++nh)
-                tma_load_3d(sbase + kc * 16384 + nh * 8192, &map_w, wfull, 64 * nh, 64 * kc, h, pol);
+                tma_load_3d(sbase + kc * 16384 + nh * 8192, &map_w, wbar, 64 * nh, 64 * kc, h, pol);
     }
+    griddep_wait();   // the split-L partials come from the attention kernel
+    // Only now may the next kernel (the next step's summary-query fold)
+    // start: the attention kernel that read its output buffer has finished.
+    griddep_launch_dependents();
 
-    for (int r = 0; r < CW_N; ++r) {
-        float o[2] = {0.f, 0.f};   // merged o for k = 2*threadIdx.x, +1
+    // ---- per-warp merge of its share of one row's slots: the (m, l) pairs of
+    // up to 32 slots at a time are read by the lanes, reduced to their max M
+    // and sum, and then the slot vectors are accumulated with independent
+    // loads (no serial rescaling chain).
+    {
+        const int r = warp / wpr, sub = warp % wpr;
+        float M = -INFINITY, den = 0.f, acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         if (r < nb) {
             const int b = b0 + r;
             const int c0 = split_owner(int64_t(b) * n_tiles, T, G);
             const int ns = split_owner(int64_t(b + 1) * n_tiles - 1, T, G) - c0 + 1;
-            float M = -INFINITY, den = 0.f, acc[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-            for (int sidx = warp; sidx < ns; sidx += 8) {
-                const size_t sl = size_t(c0 + sidx + b) * LCA_HEADS + h;
-                const float m = part_ml[sl * 2], l = part_ml[sl * 2 + 1];
-                const float4 *po = reinterpret_cast<const float4 *>(part_o + sl * LCA_DC + 16 * lane);
-                const float4 x0 = po[0], x1 = po[1], x2 = po[2], x3 = po[3];
-                if (m > M) {
-                    const float sc = exp2f(M - m);   // 0 on the first slot
-                    den *= sc;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[e] *= sc;
-                    M = m;
+            const int mine = (ns - sub + wpr - 1) / wpr;   // slots sub, sub+wpr, ...
+            for (int base = 0; base < mine; base += 32) {
+                const int cnt = min(32, mine - base);
+                float m = -INFINITY, l = 0.f;
+                if (lane < cnt) {
+                    const size_t sl = size_t(c0 + sub + wpr * (base + lane) + b) * LCA_HEADS + h;
+                    const float2 ml = *reinterpret_cast<const float2 *>(part_ml + sl * 2);
+                    m = ml.x;
+                    l = ml.y;
                 }
-                const float wgt = exp2f(m - M);
-                den = fmaf(wgt, l, den);
-                const float xs[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
-                                      x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+                float Mc = m;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = fmaf(wgt, xs[e], acc[e]);
-            }
-            float *my = scr + warp * (LCA_DC + 2);
+                for (int off = 16; off; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
+                const float Mn = fmaxf(M, Mc);
+                const float sc = exp2f(M - Mn);   // rescale the earlier chunks (0 at first)
+                den *= sc;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) my[16 * lane + e] = acc[e];
-            if (lane == 0) {
-                my[LCA_DC] = M;
-                my[LCA_DC + 1] = den;
+                for (int e = 0; e < 16; ++e) acc[e] *= sc;
+                M = Mn;
+                const float wl = (lane < cnt) ? exp2f(m - M) : 0.f;
+                float dl = wl * l;
+#pragma unroll
+                for (int off = 16; off; off >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, off);
+                den += dl;
+#pragma unroll 4
+                for (int k = 0; k < cnt; ++k) {
+                    const float wk = __shfl_sync(0xffffffffu, wl, k);
+                    const size_t sl = size_t(c0 + sub + wpr * (base + k) + b) * LCA_HEADS + h;
+                    const float4 *po = reinterpret_cast<const float4 *>(part_o + sl * LCA_DC + 16 * lane);
+                    const float4 x0 = po[0], x1 = po[1], x2 = po[2], x3 = po[3];
+                    acc[0] = fmaf(wk, x0.x, acc[0]); acc[1] = fmaf(wk, x0.y, acc[1]);
+                    acc[2] = fmaf(wk, x0.z, acc[2]); acc[3] = fmaf(wk, x0.w, acc[3]);
+                    acc[4] = fmaf(wk, x1.x, acc[4]); acc[5] = fmaf(wk, x1.y, acc[5]);
+                    acc[6] = fmaf(wk, x1.z, acc[6]); acc[7] = fmaf(wk, x1.w, acc[7]);
+                    acc[8] = fmaf(wk, x2.x, acc[8]); acc[9] = fmaf(wk, x2.y, acc[9]);
+                    acc[10] = fmaf(wk, x2.z, acc[10]); acc[11] = fmaf(wk, x2.w, acc[11]);
+                    acc[12] = fmaf(wk, x3.x, acc[12]); acc[13] = fmaf(wk, x3.y, acc[13]);
+                    acc[14] = fmaf(wk, x3.z, acc[14]); acc[15] = fmaf(wk, x3.w, acc[15]);
+                }
             }
-            __syncthreads();
+        }
+        float *my = scr + warp * TD_SCR_STRIDE;
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<float4 *>(my + 16 * lane + 4 * v) =
+                make_float4(acc[4 * v], acc[4 * v + 1], acc[4 * v + 2], acc[4 * v + 3]);
+        if (lane == 0) {
+            my[LCA_DC] = M;
+            my[LCA_DC + 1] = den;
+        }
+    }
+    __syncthreads();
+    // ---- merge the warps of each row; o -> o_lat (fp32) and the B operand (bf16)
+    for (int r = 0; r < TD_N; ++r) {
+        const int k = 2 * threadIdx.x;   // 256 threads x 2 columns
+        float o0 = 0.f, o1 = 0.f;
+        if (r < nb) {
             float Mt = -INFINITY;
-#pragma unroll
-            for (int w8 = 0; w8 < 8; ++w8) Mt = fmaxf(Mt, scr[w8 * (LCA_DC + 2) + LCA_DC]);
+            for (int w = r * wpr; w < (r + 1) * wpr; ++w) Mt = fmaxf(Mt, scr[w * TD_SCR_STRIDE + LCA_DC]);
             float dt = 0.f;
-#pragma unroll
-            for (int w8 = 0; w8 < 8; ++w8) {
-                const float *wp = scr + w8 * (LCA_DC + 2);
+            for (int w = r * wpr; w < (r + 1) * wpr; ++w) {
+                const float *wp = scr + w * TD_SCR_STRIDE;
                 const float Mw = wp[LCA_DC];
                 const float f = (Mw == -INFINITY) ? 0.f : exp2f(Mw - Mt);
                 dt = fmaf(f, wp[LCA_DC + 1], dt);
-                o[0] = fmaf(f, wp[2 * threadIdx.x], o[0]);
-                o[1] = fmaf(f, wp[2 * threadIdx.x + 1], o[1]);
+                o0 = fmaf(f, wp[k], o0);
+                o1 = fmaf(f, wp[k + 1], o1);
             }
             const float inv = 1.f / dt;
-            o[0] *= inv;
-            o[1] *= inv;
+            o0 *= inv;
+            o1 *= inv;
             if (o_lat)
-                *reinterpret_cast<float2 *>(o_lat + (size_t(b) * LCA_HEADS + h) * LCA_DC + 2 * threadIdx.x) =
-                    make_float2(o[0], o[1]);
+                *reinterpret_cast<float2 *>(o_lat + (size_t(b0 + r) * LCA_HEADS + h) * LCA_DC + k) =
+                    make_float2(o0, o1);
         }
-        // row r of the K-major SW128 B operand: k = 2*tid -> chunk k/64, byte (k%64)*2
-        {
-            const int k = 2 * threadIdx.x;
-            const int unit = (k & 63) >> 3, within = (k & 7) * 2;
-            uint8_t *rowp = smem + CW_OFF_B + (k >> 6) * CW_BCHUNK + (r >> 3) * 1024 + (r & 7) * 128;
-            *reinterpret_cast<uint32_t *>(rowp + ((unit ^ (r & 7)) << 4) + within) = pack_bf16(o[0], o[1]);
-        }
-        __syncthreads();
+        const int unit = (k & 63) >> 3, within = (k & 7) * 2;
+        uint8_t *rowp = smem + TD_OFF_B + (k >> 6) * TD_BCHUNK + (r >> 3) * 1024 + (r & 7) * 128;
+        *reinterpret_cast<uint32_t *>(rowp + ((unit ^ (r & 7)) << 4) + within) = pack_bf16(o0, o1);
     }
     fence_proxy_async();
     __syncthreads();
 
-    if (threadIdx.x == 0) {
-        if (mbar_wait(wfull, 0, nullptr, K_GEMM, 11)) {
+    if (warp >= 4 && lane == 0) {
+        const int j = warp - 4;   // k-chunks 2j, 2j+1
+        if (mbar_wait(wbar, 0, nullptr, K_GEMM, 31)) {
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16(128, CW_N, 1, 0);
-#pragma unroll 1
-            for (int ks = 0; ks < 32; ++ks) {
-                const int kc = ks >> 2, kk = ks & 3;
-                const uint64_t ad = sdesc_sw128(sbase + kc * 16384 + kk * 2048, 8192, 1024);
-                const uint64_t bd = sdesc_sw128(sbase + CW_OFF_B + kc * CW_BCHUNK + kk * 32, 16, 1024);
-                mma_ss(tmem, ad, bd, idesc, ks ? 1u : 0u);
+            const uint32_t idesc = idesc_bf16(128, TD_N, 1, 0);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const int kc = 2 * j + (kk >> 2), ks = kk & 3;
+                const uint64_t ad = sdesc_sw128(sbase + kc * 16384 + ks * 2048, 8192, 1024);
+                const uint64_t bd = sdesc_sw128(sbase + TD_OFF_B + kc * TD_BCHUNK + ks * 32, 16, 1024);
+                mma_ss(tmem + 16 * j, ad, bd, idesc, kk ? 1u : 0u);
             }
             tc_commit(accf);
         }
-        tc_commit(drain);
-        mbar_wait(drain, 0, nullptr, K_GEMM, 12);
+        tc_commit(drain0 + 8 * j);
+        mbar_wait(drain0 + 8 * j, 0, nullptr, K_GEMM, 32);
     }
-    __syncwarp();
     if (warp < 4) {
-        bool ok = mbar_wait(accf, 0, nullptr, K_GEMM, 13);
+        bool ok = mbar_wait(accf, 0, nullptr, K_GEMM, 33);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
             tc_fence_after();
             const int n = 32 * warp + lane;
-            float v[16];
-            tmem_ld16(tmem + (uint32_t(32 * warp) << 16), v);
+            const uint32_t ta = tmem + (uint32_t(32 * warp) << 16);
+            float v[16], p[16];
+            tmem_ld16(ta, v);
+#pragma unroll 1
+            for (int j = 1; j < 4; ++j) {
+                tmem_ld16(ta + 16 * j, p);
 #pragma unroll
-            for (int e = 0; e < CW_ROWS; ++e)
+                for (int e = 0; e < 16; ++e) v[e] += p[e];
+            }
+#pragma unroll
+            for (int e = 0; e < TD_ROWS; ++e)
                 if (e < nb) out[(size_t(b0 + e) * LCA_HEADS + h) * LCA_DV + n] = v[e];
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, 32);
+    if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
 }  // namespace lca
