@@ -12,23 +12,25 @@
 // thread runs at ~one instruction per ~120 cycles whatever its shape, while
 // chains issued by different threads overlap, so the work is split into
 // independent chains, each with its own issuing thread and accumulator:
-//   S_j [128 x 64] = A_j(TMEM) * rows[:, 288j : 288j+288]^T,  j = 0, 1
-//     (two K-halves of the 576-wide row, 18 k-steps each, TS MMA)
+//   S_j [64 x 64] = A(TMEM) * rows[:, 288j : 288j+288]^T,  j = 0, 1
+//     (two K-halves of the 576-wide row, 18 k-steps each, TS MMA, M = 64)
 //   O^T[128c..128c+127, 16] += rows_lat[:, 128c..]^T * P^T,  c = 0..3
-//     (two PV issuers, two d-chunks each; A is the same smem tile read
-//     MN-major, so each tile is read from HBM exactly once)
-// The A operand (TMEM, 144 columns = 288 bf16) holds per-lane query rows.
-// In warp quadrant q (lanes 32q..32q+31), row r (h = 4q + r%8):
-//   MLA/REPS: r<4: q_h[0:288]        8<=r<12: q_h[288:576]
-//   LCA:      r<4: q_h[0:288]        8<=r<12: [q_h[288:512] | 0]     -> X = q_lat . c
-//             24<=r<28: [0 | q_h[512:576]]                           -> Y = q_rope . k^R
-//             r=4, 12: u_hi halves   r=20, 28: u_lo halves  (folded summary
-//             query u = hi + lo in bf16)                   -> s = u . row  (关键设计 1)
-//   all other rows zero.  S_0 and S_1 are read back with the 16x256b shape
-//   at lane offsets 0 and 16; thread T (g = T/4) receives rows g, g+8,
-//   16+g, 24+g for 16 of the 64 tokens (8j + 2(T%4) + {0,1}), so
-//     lo = S_0[g] + S_1[8+g]     (X, the full MLA logit, or u_hi . row)
-//     hi = S_0[16+g] + S_1[24+g] (Y, 0, or u_lo . row)
+//     (four PV chains of 4 k-steps; A is the same smem tile read MN-major,
+//     so each tile is read from HBM exactly once)
+// The A operand (TMEM, 144 columns = 288 bf16) holds per-lane query rows,
+// all in lanes 0-15 of each warp quadrant q, which is exactly the lane set of
+// an M=64 MMA.  Row r = g + 8*half (g = 0..7) holds a 288-element half-row:
+//   MLA/REPS: g<4: q_h[288*half : +288]      (h = 4q + g)          -> F = q . row
+//   LCA:      g<4: half 0: q_h[0:288], half 1: [q_h[288:512] | 0]    -> X = q_lat . c
+//             g=4: u_hi halves,  g=5: u_lo halves (folded summary query
+//                  u = u_hi + u_lo in bf16)                         -> s = u . row (关键设计 1)
+//             g=6: half 1 = [0 | q_rope] of heads 4q (r=6), 4q+2 (r=14),
+//             g=7: the same for heads 4q+1 (r=7), 4q+3 (r=15)        -> Y = q_rope . k^R
+//   everything else zero.  S_0 and S_1 are read back with the 16x256b shape:
+//   thread T (g = T/4) gets rows g and 8+g of both, for 16 of the 64 tokens
+//   (8i + 2(T%4) + {0,1}), so
+//     lo = S_0[g] + S_1[8+g]           (F, X, u_hi . row or u_lo . row)
+//     ya = S_1[g], yb = S_1[8+g]       (g = 6, 7: Y of two heads each)
 //   land in one thread, and every row's tokens are spread over 4 threads.
 // For an LCA history tile, with alpha the group softmax of s and I_j the
 // group argmax, the logit of representative j for head h is
@@ -38,9 +40,9 @@
 // its value contribution p_hj c_j^rep = sum_i (p_hj alpha_i) c_i is the PV
 // MMA with per-token weights p_hj * alpha_i.
 //
-// Warp roles (288 threads): warps 0-3 softmax / epilogue (one TMEM lane
+// Warp roles (352 threads): warps 0-3 softmax / epilogue (one TMEM lane
 // quadrant each), warps 4 and 7 issue the two S chains, warp 5 is the TMA
-// producer, warps 6 and 8 issue the PV chains for d-chunks {0,1} and {2,3}.  Online softmax
+// producer, warps 6, 8, 9, 10 issue the PV chains of d-chunks 0..3.  Online softmax
 // keeps a per-head reference max and rescales O only when the max grows by
 // more than 2^8 (the final normalisation uses the same reference, so the
 // result is exact either way).  Each CTA writes one (O, m, l) partial per
@@ -59,11 +61,11 @@ constexpr uint32_t AT_TM_Q = 0;                  // 144 columns (288 bf16 per la
 constexpr uint32_t AT_TM_S = 160;                // S[buf][half]: 4 x 64 columns
 constexpr uint32_t AT_TM_O = 416;                // 4 x 16 columns
 constexpr uint32_t AT_TM_COLS = 512;
-constexpr int AT_THREADS = 288;
+constexpr int AT_THREADS = 352;
 
 constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
-constexpr int AT_NBAR = 22;
+constexpr int AT_NBAR = 24;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
 constexpr int AT_SMEM = AT_OFF_MISC + 256;              // 225792
 constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
@@ -117,37 +119,29 @@ __device__ __forceinline__ TileInfo tile_info(const AttnArgs &a, int k)
     return ti;
 }
 
-// Write this lane's 288-wide query-row half (or zeros) into TMEM columns
+// Write this lane's 288-wide query half-row (or zeros) into TMEM columns
 // AT_TM_Q.. of its lane.  See the row map in the file header.
 template <int MODE>
 __device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int quad, int lane,
                                             uint32_t tmem)
 {
+    const int g = lane & 7, half = (lane >> 3) & 1;
     const uint16_t *src = nullptr;   // a 576-wide vector
-    int off = 0;                     // first element of the half (0 or 288)
+    int off = 288 * half;            // first element of the half-row
     int z0 = 0, z1 = 0;              // elements [z0, z1) are zeroed (32-aligned)
-    const int h = 4 * quad + (lane & 3);
-    if (MODE == MODE_LCA) {
-        if (lane < 4) {
-            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
-        } else if (lane >= 8 && lane < 12) {
-            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
+    if (lane < 16) {
+        if (g < 4) {
+            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + g) * LCA_D;
+            if (MODE == MODE_LCA) { z0 = LCA_DC; z1 = LCA_D; }   // X: latent only
+        } else if (MODE == MODE_LCA && (g == 4 || g == 5)) {
+            src = a.uhl + (size_t(b) * 2 + (g - 4)) * LCA_D;
+        } else if (MODE == MODE_LCA) {
+            // g = 6, 7: Y rows of heads 4q + (g-6) + 2*half, always the
+            // second half [0 | q_rope] so that S_1 carries q_rope . k^R
+            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + (g - 6) + 2 * half) * LCA_D;
             off = 288;
-            z0 = LCA_DC; z1 = LCA_D;
-        } else if (lane >= 24 && lane < 28) {
-            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
-            off = 288;
-            z0 = 288; z1 = LCA_DC;
-        } else if (lane == 4 || lane == 12 || lane == 20 || lane == 28) {
-            src = a.uhl + (size_t(b) * 2 + (lane >= 16 ? 1 : 0)) * LCA_D;
-            off = (lane & 8) ? 288 : 0;
-        }
-    } else {
-        if (lane < 4) {
-            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
-        } else if (lane >= 8 && lane < 12) {
-            src = a.q + (size_t(b) * LCA_HEADS + h) * LCA_D;
-            off = 288;
+            z0 = 288;
+            z1 = LCA_DC;
         }
     }
     const uint32_t base = tmem + (uint32_t(32 * quad) << 16) + AT_TM_Q;
@@ -193,7 +187,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     auto pfull = [&](int s) { return BAR(10 + s); };
     auto pempty = [&](int s) { return BAR(12 + s); };
     auto fex = [&](int s) { return BAR(17 + s); };
-    const uint32_t drain2 = BAR(19), drain3 = BAR(20), drain4 = BAR(21);
+    const uint32_t drain2 = BAR(19), drain3 = BAR(20), drain4 = BAR(21), drain5 = BAR(22), drain6 = BAR(23);
     const uint32_t ofull = BAR(14), segready = BAR(15), drain = BAR(16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
@@ -202,20 +196,22 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 3; ++s) {
             mbar_init(full(s), 1);
-            mbar_init(empty(s), 2);      // both PV issuers
+            mbar_init(empty(s), 4);      // four PV chains
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(sfull(s), 2);      // both S issuers
+            mbar_init(sfull(s), 2);      // both S chains
             mbar_init(sempty(s), 4);
             mbar_init(pfull(s), 4);
-            mbar_init(pempty(s), 2);     // both PV issuers
+            mbar_init(pempty(s), 4);     // four PV chains
         }
-        mbar_init(ofull, 2);
+        mbar_init(ofull, 4);
         mbar_init(segready, 4);
         mbar_init(drain, 1);
         mbar_init(drain2, 1);
         mbar_init(drain3, 1);
         mbar_init(drain4, 1);
+        mbar_init(drain5, 1);
+        mbar_init(drain6, 1);
         mbar_init(fex(0), 4);
         mbar_init(fex(1), 4);
         *abort_flag = 0;
@@ -265,7 +261,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         // warp 4: K-half 0 (row columns 0..287), warp 7: K-half 1 (288..575)
         if (lane == 0) {
             const int half = (warp == 7) ? 1 : 0;
-            constexpr uint32_t IDESC_S = idesc_bf16(128, AT_TILE, 0, 0);
+            constexpr uint32_t IDESC_S = idesc_bf16(64, AT_TILE, 0, 0);
             int i = 0, seg = 0;
             for (int64_t t = t_begin; t < t_end; ++t, ++i) {
                 const bool first = (i == 0) || (t % n_tiles == 0);
@@ -287,12 +283,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             tc_commit(dr);
             mbar_wait(dr, 0, nullptr, K_ATTN, 6);
         }
-    } else if (warp == 6 || warp == 8) {
-        // ------------------------------------------------------------ PV issuers
-        // Separate threads, so their commits track only PV MMAs: a stage is
-        // released as soon as both halves of its PV complete.
+    } else if (warp == 6 || warp >= 8) {
+        // ------------------------------------------------------------ PV chains
+        // One thread per d-chunk (warps 6, 8, 9, 10 -> chunks 0..3), so each
+        // chain is 4 MMAs long and the commits track only PV MMAs: a stage is
+        // released as soon as the four chunks of its PV complete.
         if (lane == 0) {
-            const int c0 = (warp == 8) ? 2 : 0;
+            const int cc = (warp == 6) ? 0 : warp - 7;
             constexpr uint32_t IDESC_PV = idesc_bf16(128, LCA_HEADS, 1, 0);
             int j = 0, first_j = 0;
             for (int64_t t = t_begin; t < t_end; ++t, ++j) {
@@ -303,19 +300,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 const uint32_t stage = sbase + (j % 3) * AT_STAGE;
                 const uint32_t pbuf = sbase + AT_OFF_P + (j & 1) * AT_PBUF;
 #pragma unroll
-                for (int cc = c0; cc < c0 + 2; ++cc) {
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = sdesc_sw128(stage + 2 * cc * AT_CHUNK + ks * 2048, AT_CHUNK, 1024);
-                        const uint64_t bd = sdesc_sw128(pbuf + ks * 32, 16, 1024);
-                        mma_ss(tmem + AT_TM_O + 16 * cc, ad, bd, IDESC_PV, (j == first_j && ks == 0) ? 0u : 1u);
-                    }
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ad = sdesc_sw128(stage + 2 * cc * AT_CHUNK + ks * 2048, AT_CHUNK, 1024);
+                    const uint64_t bd = sdesc_sw128(pbuf + ks * 32, 16, 1024);
+                    mma_ss(tmem + AT_TM_O + 16 * cc, ad, bd, IDESC_PV, (j == first_j && ks == 0) ? 0u : 1u);
                 }
                 tc_commit(empty(j % 3));
                 tc_commit(pempty(j & 1));
                 if (last) tc_commit(ofull);
             }
-            const uint32_t dr = (warp == 8) ? drain4 : drain2;
+            const uint32_t dr = cc == 0 ? drain2 : cc == 1 ? drain4 : cc == 2 ? drain5 : drain6;
             tc_commit(dr);
             mbar_wait(dr, 0, nullptr, K_ATTN, 13);
         }
@@ -349,34 +343,25 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 // thread T: rows g = T/4 (lo) and g+8 (hi), tokens
                 // tok(x) = 8*(x>>1) + 2*sub + (x&1), x = 0..15; group of x = x>>2
                 const int g = lane >> 2, sub = lane & 3;
-                float lo[16], hi[16];
+                float lo[16], ya[16], yb[16];
                 {
-                    const uint32_t s0 = tmem + AT_TM_S + 64 * (2 * sb);
-                    const uint32_t s1 = s0 + 64;
+                    const uint32_t s0 = tmem + AT_TM_S + 64 * (2 * sb) + lane_base;
                     float r[32];
-                    tmem_ld_16x256b_x8(s0 + lane_base, r);                    // rows g, 8+g of S_0
+                    tmem_ld_16x256b_x8(s0, r);                 // rows g, 8+g of S_0
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         lo[2 * j] = r[4 * j];
                         lo[2 * j + 1] = r[4 * j + 1];
                     }
-                    tmem_ld_16x256b_x8(s1 + lane_base, r);                    // rows g, 8+g of S_1
+                    tmem_ld_16x256b_x8(s0 + 64, r);            // rows g, 8+g of S_1
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         lo[2 * j] += r[4 * j + 2];
                         lo[2 * j + 1] += r[4 * j + 3];
-                    }
-                    tmem_ld_16x256b_x8(s0 + lane_base + (16u << 16), r);      // rows 16+g, 24+g of S_0
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        hi[2 * j] = r[4 * j];
-                        hi[2 * j + 1] = r[4 * j + 1];
-                    }
-                    tmem_ld_16x256b_x8(s1 + lane_base + (16u << 16), r);      // rows 16+g, 24+g of S_1
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        hi[2 * j] += r[4 * j + 2];
-                        hi[2 * j + 1] += r[4 * j + 3];
+                        ya[2 * j] = r[4 * j];
+                        ya[2 * j + 1] = r[4 * j + 1];
+                        yb[2 * j] = r[4 * j + 2];
+                        yb[2 * j + 1] = r[4 * j + 3];
                     }
                 }
                 tc_fence_before();
@@ -390,10 +375,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     float al[16];
                     int anc[4];
 #pragma unroll
+                    for (int x = 0; x < 16; ++x) al[x] = lo[x] + __shfl_down_sync(0xffffffffu, lo[x], 4);
+#pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         float sc[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) sc[e] = lo[4 * k4 + e] + hi[4 * k4 + e];
+                        for (int e = 0; e < 4; ++e) sc[e] = al[4 * k4 + e];
                         // group max and first-index argmax (token order)
                         float gm = sc[0];
                         int gi = 2 * sub;
@@ -421,31 +408,50 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         for (int e = 0; e < 4; ++e) al[4 * k4 + e] = sc[e] * inv;
                         anc[k4] = gi;
                     }
-                    // alpha of my tokens lives in thread (g=4, same sub)
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) al[x] = __shfl_sync(0xffffffffu, al[x], 16 + sub);
+                    // anchors from thread (g=4, sub=0); alpha of my tokens from (g=4, my sub)
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) anc[k4] = __shfl_sync(0xffffffffu, anc[k4], 16);
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) al[x] = __shfl_sync(0xffffffffu, al[x], 16 + sub);
                     if (a.anchor && quad == 0 && lane == 0) {
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4)
                             if (k4 < ti.valid)
                                 a.anchor[size_t(b) * a.m + size_t(k) * 4 + k4] = int32_t((k * 4 + k4) * 16 + anc[k4]);
                     }
-                    // z_j = scale * (sum_i alpha_i X_i + Y_anchor), summed over the 4 threads of the head
-                    float z[4];
+                    // per group: zx = sum alpha X (threads g < 4) and the anchor's
+                    // Y of two heads (threads g = 6, 7), each summed over the 4
+                    // threads of its row
+                    float zx[4], y0[4], y1[4];
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        float acc = 0.f;
+                        float acc = 0.f, a0 = 0.f, a1 = 0.f;
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
+                            const int x = 4 * k4 + e;
                             const int te = 8 * (e >> 1) + 2 * sub + (e & 1);
-                            acc = fmaf(al[4 * k4 + e], lo[4 * k4 + e], acc);
-                            if (te == anc[k4]) acc += hi[4 * k4 + e];
+                            acc = fmaf(al[x], lo[x], acc);
+                            if (te == anc[k4]) { a0 = ya[x]; a1 = yb[x]; }
                         }
                         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                        z[k4] = (k4 < ti.valid) ? acc * a.sl2 : NEG_INF;
+                        a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+                        a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+                        a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+                        a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+                        zx[k4] = acc;
+                        y0[k4] = a0;
+                        y1[k4] = a1;
+                    }
+                    // head 4q+g's Y lives in thread g' = 6 + (g&1): ya for g < 2, yb for g >= 2
+                    const int ysrc = 24 + 4 * (g & 1) + sub;
+                    float z[4];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float v0 = __shfl_sync(0xffffffffu, y0[k4], ysrc);
+                        const float v1 = __shfl_sync(0xffffffffu, y1[k4], ysrc);
+                        const float yv = (g & 2) ? v1 : v0;
+                        z[k4] = (k4 < ti.valid) ? (zx[k4] + yv) * a.sl2 : NEG_INF;
                     }
                     const float tmax = fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3]));
                     if (i == first) {
@@ -466,12 +472,21 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     l_run += psum;
                 } else {
                     // ---- plain rows (MLA, stored reps, window; LCA adds Y)
+                    if (MODE == MODE_LCA) {
+                        // window rows: F = X + Y, Y of head 4q+g from thread 6 + (g&1)
+                        const int ysrc = 24 + 4 * (g & 1) + sub;
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) {
+                            const float v0 = __shfl_sync(0xffffffffu, ya[x], ysrc);
+                            const float v1 = __shfl_sync(0xffffffffu, yb[x], ysrc);
+                            lo[x] += (g & 2) ? v1 : v0;
+                        }
+                    }
                     float tmax = NEG_INF;
 #pragma unroll
                     for (int x = 0; x < 16; ++x) {
                         const int tok = 8 * (x >> 1) + 2 * sub + (x & 1);
-                        const float zz = (MODE == MODE_LCA) ? lo[x] + hi[x] : lo[x];
-                        w[x] = (tok < ti.valid) ? zz * a.sl2 : NEG_INF;
+                        w[x] = (tok < ti.valid) ? lo[x] * a.sl2 : NEG_INF;
                         tmax = fmaxf(tmax, w[x]);
                     }
                     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
