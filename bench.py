@@ -183,6 +183,21 @@ def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0):
     return tok_s, oracle.num_threads(), sample, times
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's time (all ranks call this at the same point)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(rank: int) -> int:
+    """Each rank decodes its own batch (weak scaling): seed = rank."""
+    return rank
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -214,7 +229,7 @@ def run_ours(args, rank, world, local_rank):
     wl = WORKLOADS[args.workload]
     assert wl["kind"] == "decode"
     B, L = wl["B"], wl["L"]
-    inp = make_decode_inputs(B, L, seed=rank)
+    inp = make_decode_inputs(B, L, seed=replica_seed(rank))
     cache, q_recent, q, w_uv = (inp.cache.to(dev), inp.q_recent.to(dev), inp.q.to(dev),
                                 inp.w_uv.to(dev))
     ws = lca.workspace(3, B, L, device=dev)
@@ -249,11 +264,7 @@ def run_ours(args, rank, world, local_rank):
     launches = (lca.launch_count() - n0) / args.steps
     barrier()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     if sampler:
         sampler.stop()
 
@@ -288,11 +299,7 @@ def run_ours(args, rank, world, local_rank):
         h_out.copy_(out, non_blocking=True)
     x1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = x0.elapsed_time(x1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / args.e2e_steps, world, dev)
     rc, detail = lca.device_status(clear=True)
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail:#x})")
