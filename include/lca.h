@@ -68,6 +68,7 @@ extern "C" {
 #define LCA_ERR_CUDA (-5)          /* a CUDA runtime/driver call or launch failed */
 #define LCA_ERR_NO_DEVICE (-6)     /* the current device is not sm_100 */
 #define LCA_ERR_DEVICE_TIMEOUT (-7) /* a kernel's bounded wait expired */
+#define LCA_ERR_SCRATCH_LIMIT (-8) /* problem larger than lca_decode_noalloc's built-in scratch */
 
 /* Condensation parameters.  g: group size (16; g = 1 makes every token its
  * own representative, which is exactly MLA).  w: local window (>= 0).
@@ -150,6 +151,33 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
 int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L,
                       int64_t q_start, int64_t q_len, lca_params p, float *out, float *o_lat,
                       void *ws, size_t ws_bytes, void *stream);
+
+/* lca_decode without any device allocation, for callers that cannot call
+ * cudaMalloc or hand the library a workspace: code running inside a stream
+ * capture or under an allocator that forbids new device memory, plugins that
+ * only receive pre-allocated input and output buffers, and embedded runtimes
+ * with a fixed memory plan.  (The page has no counterpart: this is an
+ * interface convenience, not part of the method.)
+ *
+ * Same arguments and results as lca_decode, minus ws / ws_bytes: the scratch
+ * (summary query, split-L partials) lives in a file-scope device array of
+ * this library, about 8.4 MiB, which every GPU that loads the library keeps
+ * until the process exits.  Limits: 1 <= B <= LCA_NOALLOC_MAX_BATCH,
+ * otherwise LCA_ERR_SCRATCH_LIMIT and nothing is launched; g must be 16
+ * (or 1, which is MLA decode as for lca_decode).
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before capturing a stream.  All calls on a device share the one array:
+ * every byte a call reads is written earlier in the same call (nothing needs
+ * to start at zero), but two calls whose work overlaps on the GPU (different
+ * streams, or host threads racing) corrupt each other's results.  With
+ * kernel timing switched on (lca_profile_enable) the library creates CUDA
+ * event objects; leave it off where that is not allowed. */
+#define LCA_NOALLOC_MAX_BATCH 8
+int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, const void *w_uv,
+                       int B, int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor,
+                       void *stream);
 
 /* Text for a status code (static storage). */
 const char *lca_strerror(int status);

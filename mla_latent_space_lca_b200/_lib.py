@@ -19,13 +19,16 @@ LCA_ERR_UNSUPPORTED = -4
 LCA_ERR_CUDA = -5
 LCA_ERR_NO_DEVICE = -6
 LCA_ERR_DEVICE_TIMEOUT = -7
+LCA_ERR_SCRATCH_LIMIT = -8
+NOALLOC_MAX_BATCH = 8
 
 OP_MLA_DECODE, OP_CONDENSE, OP_DECODE_ATTN, OP_DECODE, OP_PREFILL = range(5)
 
 # every symbol include/lca.h declares
 EXPORTS = ("lca_num_groups", "lca_workspace_bytes", "mla_decode_attn", "lca_condense",
            "lca_decode_attn", "lca_decode", "lca_prefill_block", "lca_strerror",
-           "lca_device_status", "lca_profile_enable", "lca_profile_collect", "lca_launch_count")
+           "lca_device_status", "lca_profile_enable", "lca_profile_collect", "lca_launch_count",
+           "lca_decode_noalloc")
 
 
 class LcaParams(ctypes.Structure):
@@ -67,6 +70,8 @@ def lib():
         L.lca_decode_attn.argtypes = [P, P, P, P, I, I64, LcaParams, P, P, P, SZ, P]
         L.lca_decode.restype = I
         L.lca_decode.argtypes = [P, P, P, P, I, I64, LcaParams, P, P, P, P, SZ, P]
+        L.lca_decode_noalloc.restype = I
+        L.lca_decode_noalloc.argtypes = [P, P, P, P, I, I64, LcaParams, P, P, P, P]
         L.lca_prefill_block.restype = I
         L.lca_prefill_block.argtypes = [P, P, P, I, I64, I64, I64, LcaParams, P, P, P, SZ, P]
         L.lca_strerror.restype = ctypes.c_char_p

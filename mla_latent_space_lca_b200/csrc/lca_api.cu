@@ -290,6 +290,41 @@ int launch_prep(const void *q_recent, int B, const lca_params &p, const DecodeWs
     return l.done();
 }
 
+// ------------------------------------------------------------------ no-allocation decode
+// Scratch for lca_decode_noalloc lives in this module's own device memory, so
+// a caller that cannot allocate (see include/lca.h) never has to.  It is
+// sized for LCA_NOALLOC_MAX_BATCH sequences with the same layout as the
+// caller-provided workspace of lca_decode; every GPU that loads the library
+// keeps this array until the process exits.
+constexpr size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+constexpr size_t noalloc_scratch_bytes(size_t B)
+{
+    return al256(B * LCA_D * 4) + al256(B * 2 * LCA_D * 2) + al256((kMaxCtas + B) * LCA_HEADS * LCA_DC * 4) +
+           al256((kMaxCtas + B) * LCA_HEADS * 2 * 4) + al256(B * LCA_HEADS * LCA_DC * 2);
+}
+constexpr size_t kNoAllocBytes = noalloc_scratch_bytes(LCA_NOALLOC_MAX_BATCH);
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side symbol is only a stand-in and must never be
+// handed to a kernel).
+void *g_noalloc_ptr[64] = {};
+
+int noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LCA_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LCA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LCA_OK;
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -406,6 +441,32 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
     return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, anchor, w, st);
 }
 
+int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B, int64_t L,
+                       lca_params p, float *out, float *o_lat, int32_t *anchor, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (B > LCA_NOALLOC_MAX_BATCH) return LCA_ERR_SCRATCH_LIMIT;
+    if (p.g != 1 && p.g != 16) return LCA_ERR_UNSUPPORTED;
+    if (p.g != 1 && !q_recent) return LCA_ERR_INVALID_ARG;
+    if ((q_recent && !aligned16(q_recent)) || (o_lat && !aligned16(o_lat)) ||
+        (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+        return LCA_ERR_MISALIGNED;
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    const DecodeWs w = decode_ws_layout(scratch, B);
+    if (w.bytes > kNoAllocBytes) return LCA_ERR_SCRATCH_LIMIT;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (p.g == 1)
+        return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, 0, 0, p.scale, out, o_lat, nullptr, w, st);
+    const int64_t m = num_groups(L, p);
+    if (m > 0 && (rc = launch_prep(q_recent, B, p, w, st))) return rc;
+    return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, anchor, w, st);
+}
+
 int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L, int64_t q_start,
                       int64_t q_len, lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes,
                       void *stream)
@@ -426,6 +487,7 @@ const char *lca_strerror(int status)
     case LCA_ERR_CUDA: return "CUDA call or kernel launch failed";
     case LCA_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
     case LCA_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    case LCA_ERR_SCRATCH_LIMIT: return "batch larger than the built-in scratch of lca_decode_noalloc allows";
     default: return "unknown status";
     }
 }
