@@ -140,17 +140,27 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
                size_t ws_bytes, void *stream);
 
 /* Blockwise LCA prefill of query positions [q_start, q_start + q_len) (both
- * multiples of g).  Block k covers t0 = k*g .. t0+g-1; its summary query is
- * the mean of its own g queries; history rows 0 .. m_k*g-1 with
- * m_k = floor((t0 - w)/g) (0 when t0 <= w) are condensed with it; each query
- * t of the block attends [m_k representatives || cache rows m_k*g .. t].
- *   cache [B][L][576] bf16, q [B][L][16][576] bf16 (rows outside the range
- *   are not read), w_uv [16][512][128] bf16
- *   out   [B][q_len][16][128] fp32, o_lat [B][q_len][16][512] fp32 or NULL
- * Requires g == 16. */
+ * multiples of g).  The page reports prefill speed but does not spell out the
+ * procedure; this is its plainest reading.  Block k covers t0 = k*g ..
+ * t0+g-1; its summary query is the mean of its own g queries; history rows
+ * 0 .. m_k*g-1 with m_k = max(0, floor((t0 - w)/g)) are condensed with it
+ * (关键设计 1, 2); each query t of the block attends [m_k representatives ||
+ * cache rows m_k*g .. t] causally (整体框架, 关键设计 3).
+ *   cache  [B][L][576] bf16, q [B][L][16][576] bf16 (the absorbed queries of
+ *          every position; rows outside the range are not read),
+ *   w_uv   [16][512][128] bf16
+ *   out    [B][q_len][16][128] fp32            (required)
+ *   o_lat  [B][q_len][16][512] fp32 or NULL    (attention output before W_UV)
+ *   anchor [B][q_len/g][m_last] int32 or NULL, m_last = m of the range's last
+ *          block: absolute anchor positions of block k's groups j < m_k in
+ *          row (k - q_start/g); the rest of each row is not written.
+ * Representatives are rounded to bf16 like cache rows.  Requires g == 16 and
+ * L <= 2^27.  ws: lca_workspace_bytes(LCA_OP_PREFILL, B, L, q_len, p) bytes
+ * (enough for any q_start; the blocks are processed in chunks of 256 so the
+ * workspace stays near 256 * m_last * 1152 bytes). */
 int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L,
                       int64_t q_start, int64_t q_len, lca_params p, float *out, float *o_lat,
-                      void *ws, size_t ws_bytes, void *stream);
+                      int32_t *anchor, void *ws, size_t ws_bytes, void *stream);
 
 /* lca_decode without any device allocation, for callers that cannot call
  * cudaMalloc or hand the library a workspace: code running inside a stream

@@ -73,7 +73,7 @@ def lib():
         L.lca_decode_noalloc.restype = I
         L.lca_decode_noalloc.argtypes = [P, P, P, P, I, I64, LcaParams, P, P, P, P]
         L.lca_prefill_block.restype = I
-        L.lca_prefill_block.argtypes = [P, P, P, I, I64, I64, I64, LcaParams, P, P, P, SZ, P]
+        L.lca_prefill_block.argtypes = [P, P, P, I, I64, I64, I64, LcaParams, P, P, P, P, SZ, P]
         L.lca_strerror.restype = ctypes.c_char_p
         L.lca_strerror.argtypes = [I]
         L.lca_device_status.restype = I

@@ -127,17 +127,22 @@ def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
 
 
 def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, out=None,
-                      o_lat=None, ws=None, stream=None):
+                      o_lat=None, anchor=None, ws=None, stream=None):
     B, L, _ = cache.shape
     _need(cache, "cache", torch.bfloat16, (B, L, D))
     _need(q, "q", torch.bfloat16, (B, L, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     out = (torch.empty(B, q_len, H, D_V, dtype=torch.float32, device=cache.device)
            if out is None else out)
+    _need(out, "out", torch.float32, (B, q_len, H, D_V))
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, q_len, H, D_C))
+    if anchor is not None:
+        _need(anchor, "anchor", torch.int32)
     ws = workspace(_lib.OP_PREFILL, B, L, q_len, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_prefill_block(_ptr(cache), _ptr(q), _ptr(w_uv), B, L, q_start, q_len,
-                                      _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(ws),
-                                      ws.numel(), _stream(stream))
+                                      _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(anchor),
+                                      _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "lca_prefill_block")
     return out
 

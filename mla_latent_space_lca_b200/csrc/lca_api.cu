@@ -19,6 +19,7 @@
 #include "condense.cuh"
 #include "attn_decode.cuh"
 #include "wuv_gemm.cuh"
+#include "prefill.cuh"
 
 using namespace lca;
 
@@ -64,6 +65,8 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
         good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(tail_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TD_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(condense_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CP_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM_ALLOC) == cudaSuccess;
         if (!good) return LCA_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -107,7 +110,9 @@ struct ProfRec {
     cudaEvent_t a, b;
     int kid;
 };
-const char *kKernelNames[] = {"", "prep_summary", "condense", "attn_decode", "combine_wuv", "wuv_gemm", "prefill"};
+const char *kKernelNames[] = {"",         "prep_summary", "condense",    "attn_decode",
+                               "combine_wuv", "wuv_gemm",  "attn_prefill", "condense_prefill"};
+constexpr int kNumKernelIds = 8;
 bool g_prof_on = false;
 std::vector<ProfRec> g_prof_used;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
@@ -200,6 +205,37 @@ DecodeWs decode_ws_layout(void *ws, int B)
     return w;
 }
 
+// Blockwise prefill: summary queries of every block of the call, then one
+// chunk of at most kPrefillChunk blocks at a time: its packed
+// representatives and its bf16 attention output (the W_UV GEMM's A operand).
+constexpr int64_t kPrefillChunk = 256;
+
+struct PrefillWs {
+    uint16_t *uhl;      // [B * nb][2][576]
+    uint16_t *rep;      // [chunk blocks * m_bound][576]
+    uint16_t *o_bf16;   // [chunk blocks * 16][16][512]
+    size_t bytes;
+};
+
+PrefillWs prefill_ws_layout(void *ws, int B, int64_t nb, int64_t m_bound)
+{
+    PrefillWs w{};
+    const int64_t nbc = std::min<int64_t>(nb, kPrefillChunk);
+    size_t off[4];
+    off[0] = 0;
+    off[1] = off[0] + align_up(size_t(B) * size_t(nb) * 2 * LCA_D * 2);
+    off[2] = off[1] + align_up(size_t(nbc) * size_t(std::max<int64_t>(m_bound, 1)) * LCA_D * 2);
+    off[3] = off[2] + align_up(size_t(nbc) * 16 * LCA_HEADS * LCA_DC * 2);
+    w.bytes = off[3];
+    if (ws) {
+        uint8_t *p = static_cast<uint8_t *>(ws);
+        w.uhl = reinterpret_cast<uint16_t *>(p + off[0]);
+        w.rep = reinterpret_cast<uint16_t *>(p + off[1]);
+        w.o_bf16 = reinterpret_cast<uint16_t *>(p + off[2]);
+    }
+    return w;
+}
+
 bool params_ok(const lca_params &p) { return p.g >= 1 && p.w >= 0 && std::isfinite(p.scale) && p.scale > 0.f; }
 
 int64_t num_groups(int64_t L, const lca_params &p)
@@ -285,7 +321,8 @@ int launch_prep(const void *q_recent, int B, const lca_params &p, const DecodeWs
     Launch l(st, K_PREP);
     const float coef = p.scale / float(LCA_HEADS * p.g);
     const cudaError_t e = launch_ex(prep_summary_kernel, dim3(B, LCA_D / 64), dim3(PREP_THREADS), 0, st, true,
-                                    static_cast<const uint16_t *>(q_recent), p.g, coef, w.u, w.uhl);
+                                    static_cast<const uint16_t *>(q_recent), p.g, 1,
+                                    int64_t(p.g) * LCA_HEADS * LCA_D, coef, w.u, w.uhl);
     if (e != cudaSuccess) return LCA_ERR_CUDA;
     return l.done();
 }
@@ -334,8 +371,6 @@ int64_t lca_num_groups(int64_t L, lca_params p) { return num_groups(L, p); }
 
 size_t lca_workspace_bytes(int op, int B, int64_t L, int64_t q_len, lca_params p)
 {
-    (void)L;
-    (void)q_len;
     if (B < 1) return 0;
     switch (op) {
     case LCA_OP_MLA_DECODE:
@@ -344,8 +379,12 @@ size_t lca_workspace_bytes(int op, int B, int64_t L, int64_t q_len, lca_params p
     case LCA_OP_CONDENSE:
         if (op != LCA_OP_MLA_DECODE && !params_ok(p)) return 0;
         return decode_ws_layout(nullptr, B).bytes;
-    case LCA_OP_PREFILL:
-        return 0;
+    case LCA_OP_PREFILL: {
+        if (!params_ok(p) || p.g != 16 || q_len < 16 || q_len % 16 || L < q_len) return 0;
+        // the representatives of the last block a range inside [0, L) can hold
+        const int cw = (p.w + 15) / 16;
+        return prefill_ws_layout(nullptr, B, q_len / 16, pf_groups(L / 16 - 1, cw)).bytes;
+    }
     default:
         return 0;
     }
@@ -468,12 +507,109 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
 }
 
 int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L, int64_t q_start,
-                      int64_t q_len, lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes,
-                      void *stream)
+                      int64_t q_len, lca_params p, float *out, float *o_lat, int32_t *anchor, void *ws,
+                      size_t ws_bytes, void *stream)
 {
-    (void)cache; (void)q; (void)w_uv; (void)B; (void)L; (void)q_start; (void)q_len; (void)p; (void)out;
-    (void)o_lat; (void)ws; (void)ws_bytes; (void)stream;
-    return LCA_ERR_UNSUPPORTED;
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    if (q_start < 0 || q_len < 0 || q_start % 16 || q_len % 16 || q_start + q_len > L) return LCA_ERR_INVALID_ARG;
+    if (L > (int64_t(1) << 27)) return LCA_ERR_UNSUPPORTED;   // query rows 16 L index a TMA map
+    if ((o_lat && !aligned16(o_lat)) || (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+        return LCA_ERR_MISALIGNED;
+    if (q_len == 0) return LCA_OK;
+    const int cw = (p.w + 15) / 16;
+    const int64_t k0 = q_start / 16, nb = q_len / 16;
+    const int64_t m_ld = pf_groups(k0 + nb - 1, cw);   // groups of the last block: anchor row length
+    const PrefillWs w = prefill_ws_layout(ws, B, nb, m_ld);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    if ((rc = get_encode())) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint16_t *qv = static_cast<const uint16_t *>(q);
+
+    CUtensorMap map_cache, map_q, map_u, map_w;
+    if ((rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
+                        uint64_t(L) * LCA_D * 2, 64, 64, 1)))
+        return rc;
+    if ((rc = make_map3(&map_q, q, LCA_D, uint64_t(L) * LCA_HEADS, uint64_t(B), uint64_t(LCA_D) * 2,
+                        uint64_t(L) * LCA_HEADS * LCA_D * 2, 64, 64, 1)))
+        return rc;
+    if ((rc = make_map3(&map_u, w.uhl, LCA_D, 2, uint64_t(B) * uint64_t(nb), uint64_t(LCA_D) * 2,
+                        uint64_t(LCA_D) * 4, 64, 1, 128)))
+        return rc;
+    if ((rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1)))
+        return rc;
+
+    // summary query of every block (mean of its own 16 queries, folded)
+    {
+        Launch l(st, K_PREP);
+        const float coef = p.scale / float(LCA_HEADS * 16);
+        const cudaError_t e = launch_ex(prep_summary_kernel, dim3(unsigned(int64_t(B) * nb), LCA_D / 64),
+                                        dim3(PREP_THREADS), 0, st, false, qv + size_t(k0) * 16 * LCA_HEADS * LCA_D,
+                                        16, int(nb), int64_t(L) * LCA_HEADS * LCA_D, coef, (float *)nullptr, w.uhl);
+        if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
+    }
+    const float sl2 = p.scale * 1.4426950408889634f;
+    for (int b = 0; b < B; ++b) {
+        for (int64_t kc0 = k0; kc0 < k0 + nb; kc0 += kPrefillChunk) {
+            const int nbc = int(std::min<int64_t>(kPrefillChunk, k0 + nb - kc0));
+            const int64_t total = pf_tri(kc0 + nbc, cw) - pf_tri(kc0, cw);   // representatives of the chunk
+            CUtensorMap map_rep = map_cache;
+            if (total > 0) {
+                if ((rc = make_map3(&map_rep, w.rep, LCA_D, uint64_t(total), 1, uint64_t(LCA_D) * 2,
+                                    uint64_t(total) * LCA_D * 2, 64, 64, 1)))
+                    return rc;
+                CondPreArgs c{};
+                c.kc0 = kc0;
+                c.nbc = nbc;
+                c.cw = cw;
+                c.b = b;
+                c.n_gt = int((pf_groups(kc0 + nbc - 1, cw) + 3) / 4);
+                c.ublk0 = int(int64_t(b) * nb + (kc0 - k0));
+                c.rep = w.rep;
+                c.k0 = k0;
+                c.m_ld = m_ld;
+                c.anchor = anchor ? anchor + size_t(b) * size_t(nb) * size_t(m_ld) : nullptr;
+                const int n_bt = (nbc + 127) / 128;
+                Launch l(st, K_PREFILL_CONDENSE);
+                const cudaError_t e = launch_ex(condense_prefill_kernel, dim3(unsigned(n_bt * c.n_gt)),
+                                                dim3(CP_THREADS), CP_SMEM_ALLOC, st, false, map_cache, map_u, c);
+                if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
+            }
+            const size_t row_out = size_t(b) * size_t(q_len) + size_t(16 * (kc0 - k0));   // first output row
+            {
+                AttnPreArgs a{};
+                a.L = L;
+                a.b = b;
+                a.kc0 = kc0;
+                a.nbc = nbc;
+                a.cw = cw;
+                a.sl2 = sl2;
+                a.o_bf16 = w.o_bf16;
+                a.o_lat = o_lat ? o_lat + row_out * LCA_HEADS * LCA_DC : nullptr;
+                Launch l(st, K_PREFILL);
+                const cudaError_t e = launch_ex(attn_prefill_kernel, dim3(unsigned(4 * nbc)), dim3(AP_THREADS),
+                                                AP_SMEM_ALLOC, st, false, map_cache, map_q, map_rep, a);
+                if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
+            }
+            {
+                const int64_t R = int64_t(16) * nbc;
+                CUtensorMap map_a;
+                if ((rc = make_map3(&map_a, w.o_bf16, LCA_DC, LCA_HEADS, uint64_t(R), uint64_t(LCA_DC) * 2,
+                                    uint64_t(LCA_HEADS) * LCA_DC * 2, 64, 1, 128)))
+                    return rc;
+                Launch l(st, K_GEMM);
+                const cudaError_t e = launch_ex(wuv_gemm_kernel, dim3(unsigned((R + 127) / 128), LCA_HEADS),
+                                                dim3(128), GM_SMEM_ALLOC, st, false, map_a, map_w,
+                                                out + row_out * LCA_HEADS * LCA_DV, R);
+                if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
+            }
+        }
+    }
+    return LCA_OK;
 }
 
 const char *lca_strerror(int status)
@@ -519,7 +655,7 @@ int lca_profile_collect(lca_kernel_time *out, int max)
         std::lock_guard<std::mutex> lk(g_mu);
         recs.swap(g_prof_used);
     }
-    lca_kernel_time acc[8];
+    lca_kernel_time acc[kNumKernelIds];
     std::memset(acc, 0, sizeof acc);
     int rc = LCA_OK;
     for (const ProfRec &r : recs) {
@@ -535,7 +671,7 @@ int lca_profile_collect(lca_kernel_time *out, int max)
     }
     if (rc) return rc;
     int n = 0;
-    for (int k = 1; k < 7 && n < max; ++k) {
+    for (int k = 1; k < kNumKernelIds && n < max; ++k) {
         if (!acc[k].launches) continue;
         std::snprintf(out[n].name, sizeof out[n].name, "%s", kKernelNames[k]);
         out[n].launches = acc[k].launches;

@@ -9,15 +9,19 @@
 
 namespace lca {
 
-// u[b][576] fp32 and its bf16 hi/lo split uhl[b][2][576] (u = hi + lo to
-// ~2^-17 relative), used by the tensor-core importance pass.
-// Grid (B, 9): a block owns 64 columns of one sequence; its 256 threads are
+// u[b][576] fp32 (skipped when u is NULL) and its bf16 hi/lo split
+// uhl[b][2][576] (u = hi + lo to ~2^-17 relative), used by the tensor-core
+// importance pass.  Unit b reads the g*16 query rows starting at
+// q_recent + (b / nbs) * seq_stride + (b % nbs) * g*16*576: decode has one
+// unit per sequence (nbs = 1), blockwise prefill one per block of g queries.
+// Grid (units, 9): a block owns 64 columns of one unit; its 256 threads are
 // 8 column groups (16-byte loads) x 32 row slices of the g*16 (t, h) query
 // rows, combined through shared memory.
 constexpr int PREP_THREADS = 256;
 
 __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16_t *__restrict__ q_recent,
-                                                                    int g, float coef, float *__restrict__ u,
+                                                                    int g, int nbs, int64_t seq_stride,
+                                                                    float coef, float *__restrict__ u,
                                                                     uint16_t *__restrict__ uhl)
 {
     __shared__ float part[32][64 + 1];
@@ -25,7 +29,8 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16
     const int cg = threadIdx.x & 7, sl = threadIdx.x >> 3;
     const int col0 = blockIdx.y * 64 + 8 * cg;
     const int rows = g * LCA_HEADS;
-    const uint16_t *base = q_recent + size_t(b) * rows * LCA_D + col0;
+    const uint16_t *base =
+        q_recent + size_t(b / nbs) * size_t(seq_stride) + size_t(b % nbs) * rows * LCA_D + col0;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int r0 = sl; r0 < rows; r0 += 32 * 8) {
         uint4 x[8];
@@ -53,7 +58,7 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16
         for (int k = 0; k < 32; ++k) t += part[k][c];
         const int col = blockIdx.y * 64 + c;
         const float uu = t * coef;
-        u[size_t(b) * LCA_D + col] = uu;
+        if (u) u[size_t(b) * LCA_D + col] = uu;
         const __nv_bfloat16 hi = __float2bfloat16_rn(uu);
         const __nv_bfloat16 lo = __float2bfloat16_rn(uu - __bfloat162float(hi));
         uhl[(size_t(b) * 2 + 0) * LCA_D + col] = __bfloat16_as_ushort(hi);
