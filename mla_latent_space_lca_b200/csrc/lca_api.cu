@@ -212,7 +212,7 @@ constexpr int64_t kPrefillChunk = 256;
 
 struct PrefillWs {
     uint16_t *uhl;      // [B * nb][2][576]
-    uint16_t *rep;      // [chunk blocks * m_bound][576]
+    uint16_t *rep;      // [4 ceil(m_bound / 4)][chunk blocks][576]
     uint16_t *o_bf16;   // [chunk blocks * 16][16][512]
     size_t bytes;
 };
@@ -224,7 +224,7 @@ PrefillWs prefill_ws_layout(void *ws, int B, int64_t nb, int64_t m_bound)
     size_t off[4];
     off[0] = 0;
     off[1] = off[0] + align_up(size_t(B) * size_t(nb) * 2 * LCA_D * 2);
-    off[2] = off[1] + align_up(size_t(nbc) * size_t(std::max<int64_t>(m_bound, 1)) * LCA_D * 2);
+    off[2] = off[1] + align_up(size_t(nbc) * size_t(4 * std::max<int64_t>((m_bound + 3) / 4, 1)) * LCA_D * 2);
     off[3] = off[2] + align_up(size_t(nbc) * 16 * LCA_HEADS * LCA_DC * 2);
     w.bytes = off[3];
     if (ws) {
@@ -556,18 +556,19 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     for (int b = 0; b < B; ++b) {
         for (int64_t kc0 = k0; kc0 < k0 + nb; kc0 += kPrefillChunk) {
             const int nbc = int(std::min<int64_t>(kPrefillChunk, k0 + nb - kc0));
-            const int64_t total = pf_tri(kc0 + nbc, cw) - pf_tri(kc0, cw);   // representatives of the chunk
+            const int n_gt = int((pf_groups(kc0 + nbc - 1, cw) + 3) / 4);   // group tiles of the chunk
             CUtensorMap map_rep = map_cache;
-            if (total > 0) {
-                if ((rc = make_map3(&map_rep, w.rep, LCA_D, uint64_t(total), 1, uint64_t(LCA_D) * 2,
-                                    uint64_t(total) * LCA_D * 2, 64, 64, 1)))
+            if (n_gt > 0) {
+                // group-major [4 n_gt][nbc][576]; a box is 64 groups of one block
+                if ((rc = make_map3(&map_rep, w.rep, LCA_D, uint64_t(nbc), uint64_t(4 * n_gt), uint64_t(LCA_D) * 2,
+                                    uint64_t(nbc) * LCA_D * 2, 64, 1, 64)))
                     return rc;
                 CondPreArgs c{};
                 c.kc0 = kc0;
                 c.nbc = nbc;
                 c.cw = cw;
                 c.b = b;
-                c.n_gt = int((pf_groups(kc0 + nbc - 1, cw) + 3) / 4);
+                c.n_gt = n_gt;
                 c.ublk0 = int(int64_t(b) * nb + (kc0 - k0));
                 c.rep = w.rep;
                 c.k0 = k0;

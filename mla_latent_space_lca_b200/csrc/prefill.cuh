@@ -5,8 +5,9 @@
 // the mean of its own 16 queries as summary query (LCT 关键设计 1, 2), and each
 // of its queries t attends [m_k representatives || cache rows 16 m_k .. t]
 // causally (整体框架, 关键设计 3).  With g = 16, m_k = max(0, k - cw) where
-// cw = ceil(w / 16), so the representatives of consecutive blocks pack into
-// one array with closed-form offsets (pf_tri).
+// cw = ceil(w / 16).  A chunk's representatives are stored group-major,
+// rep[j][block], so a condense task writes contiguous runs and the attention
+// reads a block's tile of 64 groups as one strided TMA box.
 //
 // Every block has its own representatives, and one representative tile is
 // attended by only 16 queries x 16 heads, so fusing the pooling into the
@@ -20,8 +21,11 @@
 //     (TMEM lane = block), then the pooling itself on the tensor cores:
 //     rep_j [128 blocks x 512] = alpha_j [128 x 16] * C_j [16 x 512]
 //     (K = 16, four N = 128 MMAs per group through three TMEM buffers), the
-//     anchor's RoPE key copied bit for bit.  Bound: the representative
-//     writes (1152 B per block and group).
+//     anchor's RoPE key copied bit for bit.  Every (group < 4 n_gt, block)
+//     entry of the chunk is written, so the rows the attention masks out are
+//     finite.  Outputs leave through a per-warp shared-memory transpose, so
+//     each store instruction writes whole 256-byte row segments.  Bound: the
+//     representative writes (1152 B per block and group).
 //
 //   attn_prefill_kernel: one CTA per (block, 4 consecutive queries) = 64
 //     query rows (query-major, 16 heads each), Q in shared memory.  Per tile
@@ -40,13 +44,8 @@
 
 namespace lca {
 
-// Representatives of block k, and their packed offset sum_{k' < k} m_k'.
+// Representatives of block k.
 __host__ __device__ __forceinline__ int64_t pf_groups(int64_t k, int cw) { return k > cw ? k - cw : 0; }
-__host__ __device__ __forceinline__ int64_t pf_tri(int64_t k, int cw)
-{
-    const int64_t x = k - cw;
-    return x > 0 ? x * (x - 1) / 2 : 0;
-}
 
 // ====================================================================== condense
 constexpr int CP_THREADS = 224;                 // 7 warps
@@ -71,7 +70,7 @@ struct CondPreArgs {
     int b;             // sequence
     int n_gt;          // group tiles per block tile (grid = block tiles x n_gt)
     int ublk0;         // row of block kc0 in the summary-query array
-    uint16_t *rep;     // the chunk's packed representatives [rows][576]
+    uint16_t *rep;     // the chunk's representatives, group-major [4 n_gt][nbc][576]
     int64_t k0;        // first block of the call (anchor rows)
     int64_t m_ld;      // anchor row length
     int32_t *anchor;   // this sequence's anchor rows [(k - k0)][m_ld], or NULL
@@ -84,8 +83,6 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
     const int bt = blockIdx.x / a.n_gt, gt = blockIdx.x - bt * a.n_gt;
     const int64_t kb0 = a.kc0 + int64_t(bt) * 128;
     const int nblk = min(128, a.nbc - 128 * bt);
-    // no block of this tile has a group in this group tile
-    if (int64_t(4) * gt >= pf_groups(kb0 + nblk - 1, a.cw)) return;
 
     extern __shared__ uint8_t cp_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -201,7 +198,6 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         const int64_t k = kb0 + row;
         const bool vblk = row < nblk;
         const int64_t mk = vblk ? pf_groups(k, a.cw) : 0;
-        const int64_t off = pf_tri(k, a.cw) - pf_tri(a.kc0, a.cw);
         const uint32_t lane_base = uint32_t(32 * warp) << 16;
         int anc[4] = {0, 0, 0, 0};
         bool ok = __all_sync(0xffffffffu, mbar_wait(sfull, 0, abort_flag, K_PREFILL_CONDENSE, 8));
@@ -257,21 +253,40 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive(aready);
 
+        // Output rows go through a per-warp staging area in the (now idle)
+        // U ring so that every store instruction writes whole row segments:
+        // lat: 32 rows x 256 B (one d-chunk), rope: 32 rows x 128 B.
+        uint8_t *stg_lat = smem + CP_OFF_U + warp * 8192;
+        uint8_t *stg_rope = smem + CP_OFF_U + 4 * 8192 + warp * 4096;
+        const int64_t kk_warp = int64_t(128) * bt + 32 * warp;   // chunk block of the warp's first lane
+        const int hl = lane >> 4, c16 = lane & 15;                // store phase: row 2x + hl, chunk c16
+
         // anchor keys (bit copies from the tile) and anchor positions
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(rfull, 0, abort_flag, K_PREFILL_CONDENSE, 9));
-        if (ok && vblk) {
+#pragma unroll 1
+        for (int jj = 0; jj < 4 && ok; ++jj) {
+            const int64_t j = 4 * int64_t(gt) + jj;
+            {
+                const int rr = 16 * jj + anc[jj];
+                const uint8_t *src = smem + 8 * CP_BOX + rr * 128;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int64_t j = 4 * int64_t(gt) + jj;
-                if (j < mk) {
-                    const int rr = 16 * jj + anc[jj];
-                    const uint8_t *src = smem + 8 * CP_BOX + rr * 128;
-                    uint4 *dst = reinterpret_cast<uint4 *>(a.rep + size_t(off + j) * LCA_D + LCA_DC);
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(stg_rope + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                        *reinterpret_cast<const uint4 *>(src + ((c ^ (rr & 7)) << 4));
+                if (a.anchor && vblk && j < mk)
+                    a.anchor[size_t(k - a.k0) * size_t(a.m_ld) + size_t(j)] = int32_t(16 * j + anc[jj]);
+            }
+            __syncwarp();
+            // 4 rows of 128 B per instruction: lane -> row 4x + lane/8, chunk lane%8
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) dst[c] = *reinterpret_cast<const uint4 *>(src + ((c ^ (rr & 7)) << 4));
-                    if (a.anchor) a.anchor[size_t(k - a.k0) * size_t(a.m_ld) + size_t(j)] = int32_t(16 * j + anc[jj]);
+            for (int x = 0; x < 8; ++x) {
+                const int rr = 4 * x + (lane >> 3), c = lane & 7;
+                if (kk_warp + rr < a.nbc) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stg_rope + rr * 128 + ((c ^ (rr & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(a.rep + (size_t(j) * a.nbc + size_t(kk_warp + rr)) * LCA_D + LCA_DC + 8 * c) = v;
                 }
             }
+            __syncwarp();
         }
 
         // drain the pooled latents: group jj, d-chunk cc, buffer idx % 3
@@ -292,12 +307,22 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(pempty(buf));
-            const int64_t j = 4 * int64_t(gt) + jj;
-            if (vblk && j < mk) {
-                uint4 *dst = reinterpret_cast<uint4 *>(a.rep + size_t(off + j) * LCA_D + 128 * cc);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            for (int e = 0; e < 16; ++e)
+                *reinterpret_cast<uint4 *>(stg_lat + lane * 256 + ((e ^ c16) << 4)) =
+                    make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            __syncwarp();
+            const int64_t j = 4 * int64_t(gt) + jj;
+            // 2 rows of 256 B per instruction
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const int rr = 2 * x + hl;
+                if (kk_warp + rr < a.nbc) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stg_lat + rr * 256 + ((c16 ^ (rr & 15)) << 4));
+                    *reinterpret_cast<uint4 *>(a.rep + (size_t(j) * a.nbc + size_t(kk_warp + rr)) * LCA_D + 128 * cc + 8 * c16) = v;
+                }
             }
+            __syncwarp();
         }
     }
 
@@ -343,7 +368,6 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     const int64_t k = a.kc0 + blk;
     const int64_t t_first = 16 * k + 4 * qq;
     const int64_t mk = pf_groups(k, a.cw);
-    const int64_t off = pf_tri(k, a.cw) - pf_tri(a.kc0, a.cw);
     const int64_t win0 = 16 * mk;
     const int n_rep = int((mk + 63) / 64);
     const int n_tiles = n_rep + int((t_first + 4 - win0 + 63) / 64);
@@ -414,7 +438,7 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
                 if (i < n_rep) {
 #pragma unroll 1
                     for (int ch = 0; ch < 9; ++ch)
-                        tma_load_3d_plain(dst + ch * AP_CHUNK, &map_rep, full(s), 64 * ch, int(off + 64 * i), 0);
+                        tma_load_3d_plain(dst + ch * AP_CHUNK, &map_rep, full(s), 64 * ch, int(k - a.kc0), 64 * i);
                 } else {
                     const int row = int(win0 + 64 * (i - n_rep));
 #pragma unroll 1
