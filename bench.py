@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+    python bench.py --workload prefill_b1_l128k --steps 10 --warmup 3   # blockwise prefill
 
 One step = one whole fused LCA decode step (summary query, importance,
 group softmax pooling, anchor pick, split-L attention over
@@ -13,6 +14,10 @@ default workload's cache (1.2 GB) is ~10x the L2, so no flush is needed
 between steps.  Multi-GPU (torchrun): each rank decodes its own batch (weak
 scaling, no data-path collective); timing is the max over ranks.  Rank 0
 prints one JSON line.
+
+The prefill workload times one blockwise prefill of the whole sequence
+(lca_prefill_block over [0, L)) per step; its roofline is the attention
+kernel's algorithmic flops against the sustained bf16 tensor peak.
 """
 from __future__ import annotations
 
@@ -31,24 +36,74 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from mla_latent_space_lca_b200.inputs import WORKLOADS, make_decode_inputs  # noqa: E402
+from mla_latent_space_lca_b200.inputs import WORKLOADS, make_decode_inputs, make_prefill_inputs  # noqa: E402
 
 ROW_BYTES = 576 * 2
 METRIC = "LCA decode tokens/s and cache-read GB/s (fraction of B200 HBM roofline)"
+PREFILL_METRIC = "LCA blockwise prefill tokens/s (fraction of B200 bf16 tensor roofline)"
 PROFILE_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None, help="default 2000 (decode), 10 (prefill)")
+    ap.add_argument("--warmup", type=int, default=None, help="default 20 (decode), 3 (prefill)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_b32_l32k")
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
+
+
+def measured_tensor_peak():
+    """Sustained bf16 GEMM peak (a kernel timed inside a long step)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except (OSError, KeyError, ValueError):
+        return 1400.0, "fallback (sustained)"
+
+
+def prefill_flops(L: int, w: int, g: int = 16):
+    """Algorithmic flops of a blockwise prefill over [0, L): block k has
+    m_k = max(0, floor((16k - w)/16)) representatives; its query t attends
+    m_k + (t - 16 m_k + 1) keys, each 16 heads x (576 + 512) x 2 flops; the
+    condensation scores (folded summary query, 576 x 2) and pools (512 x 2)
+    every history row of the block; W_UV is 16 x 512 x 128 x 2 per query."""
+    cw = -(-w // 16)
+    att = cond = 0
+    for k in range(L // 16):
+        m = max(0, k - cw)
+        keys = 16 * m + sum(16 * k + tt - 16 * m + 1 for tt in range(16))
+        att += keys * 16 * (576 + 512) * 2
+        cond += 16 * m * (576 + 512) * 2
+    wuv = L * 16 * 512 * 128 * 2
+    return {"attention": att, "condense": cond, "wuv": wuv}
+
+
+def prefill_cpu_baseline(inp, n_blocks: int, steps: int = 1, warmup: int = 0):
+    """The oracle on `n_blocks` evenly spaced blocks of the prefill (their
+    average cost matches the whole range's); tokens/s extrapolated."""
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits
+
+    nb = inp.L // 16
+    blocks = sorted(set(int(round(x)) for x in
+                        [i * (nb - 1) / max(1, n_blocks - 1) for i in range(n_blocks)]))
+    c, q, w = bf16_bits(inp.cache), bf16_bits(inp.q), bf16_bits(inp.w_uv)
+    for _ in range(warmup):
+        oracle.lca_prefill(c, q, w, 0, inp.L, 16, inp.w, inp.scale, blocks=blocks, want_olat=False)
+    times = []
+    for _ in range(max(1, steps)):
+        t0 = time.perf_counter()
+        oracle.lca_prefill(c, q, w, 0, inp.L, 16, inp.w, inp.scale, blocks=blocks, want_olat=False)
+        times.append(time.perf_counter() - t0)
+    tok_s = 16 * len(blocks) * inp.B / statistics.mean(times)
+    sample = (f"{len(blocks)} evenly spaced blocks of {nb} (16 queries each) per oracle call, "
+              f"{len(times)} calls; tokens/s extrapolated to the whole prefill")
+    return tok_s, oracle.num_threads(), sample, times
 
 
 def measured_hbm_peak():
@@ -202,6 +257,25 @@ def run_reference(args, rank, world):
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
+    if wl["kind"] == "prefill":
+        import oracle
+        inp = make_prefill_inputs(wl["B"], wl["L"], seed=0)
+        n = 2 * oracle.num_threads()
+        tok_s, cores, sample, times = prefill_cpu_baseline(inp, n, steps=args.steps, warmup=args.warmup)
+        ms = 1e3 * statistics.mean(times)
+        line = {
+            "impl": "reference", "metric": PREFILL_METRIC, "value": tok_s, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "B": wl["B"], "L": wl["L"], "g": 16, "w": 1024},
+            "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     inp = make_decode_inputs(wl["B"], wl["L"], seed=0)
     tok_s, cores, sample, times = cpu_baseline(inp, 0, steps=args.steps, warmup=args.warmup)
     ms = 1e3 * statistics.mean(times)
@@ -342,8 +416,131 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_ours_prefill(args, rank, world, local_rank):
+    import torch.distributed as dist
+
+    import mla_latent_space_lca_b200 as lca
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    B, L = wl["B"], wl["L"]
+    inp = make_prefill_inputs(B, L, seed=replica_seed(rank))
+    cache, q, w_uv = inp.cache.to(dev), inp.q.to(dev), inp.w_uv.to(dev)
+    ws = lca.workspace(4, B, L, L, device=dev)
+    out = torch.empty(B, L, 16, 128, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lca.lca_prefill_block(cache, q, w_uv, 0, L, scale=inp.scale, out=out, ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)
+    n0 = lca.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    launches = (lca.launch_count() - n0) / args.steps
+    barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    if sampler:
+        sampler.stop()
+
+    lca.profile_enable(True)
+    for _ in range(min(args.steps, 3)):
+        step()
+    torch.cuda.synchronize()
+    prof = lca.profile_collect()
+    lca.profile_enable(False)
+
+    # end to end: cache and queries from pinned host memory, out back to host
+    pin = [t.pin_memory() for t in (inp.cache, inp.q)]
+    h_out = torch.empty(B, L, 16, 128, dtype=torch.float32).pin_memory()
+    dbuf = [torch.empty_like(t, device=dev) for t in pin]
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    d2h = h_out.numel() * 4
+
+    def e2e_step():
+        for d, h in zip(dbuf, pin):
+            d.copy_(h, non_blocking=True)
+        lca.lca_prefill_block(dbuf[0], dbuf[1], w_uv, 0, L, scale=inp.scale, out=out, ws=ws)
+        h_out.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    n_e2e = max(1, min(args.e2e_steps, 3))
+    for _ in range(n_e2e):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / n_e2e, world, dev)
+    rc, detail = lca.device_status(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    if rank != 0:
+        return
+    tokens = B * L * world
+    fl = prefill_flops(L, inp.w)
+    step_flops = B * sum(fl.values())
+    peak, peak_kind = measured_tensor_peak()
+    attn = prof.get("attn_prefill")
+    attn_ms = attn[1] / attn[0] if attn else None
+    attn_flops_launch = B * fl["attention"] / (attn[0] / min(args.steps, 3)) if attn else None
+    achieved = attn_flops_launch / (attn_ms / 1e3) / 1e12 if attn_ms else None
+    line = {
+        "metric": PREFILL_METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B_per_gpu": B, "L": L, "q_len": L, "g": 16, "w": 1024,
+                   "heads": 16, "d_c": 512, "d_r": 64, "parallelism": f"replicas x{world}",
+                   "l2": "queries (B*L*16*1152 B) and representatives far larger than the 126 MB L2; no flush"},
+        "step_tflops": step_flops / (ms / 1e3) / 1e12,
+        "roofline": {"bound": "tensor", "kernel": "attn_prefill", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
+                     "traffic": None, "algorithmic_flops_per_launch": attn_flops_launch,
+                     "launch_ms": attn_ms},
+        "kernels_ms_per_step": {k: v[1] / min(args.steps, 3) for k, v in prof.items()},
+        "gpu_launches": launches,
+        "clocks": sampler.summary() if sampler else None,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        tok_s, cores, sample, _ = prefill_cpu_baseline(inp, 2 * oracle.num_threads())
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
+    prefill = WORKLOADS[args.workload]["kind"] == "prefill"
+    if args.steps is None:
+        args.steps = 10 if prefill else 2000
+    if args.warmup is None:
+        args.warmup = 3 if prefill else 20
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
@@ -358,7 +555,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        (run_ours_prefill if prefill else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -30,15 +30,16 @@
 //   attn_prefill_kernel: one CTA per (block, 4 consecutive queries) = 64
 //     query rows (query-major, 16 heads each), Q in shared memory.  Per tile
 //     of 64 rows (representatives, then window rows):
-//       S_j [64 x 64] = Q[:, 288j : +288] * tile[:, 288j : +288]^T, j = 0, 1
-//         (two K-half chains, SS MMA, M = 64 -> TMEM lanes 0-15 per quadrant)
+//       S_c [64 x 64] = Q[:, 144c : +144] * tile[:, 144c : +144]^T, c = 0..3
+//         (four K-quarter chains on four issuing warps, SS MMA, M = 64 ->
+//         TMEM lanes 0-15 per quadrant; S = sum of the four)
 //       O^T[128c .. +127, 64] += tile_lat[:, 128c ..]^T * P^T, c = 0..3
 //         (four PV chains, M = 128, N = 64)
 //     Online softmax per query row with a reference max moved only when it
 //     grows by more than 2^8; causal and ragged-tile masks; the epilogue
 //     writes o = O / l as bf16 (the W_UV GEMM's A operand) and optionally fp32.
-//     O^T (256 columns) plus double-buffered S (256) fill TMEM exactly, which
-//     is what caps a CTA at 64 query rows.
+//     O^T (256 columns) plus the four S partials (256) fill TMEM exactly,
+//     which is what caps a CTA at 64 query rows.
 #pragma once
 #include "common.cuh"
 
@@ -260,6 +261,8 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         uint8_t *stg_rope = smem + CP_OFF_U + 4 * 8192 + warp * 4096;
         const int64_t kk_warp = int64_t(128) * bt + 32 * warp;   // chunk block of the warp's first lane
         const int hl = lane >> 4, c16 = lane & 15;                // store phase: row 2x + hl, chunk c16
+        // representative (group j, chunk block kk) lives in row j nbc + kk
+        auto rep_row = [&](int64_t j, int64_t kk) -> size_t { return size_t(j * a.nbc + kk); };
 
         // anchor keys (bit copies from the tile) and anchor positions
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(rfull, 0, abort_flag, K_PREFILL_CONDENSE, 9));
@@ -283,7 +286,7 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
                 const int rr = 4 * x + (lane >> 3), c = lane & 7;
                 if (kk_warp + rr < a.nbc) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(stg_rope + rr * 128 + ((c ^ (rr & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(a.rep + (size_t(j) * a.nbc + size_t(kk_warp + rr)) * LCA_D + LCA_DC + 8 * c) = v;
+                    *reinterpret_cast<uint4 *>(a.rep + rep_row(j, kk_warp + rr) * LCA_D + LCA_DC + 8 * c) = v;
                 }
             }
             __syncwarp();
@@ -319,7 +322,7 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
                 const int rr = 2 * x + hl;
                 if (kk_warp + rr < a.nbc) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(stg_lat + rr * 256 + ((c16 ^ (rr & 15)) << 4));
-                    *reinterpret_cast<uint4 *>(a.rep + (size_t(j) * a.nbc + size_t(kk_warp + rr)) * LCA_D + 128 * cc + 8 * c16) = v;
+                    *reinterpret_cast<uint4 *>(a.rep + rep_row(j, kk_warp + rr) * LCA_D + 128 * cc + 8 * c16) = v;
                 }
             }
             __syncwarp();
@@ -333,17 +336,16 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
 }
 
 // ====================================================================== attention
-constexpr int AP_THREADS = 352;                 // 11 warps
+constexpr int AP_THREADS = 416;                 // 13 warps
 constexpr int AP_CHUNK = 8192;                  // [64 rows x 64 cols] bf16
 constexpr int AP_STAGE = 9 * AP_CHUNK;          // 73728: Q, then two row stages
-constexpr int AP_OFF_P = 3 * AP_STAGE;          // P [64 query rows x 64] bf16
-constexpr int AP_OFF_BAR = AP_OFF_P + 8192;
+constexpr int AP_OFF_BAR = 3 * AP_STAGE;
 constexpr int AP_OFF_MISC = AP_OFF_BAR + 8 * 20;
 constexpr int AP_OFF_FSC = AP_OFF_MISC + 16;    // [2][64] rescale factors
 constexpr int AP_OFF_LINV = AP_OFF_FSC + 512;   // [64] 1 / l
 constexpr int AP_SMEM = AP_OFF_LINV + 256;
 constexpr int AP_SMEM_ALLOC = AP_SMEM + 1024;
-constexpr uint32_t AP_TM_S = 0;                 // S[buf][half]: 4 x 64 columns
+constexpr uint32_t AP_TM_S = 0;                 // S partials of the 4 K-quarter chains: 4 x 64 columns
 constexpr uint32_t AP_TM_O = 256;               // O^T: 4 d-chunks x 64 columns
 constexpr uint32_t AP_TM_COLS = 512;
 
@@ -379,13 +381,12 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     auto BAR = [&](int i) -> uint32_t { return sbase + AP_OFF_BAR + 8 * i; };
-    const uint32_t qfull = BAR(0), pfull = BAR(9), pempty = BAR(10), ofull = BAR(11);
+    const uint32_t qfull = BAR(0), sfull = BAR(5), sempty = BAR(6), pfull = BAR(7), pempty = BAR(8),
+                   ofull = BAR(9);
     auto full = [&](int s) { return BAR(1 + s); };
     auto empty = [&](int s) { return BAR(3 + s); };
-    auto sfull = [&](int s) { return BAR(5 + s); };
-    auto sempty = [&](int s) { return BAR(7 + s); };
-    auto fex = [&](int s) { return BAR(12 + s); };
-    auto drain = [&](int w) { return BAR(14 + (w == 4 ? 0 : w == 7 ? 1 : w == 6 ? 2 : w - 5)); };
+    auto fex = [&](int s) { return BAR(10 + s); };
+    auto drain = [&](int w) { return BAR(12 + (w - 5)); };   // issuing warps 5..12
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AP_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AP_OFF_MISC + 4);
     float *fsc = reinterpret_cast<float *>(smem + AP_OFF_FSC);
@@ -396,14 +397,14 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 4);      // four PV chains
-            mbar_init(sfull(s), 2);      // both S chains
-            mbar_init(sempty(s), 4);     // four softmax warps
             mbar_init(fex(s), 4);
         }
+        mbar_init(sfull, 4);             // four S chains
+        mbar_init(sempty, 4);            // four softmax warps
         mbar_init(pfull, 4);
         mbar_init(pempty, 4);
         mbar_init(ofull, 4);
-        for (int i = 14; i < 20; ++i) mbar_init(BAR(i), 1);
+        for (int i = 12; i < 20; ++i) mbar_init(BAR(i), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -415,10 +416,12 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t qbase = sbase, pbase = sbase + AP_OFF_P;
+    const uint32_t qbase = sbase;
+    // tile i lives in stage i & 1; once S(i) has completed, its RoPE box (box
+    // 8) is dead and holds P(i) [64 query rows x 64 tile rows] for PV(i)
     auto stage_addr = [&](int i) -> uint32_t { return sbase + AP_STAGE * (1 + (i & 1)); };
 
-    if (warp == 5) {
+    if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tensormap(&map_q);
@@ -451,35 +454,38 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
             for (int s = 0; s < 2; ++s)
                 if (last[s] >= 0) mbar_wait(full(s), (last[s] >> 1) & 1, nullptr, K_PREFILL, 2);
         }
-    } else if (warp == 4 || warp == 7) {
-        // ------------------------------------------------------------ S chains (K halves)
+    } else if (warp >= 5 && warp <= 8) {
+        // ------------------------------------------------------------ S chains (K quarters)
+        // chain c = warp - 5 accumulates k-steps 9c .. 9c+8 into its own 64
+        // columns; a single S buffer, released by the softmax warps as soon as
+        // they have loaded it
         if (lane == 0) {
-            const int half = (warp == 7) ? 1 : 0;
+            const int c = warp - 5;
             constexpr uint32_t IDESC_S = idesc_bf16(64, 64, 0, 0);
             bool ok = mbar_wait(qfull, 0, abort_flag, K_PREFILL, 3);
 #pragma unroll 1
             for (int i = 0; i < n_tiles && ok; ++i) {
                 if (!(ok = mbar_wait(full(i & 1), (i >> 1) & 1, abort_flag, K_PREFILL, 4))) break;
-                if (!(ok = mbar_wait(sempty(i & 1), ((i >> 1) & 1) ^ 1, abort_flag, K_PREFILL, 5))) break;
+                if (!(ok = mbar_wait(sempty, (i & 1) ^ 1, abort_flag, K_PREFILL, 5))) break;
                 tc_fence_after();
                 const uint32_t stage = stage_addr(i);
-                const uint32_t dS = tmem + AP_TM_S + 64 * (2 * (i & 1) + half);
-#pragma unroll 6
-                for (int ks = 0; ks < 18; ++ks) {
-                    const int kg = 18 * half + ks;
+                const uint32_t dS = tmem + AP_TM_S + 64 * c;
+#pragma unroll
+                for (int ks = 0; ks < 9; ++ks) {
+                    const int kg = 9 * c + ks;
                     const uint32_t o = (kg >> 2) * AP_CHUNK + (kg & 3) * 32;
                     mma_ss(dS, sdesc_sw128(qbase + o, 16, 1024), sdesc_sw128(stage + o, 16, 1024), IDESC_S,
                            ks > 0 ? 1u : 0u);
                 }
-                tc_commit(sfull(i & 1));
+                tc_commit(sfull);
             }
             tc_commit(drain(warp));
             mbar_wait(drain(warp), 0, nullptr, K_PREFILL, 6);
         }
-    } else if (warp == 6 || warp >= 8) {
+    } else if (warp >= 9) {
         // ------------------------------------------------------------ PV chains (d-chunks)
         if (lane == 0) {
-            const int cc = (warp == 6) ? 0 : warp - 7;
+            const int cc = warp - 9;
             constexpr uint32_t IDESC_PV = idesc_bf16(128, 64, 1, 0);
             bool ok = true;
 #pragma unroll 1
@@ -490,7 +496,7 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_ss(tmem + AP_TM_O + 64 * cc, sdesc_sw128(stage + 2 * cc * AP_CHUNK + ks * 2048, AP_CHUNK, 1024),
-                           sdesc_sw128(pbase + ks * 32, 16, 1024), IDESC_PV, (j | ks) ? 1u : 0u);
+                           sdesc_sw128(stage + 8 * AP_CHUNK + ks * 32, 16, 1024), IDESC_PV, (j | ks) ? 1u : 0u);
                 tc_commit(empty(j & 1));
                 tc_commit(pempty);
                 if (j == n_tiles - 1) tc_commit(ofull);
@@ -513,33 +519,27 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 #pragma unroll 1
         for (int i = 0; i < n_tiles; ++i) {
             const int sb = i & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(sfull(sb), (i >> 1) & 1, abort_flag, K_PREFILL, 9));
+            ok = __all_sync(0xffffffffu, mbar_wait(sfull, i & 1, abort_flag, K_PREFILL, 9));
             if (!ok) break;
             tc_fence_after();
             float va[16], vb[16];
-            {
-                float r[32];
-                const uint32_t s0 = tmem + AP_TM_S + 128 * sb + lane_base;
-                tmem_ld_16x256b_x8(s0, r);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    va[2 * j] = r[4 * j];
-                    va[2 * j + 1] = r[4 * j + 1];
-                    vb[2 * j] = r[4 * j + 2];
-                    vb[2 * j + 1] = r[4 * j + 3];
-                }
-                tmem_ld_16x256b_x8(s0 + 64, r);
+            for (int x = 0; x < 16; ++x) va[x] = vb[x] = 0.f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    va[2 * j] += r[4 * j];
-                    va[2 * j + 1] += r[4 * j + 1];
-                    vb[2 * j] += r[4 * j + 2];
-                    vb[2 * j + 1] += r[4 * j + 3];
+            for (int c = 0; c < 2; ++c) {   // partials 2c and 2c+1 in one load
+                uint32_t r[64];
+                tmem_ld_16x256b_x16(tmem + AP_TM_S + 128 * c + lane_base, r);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    va[2 * (j & 7)] += __uint_as_float(r[4 * j]);
+                    va[2 * (j & 7) + 1] += __uint_as_float(r[4 * j + 1]);
+                    vb[2 * (j & 7)] += __uint_as_float(r[4 * j + 2]);
+                    vb[2 * (j & 7) + 1] += __uint_as_float(r[4 * j + 3]);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(sempty(sb));
+            if (lane == 0) mbar_arrive(sempty);
 
             // valid columns of this tile for query t
             int64_t nv;
@@ -590,14 +590,11 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
                 fsc[sb * 64 + r1] = fb;
             }
 
-            // P rows (K-major, 128-byte swizzle); the single P buffer is free
-            // once PV(i-1) has completed, which also makes O safe to rescale
-            ok = __all_sync(0xffffffffu, mbar_wait(pempty, (i & 1) ^ 1, abort_flag, K_PREFILL, 10));
-            if (!ok) break;
-            tc_fence_after();
+            // P rows (K-major, 128-byte swizzle) into box 8 of this tile's stage
             {
-                uint8_t *p0 = smem + AP_OFF_P + (r0 >> 3) * 1024 + (r0 & 7) * 128;
-                uint8_t *p1 = smem + AP_OFF_P + (r1 >> 3) * 1024 + (r1 & 7) * 128;
+                uint8_t *pb = smem + AP_STAGE * (1 + sb) + 8 * AP_CHUNK;
+                uint8_t *p0 = pb + (r0 >> 3) * 1024 + (r0 & 7) * 128;
+                uint8_t *p1 = pb + (r1 >> 3) * 1024 + (r1 & 7) * 128;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     *reinterpret_cast<uint32_t *>(p0 + ((j ^ (r0 & 7)) << 4) + 4 * sub) = pack_bf16(va[2 * j], va[2 * j + 1]);
@@ -613,6 +610,10 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
             if (!ok) break;
             const bool any = __any_sync(0xffffffffu, fsc[sb * 64 + lane] != 1.f || fsc[sb * 64 + 32 + lane] != 1.f);
             if (any) {
+                // O must hold PV(i-1) before it is rescaled
+                ok = __all_sync(0xffffffffu, mbar_wait(pempty, (i & 1) ^ 1, abort_flag, K_PREFILL, 10));
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll 1
                 for (int cc = 0; cc < 4; ++cc) {
                     const uint32_t ta_ = tmem + lane_base + AP_TM_O + 64 * cc;

@@ -145,15 +145,15 @@ def lca_attend_reps(cache, rep, q, w_uv, g: int, w: int, scale: float, dr: int =
 
 
 def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, scale: float,
-                blocks=None, dr: int = 64, want_anchor: bool = False):
-    """Blockwise LCA prefill.  -> (o_lat [B,q_len,H,dc], out [B,q_len,H,dv], anchor|None).
+                blocks=None, dr: int = 64, want_anchor: bool = False, want_olat: bool = True):
+    """Blockwise LCA prefill.  -> (o_lat [B,q_len,H,dc] | None, out [B,q_len,H,dv], anchor|None).
     `blocks` = absolute block indices to evaluate (others left as NaN)."""
     cache, qpre, w_uv = _u16(cache), _u16(qpre), _u16(w_uv)
     B, L, D = cache.shape
     H = qpre.shape[2]
     dc = D - dr
     dv = w_uv.shape[2]
-    o_lat = np.full((B, q_len, H, dc), np.nan)
+    o_lat = np.full((B, q_len, H, dc), np.nan) if want_olat else None
     out = np.full((B, q_len, H, dv), np.nan)
     bl = None
     nbl = 0
