@@ -146,6 +146,7 @@ WORKLOADS = {
     "decode_b8_l128k":  dict(kind="decode", B=8, L=131072),
     "prefill_b1_l128k": dict(kind="prefill", B=1, L=131072),
     "decode_b1_l1m":    dict(kind="decode", B=1, L=1048576),
-    # smaller case for profiler captures (cache 302 MB, still > L2)
+    # smaller cases for profiler captures (cache 302 MB / queries 302 MB, > L2)
     "decode_b8_l32k":   dict(kind="decode", B=8, L=32768),
+    "prefill_b1_l16k":  dict(kind="prefill", B=1, L=16384),
 }
