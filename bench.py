@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mla-compare", type=int, default=0,
+                    help="prefill: also time N full causal MLA prefills (w = L) on the same inputs")
     return ap.parse_args()
 
 
@@ -494,6 +496,26 @@ def run_ours_prefill(args, rank, world, local_rank):
     x1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(x0.elapsed_time(x1) / n_e2e, world, dev)
+    # in-run comparison: full causal MLA prefill over the same inputs (the same
+    # path with a window covering the whole sequence, so nothing is condensed)
+    mla_ms = None
+    if args.mla_compare:
+        ws_mla = lca.workspace(4, B, L, L, w=L, device=dev)
+
+        def mla_step():
+            lca.lca_prefill_block(cache, q, w_uv, 0, L, w=L, scale=inp.scale, out=out, ws=ws_mla,
+                                  stream=stream)
+
+        mla_step()
+        torch.cuda.synchronize()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        for _ in range(args.mla_compare):
+            mla_step()
+        m1.record(stream)
+        torch.cuda.synchronize()
+        mla_ms = max_over_ranks(m0.elapsed_time(m1) / args.mla_compare, world, dev)
+        del ws_mla
     rc, detail = lca.device_status(clear=True)
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail:#x})")
@@ -526,6 +548,11 @@ def run_ours_prefill(args, rank, world, local_rank):
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
+    if mla_ms is not None:
+        mla_fl = prefill_flops(L, L)
+        line["mla_prefill"] = {"ms_per_step": mla_ms, "tokens_per_s": tokens / (mla_ms / 1e3),
+                               "speedup_of_lca": mla_ms / ms,
+                               "step_tflops": B * sum(mla_fl.values()) / (mla_ms / 1e3) / 1e12}
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         tok_s, cores, sample, _ = prefill_cpu_baseline(inp, 2 * oracle.num_threads())

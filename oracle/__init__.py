@@ -55,6 +55,8 @@ def _load():
         lib.ora_lca_decode.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
         lib.ora_lca_attend_reps.restype = I
         lib.ora_lca_attend_reps.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P]
+        lib.ora_lca_decode_stored.restype = I
+        lib.ora_lca_decode_stored.argtypes = [P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
         lib.ora_lca_prefill.restype = I
         lib.ora_lca_prefill.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, P, Lg,
                                         P, P, P]
@@ -142,6 +144,25 @@ def lca_attend_reps(cache, rep, q, w_uv, g: int, w: int, scale: float, dr: int =
     _load().ora_lca_attend_reps(_ptr(cache), _ptr(rep), _ptr(q), _ptr(w_uv), B, L, H, dc, dr,
                                 dv, g, w, scale, _ptr(o_lat), _ptr(out))
     return o_lat, out
+
+
+def lca_decode_stored(cache, q_all, w_uv, g: int, w: int, scale: float, dr: int = 64):
+    """Stored-representative decode at cache length L: group j condensed with
+    the summary query of the step where it left the window (queries at
+    positions w + g j .. w + g j + g - 1), query at L-1 attends [reps || window].
+    q_all [B,L,H,D] u16.  -> (o_lat [B,H,dc], out [B,H,dv], anchor [B,m])."""
+    cache, q_all, w_uv = _u16(cache), _u16(q_all), _u16(w_uv)
+    B, L, D = cache.shape
+    H = q_all.shape[2]
+    dc = D - dr
+    dv = w_uv.shape[2]
+    m = num_groups(L, g, w)
+    o_lat = np.zeros((B, H, dc))
+    out = np.zeros((B, H, dv))
+    anchor = np.zeros((B, max(m, 1)), np.int32)
+    _load().ora_lca_decode_stored(_ptr(cache), _ptr(q_all), _ptr(w_uv), B, L, H, dc, dr, dv, g, w,
+                                  scale, _ptr(o_lat), _ptr(out), _ptr(anchor))
+    return o_lat, out, anchor[:, :m]
 
 
 def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, scale: float,

@@ -356,3 +356,51 @@ int ora_lca_prefill(const uint16_t *cache, const uint16_t *qpre, const uint16_t 
         }
     return 0;
 }
+
+/* Stored-representative decode: the reading of the page's "90% KV-cache
+ * compression" (一句话总结, 关键发现) in which a group is condensed once and
+ * kept.  Group j leaves the window at the decode step whose cache length is
+ * L_j = w + g (j + 1) (the first L with floor((L - w)/g) > j); it is condensed
+ * then, with the summary query of that step: the mean of the g queries at
+ * positions L_j - g .. L_j - 1 (关键设计 1, 2).  The decode step at length L
+ * attends [the m(L) kept representatives || rows m g .. L-1] with the query
+ * at position L - 1 (整体框架).
+ *   q_all [B][L][H][D] holds the query of every position.
+ *   anchor_out [B][m] (absolute positions) may be NULL. */
+int ora_lca_decode_stored(const uint16_t *cache, const uint16_t *q_all, const uint16_t *w_uv,
+                          int B, long L, int H, int dc, int dr, int dv, int g, int w,
+                          double scale, double *o_lat, double *out, int32_t *anchor_out)
+{
+    int D = dc + dr;
+    long m = ora_num_groups(L, g, w);
+    size_t mm = (size_t)(m > 0 ? m : 1);
+    double *rc = (double *)malloc(sizeof(double) * (size_t)B * mm * dc);
+    double *rk = (double *)malloc(sizeof(double) * (size_t)B * mm * dr);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; b++)
+        for (long j = 0; j < m; j++) {
+            long Lj = (long)w + (long)g * (j + 1);
+            double *qbar = (double *)malloc(sizeof(double) * H * D);
+            summary_query(q_all + ((size_t)b * L + (size_t)(Lj - g)) * H * D, g, H, D, qbar);
+            int I = condense_group(qbar, cache + ((size_t)b * L + (size_t)j * g) * D, g, H, dc,
+                                   dr, scale, rc + ((size_t)b * mm + j) * dc,
+                                   rk + ((size_t)b * mm + j) * dr, NULL, NULL);
+            if (anchor_out) anchor_out[(size_t)b * m + j] = (int32_t)(j * g + I);
+            free(qbar);
+        }
+    double *ol = (double *)malloc(sizeof(double) * (size_t)B * H * dc);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++)
+            attend_head(q_all + (((size_t)b * L + (size_t)(L - 1)) * H + h) * D, dc, dr, scale,
+                        m, rc + (size_t)b * mm * dc, rk + (size_t)b * mm * dr, NULL,
+                        cache + ((size_t)b * L + (size_t)m * g) * D, L - m * g,
+                        ol + ((size_t)b * H + h) * dc);
+    for (int b = 0; b < B; b++)
+        if (out) up_project(ol + (size_t)b * H * dc, w_uv, H, dc, dv, out + (size_t)b * H * dv);
+    if (o_lat) memcpy(o_lat, ol, sizeof(double) * (size_t)B * H * dc);
+    free(ol);
+    free(rc);
+    free(rk);
+    return 0;
+}

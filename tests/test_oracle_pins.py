@@ -308,3 +308,83 @@ def test_prefill_block_subset_matches_full(ora):
         sl = slice(k * g - 16, k * g - 16 + g)
         np.testing.assert_array_equal(out2[:, sl], out[:, sl])
     assert np.isnan(out2[:, 0]).all()
+
+
+# ----------------------------------------------------------------- stored representatives
+def stored_case(rng, B=2, L=61, H=3, dc=8, dr=4, dv=5, peak=3.0):
+    cache = rand_bits(rng, (B, L, dc + dr))
+    q_all = rand_bits(rng, (B, L, H, dc + dr), peak)
+    w_uv = rand_bits(rng, (H, dc, dv), 0.3)
+    return cache, q_all, w_uv
+
+
+def test_stored_with_identical_queries_is_recompute(ora):
+    """一句话总结 / 关键发现 (kept representatives): when every position has the
+    same query, every group's exit-time summary query is that query, so the
+    stored reading equals recomputing all groups with it."""
+    rng = np.random.default_rng(21)
+    cache, q_all, w_uv = stored_case(rng)
+    q_all[:] = q_all[:, :1]                      # one query everywhere
+    g, w = 4, 9
+    ol1, o1, a1 = ora.lca_decode_stored(cache, q_all, w_uv, g, w, 0.3, dr=4)
+    L = cache.shape[1]
+    q_recent = np.ascontiguousarray(q_all[:, L - g:L])
+    ol2, o2, a2 = ora.lca_decode(cache, q_recent, np.ascontiguousarray(q_all[:, L - 1]), w_uv, g, w,
+                                 0.3, dr=4)
+    assert ora.num_groups(L, g, w) == 13
+    assert np.array_equal(a1, a2)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(ol1, ol2, rtol=0, atol=1e-13)
+
+
+def test_stored_window_covering_everything_is_mla(ora):
+    rng = np.random.default_rng(22)
+    cache, q_all, w_uv = stored_case(rng, L=30)
+    ol1, o1, a1 = ora.lca_decode_stored(cache, q_all, w_uv, 4, 30, 0.3, dr=4)
+    ol2, o2 = ora.mla_decode(cache, np.ascontiguousarray(q_all[:, -1]), w_uv, 0.3, dr=4)
+    assert a1.shape[1] == 0
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+
+
+def test_stored_single_group_is_the_exit_step_condensation(ora):
+    """At L = w + g exactly one group has left the window, at this very step,
+    so the stored reading and the recompute reading coincide."""
+    rng = np.random.default_rng(23)
+    g, w = 4, 10
+    L = w + g
+    cache, q_all, w_uv = stored_case(rng, L=L)
+    ol1, o1, a1 = ora.lca_decode_stored(cache, q_all, w_uv, g, w, 0.3, dr=4)
+    ol2, o2, a2 = ora.lca_decode(cache, np.ascontiguousarray(q_all[:, L - g:L]),
+                                 np.ascontiguousarray(q_all[:, L - 1]), w_uv, g, w, 0.3, dr=4)
+    assert a1.shape == (2, 1)
+    assert np.array_equal(a1, a2)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+
+
+def test_stored_anchors_are_frozen_exit_time_condensations(ora):
+    """Group j's anchor is the argmax under the summary query of the step
+    where it left the window (cache length w + g (j+1)), whatever the
+    current length; different queries per position make that differ from the
+    recompute reading."""
+    rng = np.random.default_rng(24)
+    g, w = 4, 6
+    cache, q_all, w_uv = stored_case(rng, L=71, peak=20.0)
+    L = cache.shape[1]
+    _, _, a_now = ora.lca_decode_stored(cache, q_all, w_uv, g, w, 0.3, dr=4)
+    m = ora.num_groups(L, g, w)
+    assert a_now.shape == (2, m)
+    for j in range(m):
+        Lj = w + g * (j + 1)
+        r = ora.lca_condense(np.ascontiguousarray(cache[:, :Lj]), np.ascontiguousarray(q_all[:, Lj - g:Lj]),
+                             g, w, 0.3, dr=4)
+        assert r["anchor"].shape[1] == j + 1
+        assert np.array_equal(a_now[:, j], r["anchor"][:, j])
+    # an earlier length keeps the same anchors for its groups
+    Le = L - 13
+    _, _, a_early = ora.lca_decode_stored(np.ascontiguousarray(cache[:, :Le]),
+                                          np.ascontiguousarray(q_all[:, :Le]), w_uv, g, w, 0.3, dr=4)
+    assert np.array_equal(a_early, a_now[:, :a_early.shape[1]])
+    # and the recompute reading (current summary query for every group) differs somewhere
+    _, _, a_re = ora.lca_decode(cache, np.ascontiguousarray(q_all[:, L - g:L]),
+                                np.ascontiguousarray(q_all[:, L - 1]), w_uv, g, w, 0.3, dr=4)
+    assert not np.array_equal(a_re, a_now)
