@@ -127,6 +127,33 @@ int lca_decode_attn(const void *cache, const void *rep, const void *q, const voi
                     int64_t L, lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes,
                     void *stream);
 
+/* Stored-representative ("condensed cache") decode: the reading of the
+ * page's 90% KV-cache compression (一句话总结, 关键发现) in which a group is
+ * condensed once, when it leaves the window, and kept.  Group j leaves the
+ * window at the step whose cache length is w + g (j + 1); the caller keeps a
+ * representative cache rep[B][rep_cap][576] (rep_cap >= the largest m it
+ * will reach) and, at each step where m = lca_num_groups(L, p) has grown,
+ * appends the new groups with lca_condense_append, then attends with
+ * lca_decode_stored, which reads only the m kept rows and the window.
+ *
+ * lca_condense_append: condense groups j0 .. m-1 of every sequence with the
+ * summary query of q_recent (as lca_condense) into rows j0 .. m-1 of rep
+ * (row stride rep_cap rows per sequence); anchor [B][rep_cap] int32 and
+ * alpha [B][rep_cap][g] fp32 are optional, same rows.  0 <= j0 <= m;
+ * j0 == m writes nothing.  Requires g == 16.  ws: LCA_OP_CONDENSE bytes. */
+int lca_condense_append(const void *cache, const void *q_recent, int B, int64_t L, lca_params p,
+                        int64_t j0, void *rep, int64_t rep_cap, int32_t *anchor, float *alpha,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/* lca_decode_stored: the current query attends [rep rows 0 .. m-1 || cache
+ * rows m*g .. L-1] of each sequence, then W_UV (as lca_decode_attn, with the
+ * representative rows read at a stride of rep_cap rows per sequence).
+ * rep_cap >= m; rep may be NULL if m == 0.  Requires g == 16.
+ * ws: LCA_OP_DECODE_ATTN bytes. */
+int lca_decode_stored(const void *cache, const void *rep, int64_t rep_cap, const void *q,
+                      const void *w_uv, int B, int64_t L, lca_params p, float *out, float *o_lat,
+                      void *ws, size_t ws_bytes, void *stream);
+
 /* One whole LCA decode step, fused: summary query, per-group importance,
  * softmax pooling, anchor pick and attention over [representatives ||
  * window] in one pass over the cache (representatives never leave the

@@ -109,6 +109,43 @@ def lca_decode_attn(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     return out
 
 
+def lca_condense_append(cache, q_recent, rep, j0, g=16, w=1024, scale=None, anchor=None, alpha=None,
+                        ws=None, stream=None):
+    """Condense groups j0 .. m-1 into rows j0 .. of the representative cache
+    rep [B, rep_cap, 576] (bf16); returns m, the number of groups now held."""
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
+    _need(rep, "rep", torch.bfloat16)
+    if rep.dim() != 3 or rep.shape[0] != B or rep.shape[2] != D:
+        raise ValueError(f"rep has shape {tuple(rep.shape)}, expected ({B}, rep_cap, {D})")
+    m = num_groups(L, g, w)
+    ws = workspace(_lib.OP_CONDENSE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_condense_append(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale), int(j0),
+                                        _ptr(rep), rep.shape[1], _ptr(anchor), _ptr(alpha), _ptr(ws),
+                                        ws.numel(), _stream(stream))
+    check(rc, "lca_condense_append")
+    return m
+
+
+def lca_decode_stored(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None, ws=None,
+                      stream=None):
+    """Attention over the kept representatives rep [B, rep_cap, 576] (rows
+    0 .. m-1) and the window, then W_UV."""
+    B, L, _ = cache.shape
+    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    _need(rep, "rep", torch.bfloat16)
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_decode_stored(_ptr(cache), _ptr(rep), rep.shape[1], _ptr(q), _ptr(w_uv), B, L,
+                                      _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(ws), ws.numel(),
+                                      _stream(stream))
+    check(rc, "lca_decode_stored")
+    return out
+
+
 def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None,
                anchor=None, ws=None, stream=None):
     B, L, _ = cache.shape

@@ -27,11 +27,13 @@ struct CondenseArgs {
     const uint16_t *cache;   // [B][L][576]
     const float *u;          // [B][576]
     int64_t L;
-    int64_t m;               // groups per sequence
+    int64_t m;               // groups condensed per sequence: j0 .. j0+m-1
+    int64_t j0;              // first group
+    int64_t stride;          // rows per sequence of rep / anchor / alpha
     int64_t total;           // B * m
-    uint16_t *rep;           // [B][m][576]
-    int32_t *anchor;         // [B][m] or NULL
-    float *alpha;            // [B][m][16] or NULL
+    uint16_t *rep;           // [B][stride][576], rows j0 .. j0+m-1 written
+    int32_t *anchor;         // [B][stride] or NULL
+    float *alpha;            // [B][stride][16] or NULL
 };
 
 __device__ __forceinline__ float dot8(const uint4 x, const float *u)
@@ -65,7 +67,7 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
     const uint64_t pol = policy_evict_first();
 
     auto issue = [&](int64_t gi, int s) {
-        const int64_t b = gi / a.m, j = gi - b * a.m;
+        const int64_t b = gi / a.m, j = a.j0 + (gi - b * a.m);
         const uint16_t *src = a.cache + (size_t(b) * a.L + size_t(j) * 16) * LCA_D;
         const uint32_t bar = smem_u32(&bars[s]);
         mbar_expect_tx(bar, CD_GROUP_BYTES);
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
             ok = false;
             break;
         }
-        const int64_t b = gi / a.m, j = gi - b * a.m;
+        const int64_t b = gi / a.m, j = a.j0 + (gi - b * a.m);
         const uint8_t *tile = ring + s * CD_GROUP_BYTES;
 
         // importance: partial dots over this lane's 16-byte column slices
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
                 pa[r][7] = fmaf(ai, bf_hi(x.w), pa[r][7]);
             }
         }
-        uint16_t *dst = a.rep + (size_t(b) * a.m + size_t(j)) * LCA_D;
+        uint16_t *dst = a.rep + (size_t(b) * a.stride + size_t(j)) * LCA_D;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             uint4 o;
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
             const uint4 k = *reinterpret_cast<const uint4 *>(tile + bi * (LCA_D * 2) + LCA_DC * 2 + lane * 16);
             reinterpret_cast<uint4 *>(dst + LCA_DC)[lane] = k;
         }
-        const size_t gidx = size_t(b) * a.m + size_t(j);
+        const size_t gidx = size_t(b) * a.stride + size_t(j);
         if (a.anchor && lane == 0) a.anchor[gidx] = int32_t(j * 16 + bi);
         if (a.alpha && (lane & 1) == 0) a.alpha[gidx * 16 + tok] = al;
 

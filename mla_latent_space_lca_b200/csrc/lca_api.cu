@@ -263,7 +263,7 @@ int check_ws(void *ws, size_t ws_bytes, size_t need)
 template <int MODE>
 int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const void *q, const void *w_uv, int B,
                   int64_t L, int64_t m, int64_t win0, float scale, float *out, float *o_lat, int32_t *anchor,
-                  const DecodeWs &w, cudaStream_t st)
+                  const DecodeWs &w, cudaStream_t st, int64_t rep_stride = 0)
 {
     int rc = get_encode();
     if (rc) return rc;
@@ -289,8 +289,10 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
                    uint64_t(L) * LCA_D * 2, 64, AT_TILE, 1);
     if (rc) return rc;
     if (MODE == MODE_REPS && m > 0) {
+        // rows per sequence: m, or the capacity of a representative cache
+        const uint64_t stride_rows = uint64_t(rep_stride > 0 ? rep_stride : m);
         rc = make_map3(&map_rep, rep, LCA_D, uint64_t(m), uint64_t(B), uint64_t(LCA_D) * 2,
-                       uint64_t(m) * LCA_D * 2, 64, AT_TILE, 1);
+                       stride_rows * LCA_D * 2, 64, AT_TILE, 1);
         if (rc) return rc;
     } else {
         map_rep = map_cache;
@@ -408,12 +410,21 @@ int mla_decode_attn(const void *cache, const void *q, const void *w_uv, int B, i
 int lca_condense(const void *cache, const void *q_recent, int B, int64_t L, lca_params p, void *rep,
                  int32_t *anchor, float *alpha, void *ws, size_t ws_bytes, void *stream)
 {
+    const int64_t m = num_groups(L, p);
+    return lca_condense_append(cache, q_recent, B, L, p, 0, rep, m, anchor, alpha, ws, ws_bytes, stream);
+}
+
+int lca_condense_append(const void *cache, const void *q_recent, int B, int64_t L, lca_params p, int64_t j0,
+                        void *rep, int64_t rep_cap, int32_t *anchor, float *alpha, void *ws, size_t ws_bytes,
+                        void *stream)
+{
     if (!cache || !q_recent) return LCA_ERR_INVALID_ARG;
     if (B < 1 || L < 1 || L >= (int64_t(1) << 31)) return LCA_ERR_INVALID_ARG;
     if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
     if (p.g != 16) return LCA_ERR_UNSUPPORTED;
     const int64_t m = num_groups(L, p);
-    if (m > 0 && !rep) return LCA_ERR_INVALID_ARG;
+    if (j0 < 0 || j0 > m || rep_cap < m) return LCA_ERR_INVALID_ARG;
+    if (m > j0 && !rep) return LCA_ERR_INVALID_ARG;
     if (!aligned16(cache) || !aligned16(q_recent) || (rep && !aligned16(rep)) || (alpha && !aligned16(alpha)) ||
         (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
         return LCA_ERR_MISALIGNED;
@@ -423,14 +434,16 @@ int lca_condense(const void *cache, const void *q_recent, int B, int64_t L, lca_
     DeviceInfo *dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (m == 0) return LCA_OK;
+    if (m == j0) return LCA_OK;
     if ((rc = launch_prep(q_recent, B, p, w, st))) return rc;
     CondenseArgs a{};
     a.cache = static_cast<const uint16_t *>(cache);
     a.u = w.u;
     a.L = L;
-    a.m = m;
-    a.total = int64_t(B) * m;
+    a.m = m - j0;
+    a.j0 = j0;
+    a.stride = rep_cap;
+    a.total = int64_t(B) * a.m;
     a.rep = static_cast<uint16_t *>(rep);
     a.anchor = anchor;
     a.alpha = alpha;
@@ -439,6 +452,24 @@ int lca_condense(const void *cache, const void *q_recent, int B, int64_t L, lca_
     Launch l(st, K_CONDENSE);
     condense_kernel<<<grid, CD_WARPS * 32, CD_SMEM, st>>>(a);
     return l.done();
+}
+
+int lca_decode_stored(const void *cache, const void *rep, int64_t rep_cap, const void *q, const void *w_uv, int B,
+                      int64_t L, lca_params p, float *out, float *o_lat, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    const int64_t m = num_groups(L, p);
+    if (rep_cap < m || (m > 0 && !rep)) return LCA_ERR_INVALID_ARG;
+    if ((rep && !aligned16(rep)) || (o_lat && !aligned16(o_lat))) return LCA_ERR_MISALIGNED;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, nullptr, w,
+                                    static_cast<cudaStream_t>(stream), rep_cap);
 }
 
 int lca_decode_attn(const void *cache, const void *rep, const void *q, const void *w_uv, int B, int64_t L,
