@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stored", action="store_true",
+                    help="decode: stored-representative mode (groups condensed once and kept)")
     ap.add_argument("--mla-compare", type=int, default=0,
                     help="prefill: also time N full causal MLA prefills (w = L) on the same inputs")
     return ap.parse_args()
@@ -418,6 +420,126 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_ours_stored(args, rank, world, local_rank):
+    """Stored-representative decode: the representative cache is built once
+    (untimed); a step is lca_decode_stored, plus every 16th step the append of
+    one group per sequence (the rate at which groups leave the window).  The
+    rows a step reads ((m + w') x 1152 B per sequence) fit in L2 at these
+    sizes, so L2 is flushed before every step and steps are timed one by one."""
+    import torch.distributed as dist
+
+    import mla_latent_space_lca_b200 as lca
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    B, L = wl["B"], wl["L"]
+    inp = make_decode_inputs(B, L, seed=replica_seed(rank))
+    cache, q_recent, q, w_uv = (inp.cache.to(dev), inp.q_recent.to(dev), inp.q.to(dev),
+                                inp.w_uv.to(dev))
+    m = lca.num_groups(L)
+    rep = torch.empty(B, max(m, 1), 576, dtype=torch.bfloat16, device=dev)
+    ws = lca.workspace(3, B, L, device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    lca.lca_condense_append(cache, q_recent, rep, 0, scale=inp.scale, ws=ws, stream=stream)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        if i % 16 == 15 and m > 0:   # one group per sequence leaves the window every 16 steps
+            lca.lca_condense_append(cache, q_recent, rep, m - 1, scale=inp.scale, ws=ws, stream=stream)
+        lca.lca_decode_stored(cache, rep, q, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    barrier()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    n0 = lca.launch_count()
+    if sampler:
+        sampler.mark()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    launches = (lca.launch_count() - n0) / args.steps
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world, dev)
+    barrier()
+    if sampler:
+        sampler.stop()
+
+    # per-kernel times (events around each launch), L2 flushed before each step
+    lca.profile_enable(True)
+    prof_steps = min(args.steps, 160)
+    for i in range(prof_steps):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    prof = lca.profile_collect()
+    lca.profile_enable(False)
+
+    # end to end: the step's query and recent queries from pinned memory, out back
+    pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
+    h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
+    dbuf = [torch.empty_like(t, device=dev) for t in pin]
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    x0.record(stream)
+    n_e2e = max(1, args.e2e_steps)
+    for i in range(n_e2e):
+        for d, h in zip(dbuf, pin):
+            d.copy_(h, non_blocking=True)
+        lca.lca_decode_stored(cache, rep, dbuf[1], w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / n_e2e, world, dev)
+    rc, detail = lca.device_status(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    if rank != 0:
+        return
+    rows = m + (L - 16 * m)                     # kept representatives + window rows
+    read_bytes = B * rows * ROW_BYTES
+    peak, peak_kind = measured_hbm_peak()
+    attn = prof.get("attn_decode")
+    attn_ms = attn[1] / attn[0] if attn else None
+    achieved = read_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
+    line = {
+        "metric": METRIC, "value": B * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "mode": "stored representatives", "B_per_gpu": B, "L": L,
+                   "g": 16, "w": 1024, "kept_rows_per_seq": rows, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (256 MB write) before every step; steps timed one by one"},
+        "read_gbps": read_bytes * world / (ms / 1e3) / 1e9,
+        "kv_rows_read_fraction": rows / L,
+        "roofline": {"bound": "hbm", "kernel": "attn_decode (stored representatives)", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak if achieved else None, "traffic": None,
+                     "algorithmic_bytes_per_launch": read_bytes, "launch_ms": attn_ms},
+        "kernels_ms_per_step": {k: v[1] / prof_steps for k, v in prof.items()},
+        "gpu_launches": launches,
+        "clocks": sampler.summary() if sampler else None,
+        "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 4,
+                "note": "cache and representative cache resident on the device (a decode server's state)"},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours_prefill(args, rank, world, local_rank):
     import torch.distributed as dist
 
@@ -582,7 +704,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        (run_ours_prefill if prefill else run_ours)(args, rank, world, local_rank)
+        fn = run_ours_prefill if prefill else (run_ours_stored if args.stored else run_ours)
+        fn(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -310,9 +310,11 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     if (rc) return rc;
     {
         Launch l(st, K_COMBINE);
-        const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + TD_ROWS - 1) / TD_ROWS), dim3(256),
+        // rows per CTA: enough CTAs (16 heads x row groups) to cover the SMs
+        const int rpc = std::max(1, std::min(TD_ROWS, (LCA_HEADS * B + dev->sms - 1) / dev->sms));
+        const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + rpc - 1) / rpc), dim3(256),
                                         TD_SMEM_ALLOC, st, true, map_w, (const float *)w.part_o,
-                                        (const float *)w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out);
+                                        (const float *)w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out, rpc);
         if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     return LCA_OK;

@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(128, 1)
 // 128 output columns:
 //   out^T[128 x 16] = W_UV[h]^T[128 x 512] * o^T[512 x 16]
 // (N = 16: up to 8 batch rows per CTA, the rest zero).  Grid (16 heads,
-// ceil(B/8)), 256 threads.  W_UV[h] (128 KB, MN-major A) is TMA-loaded before
+// ceil(B/rpc)), 256 threads, rpc rows per CTA chosen by the host so that the
+// grid fills the GPU (fewer rows per CTA = more warps per row's slots).  W_UV[h] (128 KB, MN-major A) is TMA-loaded before
 // waiting on the attention kernel.  Combine: with nb rows, each row gets
 // 8/nb warps (at least one); a warp merges its share of the row's partial
 // slots online (rescaling on a new maximum, lanes own 16 of the 512 columns),
@@ -149,7 +150,7 @@ constexpr int TD_SMEM_ALLOC = TD_SMEM + 1024;
 __global__ void __launch_bounds__(256, 1)
     tail_decode_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
                        const float *__restrict__ part_ml, int B, int n_tiles, int64_t T, int G,
-                       float *__restrict__ o_lat, float *__restrict__ out)
+                       float *__restrict__ o_lat, float *__restrict__ out, int rpc)
 {
     extern __shared__ uint8_t td_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -157,8 +158,8 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t sbase = smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x;
-    const int b0 = blockIdx.y * TD_ROWS;
-    const int nb = min(TD_ROWS, B - b0);
+    const int b0 = blockIdx.y * rpc;           // rpc <= TD_ROWS rows (sequences) per CTA
+    const int nb = min(rpc, B - b0);
     const int wpr = max(1, TD_ROWS / nb);     // warps per row
     const uint32_t wbar = sbase + TD_OFF_BAR, accf = wbar + 8, drain0 = wbar + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TD_OFF_BAR + 128);
