@@ -47,8 +47,8 @@ def _load():
         lib.ora_num_threads.restype = I
         lib.ora_num_groups.restype = Lg
         lib.ora_num_groups.argtypes = [Lg, I, I]
-        lib.ora_lca_condense.restype = I
-        lib.ora_lca_condense.argtypes = [P, P, I, Lg, I, I, I, I, I, Dd, P, P, P, P, P]
+        lib.ora_lca_condense_v.restype = I
+        lib.ora_lca_condense_v.argtypes = [P, P, I, Lg, I, I, I, I, I, Dd, I, P, P, P, P, P]
         lib.ora_mla_decode.restype = I
         lib.ora_mla_decode.argtypes = [P, P, P, I, Lg, I, I, I, I, Dd, P, P]
         lib.ora_lca_decode.restype = I
@@ -83,7 +83,12 @@ def num_groups(L: int, g: int, w: int) -> int:
     return int(_load().ora_num_groups(L, g, w))
 
 
-def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64):
+# condensation variants: the method and the two ablations (pool the RoPE key
+# too; keep only the most important token)
+LCA, POOL_POSITION, SPARSE = 0, 1, 2
+
+
+def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64, variant: int = LCA):
     """cache [B,L,dc+dr] u16, q_recent [B,g,H,dc+dr] u16 ->
     dict(rep_c [B,m,dc], rep_k [B,m,dr], anchor [B,m] int32 (position in the
     sequence), alpha [B,m,g], score [B,m,g])."""
@@ -95,7 +100,7 @@ def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64):
     out = dict(rep_c=np.zeros((B, m, dc)), rep_k=np.zeros((B, m, dr)),
                anchor=np.zeros((B, m), np.int32), alpha=np.zeros((B, m, g)),
                score=np.zeros((B, m, g)))
-    _load().ora_lca_condense(_ptr(cache), _ptr(q_recent), B, L, H, dc, dr, g, w, scale,
+    _load().ora_lca_condense_v(_ptr(cache), _ptr(q_recent), B, L, H, dc, dr, g, w, scale, int(variant),
                              _ptr(out["rep_c"]), _ptr(out["rep_k"]), _ptr(out["anchor"]),
                              _ptr(out["alpha"]), _ptr(out["score"]))
     return out

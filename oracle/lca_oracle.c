@@ -88,13 +88,20 @@ static double importance(const double *qv, const uint16_t *row, int H, int dc, i
     return acc / H;
 }
 
+/* Condensation variants: the method (关键设计 1 + 2) and the two ablations of
+ * the page's 消融实验 table. */
+enum { ORA_LCA = 0, ORA_POOL_POSITION = 1, ORA_SPARSE = 2 };
+
 /* 关键设计 1 + 2 for one group of g rows starting at `rows`:
  * alpha = softmax(s) over the group, rep_c = sum_i alpha_i c_i,
  * I = argmax_i s_i (first index on an exact tie), rep_k = k^R_I.
+ * Ablations (消融实验): ORA_POOL_POSITION pools the RoPE key with the same
+ * weights, rep_k = sum_i alpha_i k^R_i ("纯池化（含位置）"); ORA_SPARSE keeps
+ * only the most important token, rep_c = c_I, rep_k = k^R_I ("纯稀疏").
  * Returns I (offset inside the group). */
-static int condense_group(const double *qv, const uint16_t *rows, int g, int H, int dc, int dr,
-                          double scale, double *rep_c, double *rep_k, double *alpha_out,
-                          double *score_out)
+static int condense_group_v(const double *qv, const uint16_t *rows, int g, int H, int dc, int dr,
+                            double scale, int variant, double *rep_c, double *rep_k,
+                            double *alpha_out, double *score_out)
 {
     int D = dc + dr;
     double *s = (double *)malloc(sizeof(double) * g);
@@ -109,10 +116,22 @@ static int condense_group(const double *qv, const uint16_t *rows, int g, int H, 
     for (int i = 0; i < g; i++) a[i] /= den;
     for (int k = 0; k < dc; k++) {
         double acc = 0.0;
-        for (int i = 0; i < g; i++) acc += a[i] * bf(rows[(size_t)i * D + k]);
+        if (variant == ORA_SPARSE) {
+            acc = bf(rows[(size_t)I * D + k]);
+        } else {
+            for (int i = 0; i < g; i++) acc += a[i] * bf(rows[(size_t)i * D + k]);
+        }
         rep_c[k] = acc;
     }
-    for (int k = 0; k < dr; k++) rep_k[k] = bf(rows[(size_t)I * D + dc + k]);
+    for (int k = 0; k < dr; k++) {
+        if (variant == ORA_POOL_POSITION) {
+            double acc = 0.0;
+            for (int i = 0; i < g; i++) acc += a[i] * bf(rows[(size_t)i * D + dc + k]);
+            rep_k[k] = acc;
+        } else {
+            rep_k[k] = bf(rows[(size_t)I * D + dc + k]);
+        }
+    }
     if (alpha_out) for (int i = 0; i < g; i++) alpha_out[i] = a[i];
     if (score_out) for (int i = 0; i < g; i++) score_out[i] = s[i];
     free(s);
@@ -120,13 +139,22 @@ static int condense_group(const double *qv, const uint16_t *rows, int g, int H, 
     return I;
 }
 
+static int condense_group(const double *qv, const uint16_t *rows, int g, int H, int dc, int dr,
+                          double scale, double *rep_c, double *rep_k, double *alpha_out,
+                          double *score_out)
+{
+    return condense_group_v(qv, rows, g, H, dc, dr, scale, ORA_LCA, rep_c, rep_k, alpha_out,
+                            score_out);
+}
+
 /* Condense every group of every sequence (decode: summary query from
  * q_recent).  Outputs (any may be NULL except none are required):
  * rep_c [B][m][dc], rep_k [B][m][dr], anchor [B][m] (absolute position
- * inside the sequence), alpha [B][m][g], score [B][m][g]. */
-int ora_lca_condense(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
-                     int dc, int dr, int g, int w, double scale, double *rep_c, double *rep_k,
-                     int32_t *anchor, double *alpha, double *score)
+ * inside the sequence), alpha [B][m][g], score [B][m][g].  `variant`
+ * selects the method or one of its ablations (condense_group_v). */
+int ora_lca_condense_v(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
+                       int dc, int dr, int g, int w, double scale, int variant, double *rep_c,
+                       double *rep_k, int32_t *anchor, double *alpha, double *score)
 {
     int D = dc + dr;
     long m = ora_num_groups(L, g, w);
@@ -144,8 +172,8 @@ int ora_lca_condense(const uint16_t *cache, const uint16_t *q_recent, int B, lon
         for (int b = 0; b < B; b++)
             for (long j = 0; j < m; j++) {
                 const uint16_t *rows = cache + ((size_t)b * L + (size_t)j * g) * D;
-                int I = condense_group(qbar + (size_t)b * H * D, rows, g, H, dc, dr, scale, rc,
-                                       rk, al, sc);
+                int I = condense_group_v(qbar + (size_t)b * H * D, rows, g, H, dc, dr, scale,
+                                         variant, rc, rk, al, sc);
                 size_t o = (size_t)b * m + j;
                 if (rep_c) memcpy(rep_c + o * dc, rc, sizeof(double) * dc);
                 if (rep_k) memcpy(rep_k + o * dr, rk, sizeof(double) * dr);
@@ -160,6 +188,14 @@ int ora_lca_condense(const uint16_t *cache, const uint16_t *q_recent, int B, lon
     }
     free(qbar);
     return 0;
+}
+
+int ora_lca_condense(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
+                     int dc, int dr, int g, int w, double scale, double *rep_c, double *rep_k,
+                     int32_t *anchor, double *alpha, double *score)
+{
+    return ora_lca_condense_v(cache, q_recent, B, L, H, dc, dr, g, w, scale, ORA_LCA, rep_c,
+                              rep_k, anchor, alpha, score);
 }
 
 /* 整体框架: standard attention of one query token (H heads, absorbed

@@ -388,3 +388,43 @@ def test_stored_anchors_are_frozen_exit_time_condensations(ora):
     _, _, a_re = ora.lca_decode(cache, np.ascontiguousarray(q_all[:, L - g:L]),
                                 np.ascontiguousarray(q_all[:, L - 1]), w_uv, g, w, 0.3, dr=4)
     assert not np.array_equal(a_re, a_now)
+
+
+# ----------------------------------------------------------------- ablations (消融实验)
+def test_ablation_pool_position_pools_the_key(ora):
+    """"纯池化（含位置）": the RoPE key is pooled with the same weights as the
+    latent.  Latent and anchor are the method's; with equal scores the pooled
+    key is the plain mean; in general it satisfies sum_i alpha_i (k_i - k_rep)
+    = 0 (the stationarity of 关键设计 1, here for k^R)."""
+    rng = np.random.default_rng(31)
+    cache, _, q_recent, _ = small_case(rng, B=2, L=45, g=4, peak=3.0)
+    g, w = 4, 5
+    base = ora.lca_condense(cache, q_recent, g, w, 0.3, dr=4)
+    pp = ora.lca_condense(cache, q_recent, g, w, 0.3, dr=4, variant=ora.POOL_POSITION)
+    assert np.array_equal(pp["rep_c"], base["rep_c"])
+    assert np.array_equal(pp["anchor"], base["anchor"])
+    kr = from_bits(cache)[..., 8:]
+    m = base["anchor"].shape[1]
+    groups = kr[:, :m * g].reshape(2, m, g, 4)
+    resid = np.einsum("bjg,bjgk->bjk", pp["alpha"], groups - pp["rep_k"][:, :, None, :])
+    np.testing.assert_allclose(resid, 0.0, atol=1e-13)
+    assert not np.allclose(pp["rep_k"], base["rep_k"])
+    zero = np.zeros_like(q_recent)
+    eq = ora.lca_condense(cache, zero, g, w, 0.3, dr=4, variant=ora.POOL_POSITION)
+    np.testing.assert_allclose(eq["rep_k"], groups.mean(axis=2), rtol=0, atol=1e-15)
+
+
+def test_ablation_sparse_keeps_the_anchor_row(ora):
+    """"纯稀疏": the representative is the most important token's own row."""
+    rng = np.random.default_rng(32)
+    cache, _, q_recent, _ = small_case(rng, B=2, L=45, g=4, peak=3.0)
+    g, w = 4, 5
+    base = ora.lca_condense(cache, q_recent, g, w, 0.3, dr=4)
+    sp = ora.lca_condense(cache, q_recent, g, w, 0.3, dr=4, variant=ora.SPARSE)
+    assert np.array_equal(sp["anchor"], base["anchor"])
+    rows = from_bits(cache)
+    for b in range(2):
+        for j, a in enumerate(sp["anchor"][b]):
+            assert np.array_equal(sp["rep_c"][b, j], rows[b, a, :8])
+            assert np.array_equal(sp["rep_k"][b, j], rows[b, a, 8:])
+    assert np.array_equal(sp["rep_k"], base["rep_k"])
