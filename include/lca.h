@@ -72,11 +72,24 @@ extern "C" {
 
 /* Condensation parameters.  g: group size (16; g = 1 makes every token its
  * own representative, which is exactly MLA).  w: local window (>= 0).
- * scale: logit scale (1/sqrt(192) for the 128+64 per-head MLA width). */
+ * scale: logit scale (1/sqrt(192) for the 128+64 per-head MLA width).
+ * variant: LCA_VARIANT_LCA (0) is the method; the other two are the
+ * ablations of the page's 消融实验 table, accepted by lca_condense and
+ * lca_condense_append only (other entry points that condense return
+ * LCA_ERR_UNSUPPORTED for them; the attention over stored representatives
+ * is the same for all three):
+ *   LCA_VARIANT_POOL_POSITION: the RoPE key is pooled with the same weights
+ *     as the latent, k_rep = sum_i alpha_i k^R_i ("纯池化（含位置）");
+ *   LCA_VARIANT_SPARSE: the representative is the most important token's row,
+ *     [c_I | k^R_I] ("纯稀疏"). */
+#define LCA_VARIANT_LCA 0
+#define LCA_VARIANT_POOL_POSITION 1
+#define LCA_VARIANT_SPARSE 2
 typedef struct {
     int g;
     int w;
     float scale;
+    int variant;
 } lca_params;
 
 /* Operation ids for lca_workspace_bytes. */

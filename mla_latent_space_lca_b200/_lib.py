@@ -23,6 +23,8 @@ LCA_ERR_SCRATCH_LIMIT = -8
 NOALLOC_MAX_BATCH = 8
 
 OP_MLA_DECODE, OP_CONDENSE, OP_DECODE_ATTN, OP_DECODE, OP_PREFILL = range(5)
+# condensation variants: the method, and the two ablations
+VARIANT_LCA, VARIANT_POOL_POSITION, VARIANT_SPARSE = range(3)
 
 # every symbol include/lca.h declares
 EXPORTS = ("lca_num_groups", "lca_workspace_bytes", "mla_decode_attn", "lca_condense",
@@ -32,7 +34,8 @@ EXPORTS = ("lca_num_groups", "lca_workspace_bytes", "mla_decode_attn", "lca_cond
 
 
 class LcaParams(ctypes.Structure):
-    _fields_ = [("g", ctypes.c_int), ("w", ctypes.c_int), ("scale", ctypes.c_float)]
+    _fields_ = [("g", ctypes.c_int), ("w", ctypes.c_int), ("scale", ctypes.c_float),
+                ("variant", ctypes.c_int)]
 
 
 class KernelTime(ctypes.Structure):

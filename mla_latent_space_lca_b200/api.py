@@ -23,8 +23,8 @@ def default_scale() -> float:
     return 1.0 / math.sqrt(192.0)
 
 
-def _params(g: int, w: int, scale: float | None) -> LcaParams:
-    return LcaParams(int(g), int(w), float(default_scale() if scale is None else scale))
+def _params(g: int, w: int, scale: float | None, variant: int = 0) -> LcaParams:
+    return LcaParams(int(g), int(w), float(default_scale() if scale is None else scale), int(variant))
 
 
 def _ptr(t):
@@ -76,7 +76,7 @@ def mla_decode_attn(cache, q, w_uv, scale=None, out=None, o_lat=None, ws=None, s
 
 
 def lca_condense(cache, q_recent, g=16, w=1024, scale=None, rep=None, anchor=None, alpha=None,
-                 ws=None, stream=None):
+                 ws=None, stream=None, variant=0):
     B, L, _ = cache.shape
     _need(cache, "cache", torch.bfloat16, (B, L, D))
     _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
@@ -84,7 +84,7 @@ def lca_condense(cache, q_recent, g=16, w=1024, scale=None, rep=None, anchor=Non
     dev = cache.device
     rep = torch.empty(B, m, D, dtype=torch.bfloat16, device=dev) if rep is None else rep
     ws = workspace(_lib.OP_CONDENSE, B, L, g=g, w=w, device=dev) if ws is None else ws
-    rc = _lib.lib().lca_condense(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale),
+    rc = _lib.lib().lca_condense(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale, variant),
                                  _ptr(rep) if m > 0 else None, _ptr(anchor), _ptr(alpha), _ptr(ws),
                                  ws.numel(), _stream(stream))
     check(rc, "lca_condense")
@@ -110,7 +110,7 @@ def lca_decode_attn(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
 
 
 def lca_condense_append(cache, q_recent, rep, j0, g=16, w=1024, scale=None, anchor=None, alpha=None,
-                        ws=None, stream=None):
+                        ws=None, stream=None, variant=0):
     """Condense groups j0 .. m-1 into rows j0 .. of the representative cache
     rep [B, rep_cap, 576] (bf16); returns m, the number of groups now held."""
     B, L, _ = cache.shape
@@ -121,7 +121,7 @@ def lca_condense_append(cache, q_recent, rep, j0, g=16, w=1024, scale=None, anch
         raise ValueError(f"rep has shape {tuple(rep.shape)}, expected ({B}, rep_cap, {D})")
     m = num_groups(L, g, w)
     ws = workspace(_lib.OP_CONDENSE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
-    rc = _lib.lib().lca_condense_append(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale), int(j0),
+    rc = _lib.lib().lca_condense_append(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale, variant), int(j0),
                                         _ptr(rep), rep.shape[1], _ptr(anchor), _ptr(alpha), _ptr(ws),
                                         ws.numel(), _stream(stream))
     check(rc, "lca_condense_append")

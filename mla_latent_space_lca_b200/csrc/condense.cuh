@@ -13,6 +13,9 @@
 //   alpha = softmax(s)          (shuffle max / sum over the 16 tokens)
 //   I     = first argmax s      (shuffle reduction on (s, index))
 //   rep   = [sum_i alpha_i c_i (fp32 accumulate, bf16 store) | k^R_I (bit copy)]
+// The ablations of the page's 消融实验 table replace the last step:
+// LCA_VARIANT_POOL_POSITION pools k^R with the same alpha too, and
+// LCA_VARIANT_SPARSE stores the anchor token's whole row.
 #pragma once
 #include "common.cuh"
 
@@ -34,6 +37,7 @@ struct CondenseArgs {
     uint16_t *rep;           // [B][stride][576], rows j0 .. j0+m-1 written
     int32_t *anchor;         // [B][stride] or NULL
     float *alpha;            // [B][stride][16] or NULL
+    int variant;             // LCA_VARIANT_*: the method or one of its ablations
 };
 
 __device__ __forceinline__ float dot8(const uint4 x, const float *u)
@@ -163,42 +167,54 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
         for (int off = 2; off <= 16; off <<= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
         const float al = e / den;
 
-        // pooled latent: lane owns 16-byte slices lane and lane+32 of c
-        float pa[2][8];
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) pa[r][k] = 0.f;
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const float ai = __shfl_sync(0xffffffffu, al, 2 * i);
-            const uint8_t *row = tile + i * (LCA_D * 2);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const uint4 x = *reinterpret_cast<const uint4 *>(row + (lane + 32 * r) * 16);
-                pa[r][0] = fmaf(ai, bf_lo(x.x), pa[r][0]);
-                pa[r][1] = fmaf(ai, bf_hi(x.x), pa[r][1]);
-                pa[r][2] = fmaf(ai, bf_lo(x.y), pa[r][2]);
-                pa[r][3] = fmaf(ai, bf_hi(x.y), pa[r][3]);
-                pa[r][4] = fmaf(ai, bf_lo(x.z), pa[r][4]);
-                pa[r][5] = fmaf(ai, bf_hi(x.z), pa[r][5]);
-                pa[r][6] = fmaf(ai, bf_lo(x.w), pa[r][6]);
-                pa[r][7] = fmaf(ai, bf_hi(x.w), pa[r][7]);
-            }
-        }
         uint16_t *dst = a.rep + (size_t(b) * a.stride + size_t(j)) * LCA_D;
+        const uint8_t *arow = tile + bi * (LCA_D * 2);   // the anchor token's row
+        if (a.variant == LCA_VARIANT_SPARSE) {
+            // ablation "纯稀疏": the representative is the anchor token's row
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            uint4 o;
-            o.x = pack_bf16(pa[r][0], pa[r][1]);
-            o.y = pack_bf16(pa[r][2], pa[r][3]);
-            o.z = pack_bf16(pa[r][4], pa[r][5]);
-            o.w = pack_bf16(pa[r][6], pa[r][7]);
-            reinterpret_cast<uint4 *>(dst)[lane + 32 * r] = o;
-        }
-        if (lane < 8) {
-            const uint4 k = *reinterpret_cast<const uint4 *>(tile + bi * (LCA_D * 2) + LCA_DC * 2 + lane * 16);
-            reinterpret_cast<uint4 *>(dst + LCA_DC)[lane] = k;
+            for (int r = 0; r < 2; ++r)
+                reinterpret_cast<uint4 *>(dst)[lane + 32 * r] = *reinterpret_cast<const uint4 *>(arow + (lane + 32 * r) * 16);
+            if (lane < 8)
+                reinterpret_cast<uint4 *>(dst + LCA_DC)[lane] = *reinterpret_cast<const uint4 *>(arow + LCA_DC * 2 + lane * 16);
+        } else {
+            // pooled latent: lane owns 16-byte slices lane and lane+32 of c;
+            // with LCA_VARIANT_POOL_POSITION lanes 0-7 also pool slice 64+lane (k^R)
+            const bool pool_key = a.variant == LCA_VARIANT_POOL_POSITION;
+            float pa[3][8];
+#pragma unroll
+            for (int r = 0; r < 3; ++r)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) pa[r][k] = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const float ai = __shfl_sync(0xffffffffu, al, 2 * i);
+                const uint8_t *row = tile + i * (LCA_D * 2);
+#pragma unroll
+                for (int r = 0; r < 3; ++r) {
+                    if (r == 2 && !(pool_key && lane < 8)) continue;
+                    const uint4 x = *reinterpret_cast<const uint4 *>(row + (lane + 32 * r) * 16);
+                    pa[r][0] = fmaf(ai, bf_lo(x.x), pa[r][0]);
+                    pa[r][1] = fmaf(ai, bf_hi(x.x), pa[r][1]);
+                    pa[r][2] = fmaf(ai, bf_lo(x.y), pa[r][2]);
+                    pa[r][3] = fmaf(ai, bf_hi(x.y), pa[r][3]);
+                    pa[r][4] = fmaf(ai, bf_lo(x.z), pa[r][4]);
+                    pa[r][5] = fmaf(ai, bf_hi(x.z), pa[r][5]);
+                    pa[r][6] = fmaf(ai, bf_lo(x.w), pa[r][6]);
+                    pa[r][7] = fmaf(ai, bf_hi(x.w), pa[r][7]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 3; ++r) {
+                if (r == 2 && !(pool_key && lane < 8)) continue;
+                uint4 o;
+                o.x = pack_bf16(pa[r][0], pa[r][1]);
+                o.y = pack_bf16(pa[r][2], pa[r][3]);
+                o.z = pack_bf16(pa[r][4], pa[r][5]);
+                o.w = pack_bf16(pa[r][6], pa[r][7]);
+                reinterpret_cast<uint4 *>(dst)[lane + 32 * r] = o;
+            }
+            if (!pool_key && lane < 8)   // 关键设计 2: the anchor's key, bit for bit
+                reinterpret_cast<uint4 *>(dst + LCA_DC)[lane] = *reinterpret_cast<const uint4 *>(arow + LCA_DC * 2 + lane * 16);
         }
         const size_t gidx = size_t(b) * a.stride + size_t(j);
         if (a.anchor && lane == 0) a.anchor[gidx] = int32_t(j * 16 + bi);

@@ -236,7 +236,11 @@ PrefillWs prefill_ws_layout(void *ws, int B, int64_t nb, int64_t m_bound)
     return w;
 }
 
-bool params_ok(const lca_params &p) { return p.g >= 1 && p.w >= 0 && std::isfinite(p.scale) && p.scale > 0.f; }
+bool params_ok(const lca_params &p)
+{
+    return p.g >= 1 && p.w >= 0 && std::isfinite(p.scale) && p.scale > 0.f && p.variant >= LCA_VARIANT_LCA &&
+           p.variant <= LCA_VARIANT_SPARSE;
+}
 
 int64_t num_groups(int64_t L, const lca_params &p)
 {
@@ -449,6 +453,7 @@ int lca_condense_append(const void *cache, const void *q_recent, int B, int64_t 
     a.rep = static_cast<uint16_t *>(rep);
     a.anchor = anchor;
     a.alpha = alpha;
+    a.variant = p.variant;
     const int64_t want = (a.total + CD_WARPS - 1) / CD_WARPS;
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(dev->sms, want)));
     Launch l(st, K_CONDENSE);
@@ -498,6 +503,7 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
     if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;   // ablations: lca_condense + lca_decode_attn
     if (p.g == 1) return mla_decode_attn(cache, q, w_uv, B, L, p.scale, out, o_lat, ws, ws_bytes, stream);
     if (p.g != 16) return LCA_ERR_UNSUPPORTED;
     if (!q_recent) return LCA_ERR_INVALID_ARG;
@@ -519,6 +525,7 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
     if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
     if (B > LCA_NOALLOC_MAX_BATCH) return LCA_ERR_SCRATCH_LIMIT;
     if (p.g != 1 && p.g != 16) return LCA_ERR_UNSUPPORTED;
     if (p.g != 1 && !q_recent) return LCA_ERR_INVALID_ARG;
@@ -546,7 +553,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
     if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
-    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    if (p.g != 16 || p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
     if (q_start < 0 || q_len < 0 || q_start % 16 || q_len % 16 || q_start + q_len > L) return LCA_ERR_INVALID_ARG;
     if (L > (int64_t(1) << 27)) return LCA_ERR_UNSUPPORTED;   // query rows 16 L index a TMA map
     if ((o_lat && !aligned16(o_lat)) || (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))

@@ -72,6 +72,9 @@ def call_decode(lcalib, **kw):
     (dict(p=LcaParams(16, 1024, 0.0)), _lib.LCA_ERR_INVALID_ARG),
     (dict(p=LcaParams(16, 1024, float("nan"))), _lib.LCA_ERR_INVALID_ARG),
     (dict(p=LcaParams(8, 1024, 0.07)), _lib.LCA_ERR_UNSUPPORTED),
+    (dict(p=LcaParams(16, 1024, 0.07, 3)), _lib.LCA_ERR_INVALID_ARG),
+    (dict(p=LcaParams(16, 1024, 0.07, _lib.VARIANT_SPARSE)), _lib.LCA_ERR_UNSUPPORTED),
+    (dict(p=LcaParams(16, 1024, 0.07, _lib.VARIANT_POOL_POSITION)), _lib.LCA_ERR_UNSUPPORTED),
     (dict(cache=A + 8), _lib.LCA_ERR_MISALIGNED),
     (dict(o_lat=A + 4), _lib.LCA_ERR_MISALIGNED),
     (dict(anchor=A + 2), _lib.LCA_ERR_MISALIGNED),
@@ -94,6 +97,14 @@ def test_other_entry_points_reject_bad_arguments(lcalib):
     assert lcalib.lca_condense(A, A, 1, 4096, p, A + 2, None, None, A, big, None) == _lib.LCA_ERR_MISALIGNED
     assert lcalib.lca_decode_attn(A, None, A, A, 1, 4096, p, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
     assert lcalib.lca_decode_attn(A, A, A, A, 1, 4096, p, A, None, A, 16, None) == _lib.LCA_ERR_WORKSPACE
+    # stored representatives: capacity below m, j0 past m
+    assert lcalib.lca_condense_append(A, A, 1, 4096, p, 0, A, 100, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.lca_condense_append(A, A, 1, 4096, p, 193, A, 192, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.lca_decode_stored(A, A, 100, A, A, 1, 4096, p, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    # ablation variants: prefill and the no-alloc decode condense, so they refuse them
+    pv = LcaParams(16, 1024, 0.07, _lib.VARIANT_SPARSE)
+    assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 0, 4096, pv, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
+    assert lcalib.lca_decode_noalloc(A, A, A, A, 1, 4096, pv, A, None, None, None) == _lib.LCA_ERR_UNSUPPORTED
 
 
 def test_valid_call_without_gpu_reports_no_device(lcalib):

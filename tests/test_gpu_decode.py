@@ -128,6 +128,38 @@ def test_condense_parity(B, L, peak):
     assert same.mean() > 0.99
 
 
+@pytest.mark.parametrize("variant", [1, 2])
+def test_condense_ablation_variants(variant):
+    """The two ablations of the page's 消融实验 table: pooling the RoPE key
+    too (1) and keeping only the most important token's row (2); then the
+    attention over those representatives."""
+    B, L = 2, 1024 + 16 * 90 + 3
+    inp = make_decode_inputs(B, L, seed=260 + variant, peak=10.0)
+    cache, q_recent, q, w_uv = dev(inp)
+    m = api.num_groups(L)
+    anchor = torch.full((B, m), -1, dtype=torch.int32, device="cuda")
+    rep = api.lca_condense(cache, q_recent, scale=inp.scale, anchor=anchor, variant=variant)
+    o_lat = torch.empty(B, 16, 512, device="cuda")
+    out = api.lca_decode_attn(cache, rep, q, w_uv, scale=inp.scale, o_lat=o_lat)
+    torch.cuda.synchronize()
+    c, qr, qb, wb = bits(inp)
+    r = oracle.lca_condense(c, qr, 16, 1024, inp.scale, variant=variant)
+    ga = anchor.cpu().numpy()
+    check_anchors(ga, r["anchor"], r["score"])
+    same = ga == r["anchor"]
+    rep_bits = rep.view(torch.int16).cpu().numpy().view(np.uint16)
+    rows = c[np.arange(B)[:, None], ga]                 # the GPU's anchor rows
+    if variant == 2:
+        assert np.array_equal(rep_bits, rows)           # whole row, bit for bit
+    else:
+        rep_f = rep.float().cpu().numpy()
+        compare(rep_f[:, :, :512][same], r["rep_c"][same], "rep_c (pool position)")
+        compare(rep_f[:, :, 512:][same], r["rep_k"][same], "rep_k (pooled)")
+    ol_ref, out_ref = oracle.lca_attend_reps(c, rep_bits, qb, wb, 16, 1024, inp.scale)
+    compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
+    compare(out.cpu().numpy(), out_ref, "out")
+
+
 # ---------------------------------------------------------------- attention over stored reps
 @pytest.mark.parametrize("B,L", [(2, 4096), (3, 1024 + 16 * 70 + 9), (2, 1040), (2, 700)])
 def test_decode_attn_over_stored_reps(B, L):
