@@ -143,7 +143,8 @@ constexpr int TD_BCHUNK = TD_N * 128;                   // 2048 per 64-k chunk
 constexpr int TD_OFF_B = TD_A;                          // 8 chunks = 16 KB
 constexpr int TD_OFF_SCR = TD_OFF_B + 8 * TD_BCHUNK;    // 147456
 constexpr int TD_SCR_STRIDE = LCA_DC + 4;               // floats per warp state
-constexpr int TD_OFF_BAR = TD_OFF_SCR + 8 * TD_SCR_STRIDE * 4;
+constexpr int TD_OFF_COEF = TD_OFF_SCR + 8 * TD_SCR_STRIDE * 4;   // [TD_ROWS][8] warp weights
+constexpr int TD_OFF_BAR = TD_OFF_COEF + TD_ROWS * 8 * 4;
 constexpr int TD_SMEM = TD_OFF_BAR + 256;
 constexpr int TD_SMEM_ALLOC = TD_SMEM + 1024;
 
@@ -219,12 +220,12 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                 for (int off = 16; off; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
                 const float Mn = fmaxf(M, Mc);
-                const float sc = exp2f(M - Mn);   // rescale the earlier chunks (0 at first)
+                const float sc = fast_exp2(M - Mn);   // rescale the earlier chunks (0 at first)
                 den *= sc;
 #pragma unroll
                 for (int e = 0; e < 16; ++e) acc[e] *= sc;
                 M = Mn;
-                const float wl = (lane < cnt) ? exp2f(m - M) : 0.f;
+                const float wl = (lane < cnt) ? fast_exp2(m - M) : 0.f;
                 float dl = wl * l;
 #pragma unroll
                 for (int off = 16; off; off >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, off);
@@ -257,25 +258,35 @@ __global__ void __launch_bounds__(256, 1)
         }
     }
     __syncthreads();
+    // ---- per row: the warps' common max, the denominator and each warp's
+    // weight, once (thread r handles row r)
+    float *coef = reinterpret_cast<float *>(smem + TD_OFF_COEF);
+    if (threadIdx.x < nb) {
+        const int r = threadIdx.x;
+        float Mt = -INFINITY;
+        for (int i = 0; i < wpr; ++i) Mt = fmaxf(Mt, scr[(r * wpr + i) * TD_SCR_STRIDE + LCA_DC]);
+        float dt = 0.f;
+        for (int i = 0; i < wpr; ++i) {
+            const float *wp = scr + (r * wpr + i) * TD_SCR_STRIDE;
+            const float f = (wp[LCA_DC] == -INFINITY) ? 0.f : fast_exp2(wp[LCA_DC] - Mt);
+            coef[r * 8 + i] = f;
+            dt = fmaf(f, wp[LCA_DC + 1], dt);
+        }
+        const float inv = 1.f / dt;
+        for (int i = 0; i < wpr; ++i) coef[r * 8 + i] *= inv;
+    }
+    __syncthreads();
     // ---- merge the warps of each row; o -> o_lat (fp32) and the B operand (bf16)
     for (int r = 0; r < TD_N; ++r) {
         const int k = 2 * threadIdx.x;   // 256 threads x 2 columns
         float o0 = 0.f, o1 = 0.f;
         if (r < nb) {
-            float Mt = -INFINITY;
-            for (int w = r * wpr; w < (r + 1) * wpr; ++w) Mt = fmaxf(Mt, scr[w * TD_SCR_STRIDE + LCA_DC]);
-            float dt = 0.f;
-            for (int w = r * wpr; w < (r + 1) * wpr; ++w) {
-                const float *wp = scr + w * TD_SCR_STRIDE;
-                const float Mw = wp[LCA_DC];
-                const float f = (Mw == -INFINITY) ? 0.f : exp2f(Mw - Mt);
-                dt = fmaf(f, wp[LCA_DC + 1], dt);
-                o0 = fmaf(f, wp[k], o0);
-                o1 = fmaf(f, wp[k + 1], o1);
+            for (int i = 0; i < wpr; ++i) {
+                const float c = coef[r * 8 + i];
+                const float2 x = *reinterpret_cast<const float2 *>(scr + (r * wpr + i) * TD_SCR_STRIDE + k);
+                o0 = fmaf(c, x.x, o0);
+                o1 = fmaf(c, x.y, o1);
             }
-            const float inv = 1.f / dt;
-            o0 *= inv;
-            o1 *= inv;
             if (o_lat)
                 *reinterpret_cast<float2 *>(o_lat + (size_t(b0 + r) * LCA_HEADS + h) * LCA_DC + k) =
                     make_float2(o0, o1);
