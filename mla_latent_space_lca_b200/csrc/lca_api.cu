@@ -212,7 +212,7 @@ constexpr int64_t kPrefillChunk = 256;
 
 struct PrefillWs {
     uint16_t *uhl;      // [B * nb][2][576]
-    uint16_t *rep;      // [4 ceil(m_bound / 4)][chunk blocks][576]
+    uint16_t *rep;      // [CP_G ceil(m_bound / CP_G)][chunk blocks][576]
     uint16_t *o_bf16;   // [chunk blocks * 16][16][512]
     size_t bytes;
 };
@@ -224,7 +224,8 @@ PrefillWs prefill_ws_layout(void *ws, int B, int64_t nb, int64_t m_bound)
     size_t off[4];
     off[0] = 0;
     off[1] = off[0] + align_up(size_t(B) * size_t(nb) * 2 * LCA_D * 2);
-    off[2] = off[1] + align_up(size_t(nbc) * size_t(4 * std::max<int64_t>((m_bound + 3) / 4, 1)) * LCA_D * 2);
+    off[2] = off[1] + align_up(size_t(nbc) * size_t(CP_G * std::max<int64_t>((m_bound + CP_G - 1) / CP_G, 1)) *
+                               LCA_D * 2);
     off[3] = off[2] + align_up(size_t(nbc) * 16 * LCA_HEADS * LCA_DC * 2);
     w.bytes = off[3];
     if (ws) {
@@ -570,9 +571,13 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *qv = static_cast<const uint16_t *>(q);
 
-    CUtensorMap map_cache, map_q, map_u, map_w;
+    CUtensorMap map_cache, map_rows, map_q, map_u, map_w;
     if ((rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
                         uint64_t(L) * LCA_D * 2, 64, 64, 1)))
+        return rc;
+    // the condensation's history tiles: CP_ROWS rows
+    if ((rc = make_map3(&map_rows, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
+                        uint64_t(L) * LCA_D * 2, 64, CP_ROWS, 1)))
         return rc;
     if ((rc = make_map3(&map_q, q, LCA_D, uint64_t(L) * LCA_HEADS, uint64_t(B), uint64_t(LCA_D) * 2,
                         uint64_t(L) * LCA_HEADS * LCA_D * 2, 64, 64, 1)))
@@ -596,11 +601,11 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     for (int b = 0; b < B; ++b) {
         for (int64_t kc0 = k0; kc0 < k0 + nb; kc0 += kPrefillChunk) {
             const int nbc = int(std::min<int64_t>(kPrefillChunk, k0 + nb - kc0));
-            const int n_gt = int((pf_groups(kc0 + nbc - 1, cw) + 3) / 4);   // group tiles of the chunk
+            const int n_gt = int((pf_groups(kc0 + nbc - 1, cw) + CP_G - 1) / CP_G);   // group tiles of the chunk
             CUtensorMap map_rep = map_cache;
             if (n_gt > 0) {
-                // group-major [4 n_gt][nbc][576]; a box is 64 groups of one block
-                if ((rc = make_map3(&map_rep, w.rep, LCA_D, uint64_t(nbc), uint64_t(4 * n_gt), uint64_t(LCA_D) * 2,
+                // group-major [CP_G n_gt][nbc][576]; a box is 64 groups of one block
+                if ((rc = make_map3(&map_rep, w.rep, LCA_D, uint64_t(nbc), uint64_t(CP_G) * n_gt, uint64_t(LCA_D) * 2,
                                     uint64_t(nbc) * LCA_D * 2, 64, 1, 64)))
                     return rc;
                 CondPreArgs c{};
@@ -617,7 +622,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
                 const int n_bt = (nbc + 127) / 128;
                 Launch l(st, K_PREFILL_CONDENSE);
                 const cudaError_t e = launch_ex(condense_prefill_kernel, dim3(unsigned(n_bt * c.n_gt)),
-                                                dim3(CP_THREADS), CP_SMEM_ALLOC, st, false, map_cache, map_u, c);
+                                                dim3(CP_THREADS), CP_SMEM_ALLOC, st, false, map_rows, map_u, c);
                 if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
             }
             const size_t row_out = size_t(b) * size_t(q_len) + size_t(16 * (kc0 - k0));   // first output row

@@ -14,14 +14,14 @@
 // attention pass would re-read each raw history row once per block.  Instead
 // a chunk of blocks is condensed into a workspace first:
 //
-//   condense_prefill_kernel: one CTA per (128 blocks, 4 groups = 64 rows).
-//     S [128 blocks x 64 rows] = U_hi * R^T + U_lo * R^T (two MMA chains,
-//     M = 128, N = 64, K = 576; u = u_hi + u_lo is the folded summary query in
-//     two bf16 halves), a per-lane group softmax / first-index argmax
-//     (TMEM lane = block), then the pooling itself on the tensor cores:
-//     rep_j [128 blocks x 512] = alpha_j [128 x 16] * C_j [16 x 512]
-//     (K = 16, four N = 128 MMAs per group through three TMEM buffers), the
-//     anchor's RoPE key copied bit for bit.  Every (group < 4 n_gt, block)
+//   condense_prefill_kernel: one CTA per (128 blocks, 2 groups = 32 rows),
+//     two CTAs per SM.  S [128 blocks x 32 rows] = U_hi * R^T + U_lo * R^T
+//     (two MMA chains, M = 128, N = 32, K = 576; u = u_hi + u_lo is the
+//     folded summary query in two bf16 halves), a per-lane group softmax /
+//     first-index argmax (TMEM lane = block), then the pooling itself on the
+//     tensor cores: rep_j [128 blocks x 512] = alpha_j [128 x 16] * C_j [16 x 512]
+//     (K = 16, four N = 128 MMAs per group through one TMEM buffer), the
+//     anchor's RoPE key copied bit for bit.  Every (group < 2 n_gt, block)
 //     entry of the chunk is written, so the rows the attention masks out are
 //     finite.  Outputs leave through a per-warp shared-memory transpose, so
 //     each store instruction writes whole 256-byte row segments.  Bound: the
@@ -49,36 +49,48 @@ namespace lca {
 __host__ __device__ __forceinline__ int64_t pf_groups(int64_t k, int cw) { return k > cw ? k - cw : 0; }
 
 // ====================================================================== condense
+// One task = 128 blocks x CP_G groups (16 CP_G history rows); two CTAs share
+// an SM, so one CTA's loads, importance MMAs and softmax overlap the other's
+// HBM-bound output drains.
 constexpr int CP_THREADS = 224;                 // 7 warps
-constexpr int CP_BOX = 8192;                    // [64 rows x 64 cols] bf16
-constexpr int CP_R = 9 * CP_BOX;                // the 64 history rows, 73728 B
+constexpr int CP_G = 2;                         // groups per task
+constexpr int CP_ROWS = 16 * CP_G;              // history rows per task
+constexpr int CP_BOX = CP_ROWS * 128;           // [CP_ROWS rows x 64 cols] bf16
+constexpr int CP_R = 9 * CP_BOX;                // the task's rows, 36 KB
 constexpr int CP_UBOX = 16384;                  // [128 blocks x 64 cols] bf16
-constexpr int CP_USTAGES = 3;
-constexpr int CP_OFF_U = CP_R;
-constexpr int CP_OFF_A = CP_OFF_U + CP_USTAGES * 2 * CP_UBOX;   // alpha [128 x 64] bf16
-constexpr int CP_OFF_BAR = CP_OFF_A + CP_UBOX;
-constexpr int CP_OFF_MISC = CP_OFF_BAR + 8 * 20;
+constexpr int CP_USTAGES = 2;
+constexpr int CP_OFF_U = CP_R;                  // U ring; once S is done: alpha + staging
+constexpr int CP_OFF_BAR = CP_OFF_U + CP_USTAGES * 2 * CP_UBOX;
+constexpr int CP_OFF_MISC = CP_OFF_BAR + 8 * 16;
 constexpr int CP_SMEM = CP_OFF_MISC + 64;
 constexpr int CP_SMEM_ALLOC = CP_SMEM + 1024;
-constexpr uint32_t CP_TM_S = 0;                 // S_hi 0..63, S_lo 64..127
-constexpr uint32_t CP_TM_P = 128;               // 3 pooling buffers of 128 columns
-constexpr uint32_t CP_TM_COLS = 512;
+// after the importance MMAs, the U ring holds: alpha [128 x 64] bf16 (16 KB,
+// the first 16 CP_G columns used), then per drain warp 32 rows x 256 B of
+// latent and 32 rows x 128 B of RoPE key staging
+constexpr int CP_OFF_ALPHA = CP_OFF_U;
+constexpr int CP_OFF_STG_LAT = CP_OFF_ALPHA + 16384;
+constexpr int CP_OFF_STG_ROPE = CP_OFF_STG_LAT + 4 * 8192;
+static_assert(CP_OFF_STG_ROPE + 4 * 4096 <= CP_OFF_U + CP_USTAGES * 2 * CP_UBOX, "staging exceeds the U ring");
+static_assert(2 * (CP_SMEM_ALLOC + 1024) <= 228 * 1024, "two CTAs must fit an SM");
+constexpr uint32_t CP_TM_S = 0;                 // S_hi, S_lo: CP_ROWS columns each
+constexpr uint32_t CP_TM_P = 128;               // one pooling buffer of 128 columns
+constexpr uint32_t CP_TM_COLS = 256;
 
 struct CondPreArgs {
     int64_t kc0;       // first block of the chunk (block k = queries 16k .. 16k+15)
     int nbc;           // blocks in the chunk
     int cw;            // ceil(w / 16)
     int b;             // sequence
-    int n_gt;          // group tiles per block tile (grid = block tiles x n_gt)
+    int n_gt;          // group tiles (of CP_G groups) per block tile (grid = block tiles x n_gt)
     int ublk0;         // row of block kc0 in the summary-query array
-    uint16_t *rep;     // the chunk's representatives, group-major [4 n_gt][nbc][576]
+    uint16_t *rep;     // the chunk's representatives, group-major [CP_G n_gt][nbc][576]
     int64_t k0;        // first block of the call (anchor rows)
     int64_t m_ld;      // anchor row length
     int32_t *anchor;   // this sequence's anchor rows [(k - k0)][m_ld], or NULL
 };
 
-__global__ void __launch_bounds__(CP_THREADS, 1)
-    condense_prefill_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_u,
+__global__ void __launch_bounds__(CP_THREADS, 2)
+    condense_prefill_kernel(const __grid_constant__ CUtensorMap map_rows, const __grid_constant__ CUtensorMap map_u,
                             const CondPreArgs a)
 {
     const int bt = blockIdx.x / a.n_gt, gt = blockIdx.x - bt * a.n_gt;
@@ -92,24 +104,23 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     auto BAR = [&](int i) -> uint32_t { return sbase + CP_OFF_BAR + 8 * i; };
-    const uint32_t rfull = BAR(0), sfull = BAR(7), aready = BAR(8), drain5 = BAR(15), drain6 = BAR(16);
+    const uint32_t rfull = BAR(0), sfull = BAR(5), aready = BAR(6), pfull = BAR(7), pempty = BAR(8),
+                   drain5 = BAR(9), drain6 = BAR(10);
     auto ufull = [&](int s) { return BAR(1 + s); };
-    auto uempty = [&](int s) { return BAR(4 + s); };
-    auto pfull = [&](int s) { return BAR(9 + s); };
-    auto pempty = [&](int s) { return BAR(12 + s); };
+    auto uempty = [&](int s) { return BAR(3 + s); };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + CP_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + CP_OFF_MISC + 4);
 
     if (threadIdx.x == 0) {
         mbar_init(rfull, 1);
-        for (int s = 0; s < 3; ++s) {
+        for (int s = 0; s < CP_USTAGES; ++s) {
             mbar_init(ufull(s), 1);
             mbar_init(uempty(s), 2);     // both importance chains
-            mbar_init(pfull(s), 1);
-            mbar_init(pempty(s), 4);     // four drain warps
         }
         mbar_init(sfull, 2);
         mbar_init(aready, 4);
+        mbar_init(pfull, 1);
+        mbar_init(pempty, 4);            // four drain warps
         mbar_init(drain5, 1);
         mbar_init(drain6, 1);
         *abort_flag = 0;
@@ -123,24 +134,24 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t rbase = sbase, ubase = sbase + CP_OFF_U, abase = sbase + CP_OFF_A;
+    const uint32_t rbase = sbase, ubase = sbase + CP_OFF_U, abase = sbase + CP_OFF_ALPHA;
 
     if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            prefetch_tensormap(&map_cache);
+            prefetch_tensormap(&map_rows);
             prefetch_tensormap(&map_u);
             const uint64_t pol_r = policy_evict_first(), pol_u = policy_evict_last();
             mbar_expect_tx(rfull, CP_R);
 #pragma unroll 1
             for (int ch = 0; ch < 9; ++ch)
-                tma_load_3d(rbase + ch * CP_BOX, &map_cache, rfull, 64 * ch, 64 * gt, a.b, pol_r);
+                tma_load_3d(rbase + ch * CP_BOX, &map_rows, rfull, 64 * ch, CP_ROWS * gt, a.b, pol_r);
             const int ublk = a.ublk0 + 128 * bt;
-            int last[3] = {-1, -1, -1};
+            int last[CP_USTAGES] = {-1, -1};
 #pragma unroll 1
             for (int kb = 0; kb < 9; ++kb) {
-                const int s = kb % 3;
-                if (!mbar_wait(uempty(s), ((kb / 3) & 1) ^ 1, abort_flag, K_PREFILL_CONDENSE, 1)) break;
+                const int s = kb % CP_USTAGES;
+                if (!mbar_wait(uempty(s), ((kb / CP_USTAGES) & 1) ^ 1, abort_flag, K_PREFILL_CONDENSE, 1)) break;
                 mbar_expect_tx(ufull(s), 2 * CP_UBOX);
                 const uint32_t dst = ubase + s * 2 * CP_UBOX;
                 tma_load_3d(dst, &map_u, ufull(s), 64 * kb, 0, ublk, pol_u);
@@ -148,25 +159,25 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
                 last[s] = kb;
             }
             mbar_wait(rfull, 0, nullptr, K_PREFILL_CONDENSE, 2);
-            for (int s = 0; s < 3; ++s)
-                if (last[s] >= 0) mbar_wait(ufull(s), (last[s] / 3) & 1, nullptr, K_PREFILL_CONDENSE, 2);
+            for (int s = 0; s < CP_USTAGES; ++s)
+                if (last[s] >= 0) mbar_wait(ufull(s), (last[s] / CP_USTAGES) & 1, nullptr, K_PREFILL_CONDENSE, 2);
         }
     } else if (warp == 5 || warp == 6) {
         // ------------------------------------------------------------ MMA issuers
         // warp 5: S_hi chain, then the pooling MMAs; warp 6: S_lo chain
         if (lane == 0) {
             const int hl = warp - 5;
-            constexpr uint32_t IDESC_S = idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t IDESC_S = idesc_bf16(128, CP_ROWS, 0, 0);
             bool ok = mbar_wait(rfull, 0, abort_flag, K_PREFILL_CONDENSE, 3);
 #pragma unroll 1
             for (int kb = 0; kb < 9 && ok; ++kb) {
-                const int s = kb % 3;
-                if (!(ok = mbar_wait(ufull(s), (kb / 3) & 1, abort_flag, K_PREFILL_CONDENSE, 4))) break;
+                const int s = kb % CP_USTAGES;
+                if (!(ok = mbar_wait(ufull(s), (kb / CP_USTAGES) & 1, abort_flag, K_PREFILL_CONDENSE, 4))) break;
                 tc_fence_after();
                 const uint32_t ua = ubase + s * 2 * CP_UBOX + hl * CP_UBOX;
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(tmem + CP_TM_S + 64 * hl, sdesc_sw128(ua + 32 * ks, 16, 1024),
+                    mma_ss(tmem + CP_TM_S + CP_ROWS * hl, sdesc_sw128(ua + 32 * ks, 16, 1024),
                            sdesc_sw128(rbase + kb * CP_BOX + 32 * ks, 16, 1024), IDESC_S, (kb | ks) ? 1u : 0u);
                 tc_commit(uempty(s));
             }
@@ -174,19 +185,18 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
             if (hl == 0 && ok) {
                 // rep_j[128 x 128c..] = alpha_j (A, K-major, K = 16 at column 16 jj of
                 // the alpha tile) * rows 16 jj.. of the tile (B, MN-major, N = 128
-                // spanning boxes 2c and 2c+1)
+                // spanning boxes 2c and 2c+1); one TMEM buffer, drained in turn
                 constexpr uint32_t IDESC_P = idesc_bf16(128, 128, 0, 1);
                 ok = mbar_wait(aready, 0, abort_flag, K_PREFILL_CONDENSE, 5);
                 if (ok) tc_fence_after();
 #pragma unroll 1
-                for (int idx = 0; idx < 16 && ok; ++idx) {
-                    const int jj = idx >> 2, cc = idx & 3, buf = idx % 3;
-                    if (!(ok = mbar_wait(pempty(buf), ((idx / 3) & 1) ^ 1, abort_flag, K_PREFILL_CONDENSE, 6)))
-                        break;
+                for (int idx = 0; idx < 4 * CP_G && ok; ++idx) {
+                    const int jj = idx >> 2, cc = idx & 3;
+                    if (!(ok = mbar_wait(pempty, (idx & 1) ^ 1, abort_flag, K_PREFILL_CONDENSE, 6))) break;
                     tc_fence_after();
-                    mma_ss(tmem + CP_TM_P + 128 * buf, sdesc_sw128(abase + 32 * jj, 16, 1024),
+                    mma_ss(tmem + CP_TM_P, sdesc_sw128(abase + 32 * jj, 16, 1024),
                            sdesc_sw128(rbase + 2 * cc * CP_BOX + 2048 * jj, CP_BOX, 1024), IDESC_P, 0u);
-                    tc_commit(pfull(buf));
+                    tc_commit(pfull);
                 }
             }
             const uint32_t dr = hl ? drain6 : drain5;
@@ -200,30 +210,27 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         const bool vblk = row < nblk;
         const int64_t mk = vblk ? pf_groups(k, a.cw) : 0;
         const uint32_t lane_base = uint32_t(32 * warp) << 16;
-        int anc[4] = {0, 0, 0, 0};
+        int anc[CP_G];
+#pragma unroll
+        for (int jj = 0; jj < CP_G; ++jj) anc[jj] = 0;
         bool ok = __all_sync(0xffffffffu, mbar_wait(sfull, 0, abort_flag, K_PREFILL_CONDENSE, 8));
         if (ok) {
             tc_fence_after();
-            float s[64];
+            float s[CP_ROWS];
             {
                 float v[32];
                 tmem_ld32(tmem + lane_base + CP_TM_S, v);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) s[e] = v[e];
-                tmem_ld32(tmem + lane_base + CP_TM_S + 32, v);
+                for (int e = 0; e < CP_ROWS; ++e) s[e] = v[e];
+                tmem_ld32(tmem + lane_base + CP_TM_S + CP_ROWS, v);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) s[32 + e] = v[e];
-                tmem_ld32(tmem + lane_base + CP_TM_S + 64, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[e] += v[e];
-                tmem_ld32(tmem + lane_base + CP_TM_S + 96, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[32 + e] += v[e];
+                for (int e = 0; e < CP_ROWS; ++e) s[e] += v[e];
             }
-            // alpha row of this block, K-major with 128-byte swizzle
-            uint8_t *arow = smem + CP_OFF_A + (row >> 3) * 1024 + (row & 7) * 128;
+            // alpha row of this block, K-major with 128-byte swizzle (the U ring
+            // is idle: the importance MMAs have consumed every U stage)
+            uint8_t *arow = smem + CP_OFF_ALPHA + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
+            for (int jj = 0; jj < CP_G; ++jj) {
                 float gm = s[16 * jj];
                 int gi = 0;
 #pragma unroll
@@ -254,11 +261,11 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         __syncwarp();
         if (lane == 0 && ok) mbar_arrive(aready);
 
-        // Output rows go through a per-warp staging area in the (now idle)
-        // U ring so that every store instruction writes whole row segments:
-        // lat: 32 rows x 256 B (one d-chunk), rope: 32 rows x 128 B.
-        uint8_t *stg_lat = smem + CP_OFF_U + warp * 8192;
-        uint8_t *stg_rope = smem + CP_OFF_U + 4 * 8192 + warp * 4096;
+        // Output rows go through a per-warp staging area so that every store
+        // instruction writes whole row segments: lat 32 rows x 256 B (one
+        // d-chunk), rope 32 rows x 128 B.
+        uint8_t *stg_lat = smem + CP_OFF_STG_LAT + warp * 8192;
+        uint8_t *stg_rope = smem + CP_OFF_STG_ROPE + warp * 4096;
         const int64_t kk_warp = int64_t(128) * bt + 32 * warp;   // chunk block of the warp's first lane
         const int hl = lane >> 4, c16 = lane & 15;                // store phase: row 2x + hl, chunk c16
         // representative (group j, chunk block kk) lives in row j nbc + kk
@@ -267,8 +274,8 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
         // anchor keys (bit copies from the tile) and anchor positions
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(rfull, 0, abort_flag, K_PREFILL_CONDENSE, 9));
 #pragma unroll 1
-        for (int jj = 0; jj < 4 && ok; ++jj) {
-            const int64_t j = 4 * int64_t(gt) + jj;
+        for (int jj = 0; jj < CP_G && ok; ++jj) {
+            const int64_t j = int64_t(CP_G) * gt + jj;
             {
                 const int rr = 16 * jj + anc[jj];
                 const uint8_t *src = smem + 8 * CP_BOX + rr * 128;
@@ -292,30 +299,29 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
             __syncwarp();
         }
 
-        // drain the pooled latents: group jj, d-chunk cc, buffer idx % 3
+        // drain the pooled latents: group jj, d-chunk cc, one TMEM buffer
 #pragma unroll 1
-        for (int idx = 0; idx < 16 && ok; ++idx) {
-            const int jj = idx >> 2, cc = idx & 3, buf = idx % 3;
-            ok = __all_sync(0xffffffffu, mbar_wait(pfull(buf), (idx / 3) & 1, abort_flag, K_PREFILL_CONDENSE, 10));
+        for (int idx = 0; idx < 4 * CP_G && ok; ++idx) {
+            const int jj = idx >> 2, cc = idx & 3;
+            ok = __all_sync(0xffffffffu, mbar_wait(pfull, idx & 1, abort_flag, K_PREFILL_CONDENSE, 10));
             if (!ok) break;
             tc_fence_after();
-            uint32_t pk[64];
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll 1
+            for (int q4 = 0; q4 < 4; ++q4) {   // columns 32 q4 .. 32 q4 + 31
                 float v[32];
-                tmem_ld32(tmem + lane_base + CP_TM_P + 128 * buf + 32 * q4, v);
+                tmem_ld32(tmem + lane_base + CP_TM_P + 32 * q4, v);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) pk[16 * q4 + e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+                for (int e = 0; e < 4; ++e) {
+                    const int cix = 4 * q4 + e;   // 16-byte chunk of the 256-byte row segment
+                    *reinterpret_cast<uint4 *>(stg_lat + lane * 256 + ((cix ^ c16) << 4)) =
+                        make_uint4(pack_bf16(v[8 * e], v[8 * e + 1]), pack_bf16(v[8 * e + 2], v[8 * e + 3]),
+                                   pack_bf16(v[8 * e + 4], v[8 * e + 5]), pack_bf16(v[8 * e + 6], v[8 * e + 7]));
+                }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(pempty(buf));
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                *reinterpret_cast<uint4 *>(stg_lat + lane * 256 + ((e ^ c16) << 4)) =
-                    make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-            __syncwarp();
-            const int64_t j = 4 * int64_t(gt) + jj;
+            if (lane == 0) mbar_arrive(pempty);
+            const int64_t j = int64_t(CP_G) * gt + jj;
             // 2 rows of 256 B per instruction
 #pragma unroll
             for (int x = 0; x < 16; ++x) {
@@ -334,7 +340,6 @@ __global__ void __launch_bounds__(CP_THREADS, 1)
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, CP_TM_COLS);
 }
-
 // ====================================================================== attention
 constexpr int AP_THREADS = 416;                 // 13 warps
 constexpr int AP_CHUNK = 8192;                  // [64 rows x 64 cols] bf16
