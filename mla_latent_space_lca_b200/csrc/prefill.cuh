@@ -45,6 +45,15 @@
 
 namespace lca {
 
+// Prefetch a 3-D tensor box into L2 (no shared memory, no completion).
+__device__ __forceinline__ void pf_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 // Representatives of block k.
 __host__ __device__ __forceinline__ int64_t pf_groups(int64_t k, int cw) { return k > cw ? k - cw : 0; }
 
@@ -447,6 +456,12 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
 #pragma unroll 1
                     for (int ch = 0; ch < 9; ++ch)
                         tma_load_3d_plain(dst + ch * AP_CHUNK, &map_rep, full(s), 64 * ch, int(k - a.kc0), 64 * i);
+                    // the block's first CTA warms L2 with the next representative
+                    // tile for itself and the block's other three CTAs
+                    if (qq == 0 && i + 1 < n_rep) {
+#pragma unroll 1
+                        for (int ch = 0; ch < 9; ++ch) pf_prefetch_3d(&map_rep, 64 * ch, int(k - a.kc0), 64 * (i + 1));
+                    }
                 } else {
                     const int row = int(win0 + 64 * (i - n_rep));
 #pragma unroll 1
