@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stored", action="store_true",
                     help="decode: stored-representative mode (groups condensed once and kept)")
+    ap.add_argument("--unfused-compare", type=int, default=0,
+                    help="decode: also time N steps of the unfused path (condense, then attend stored reps)")
     ap.add_argument("--mla-compare", type=int, default=0,
                     help="prefill: also time N full causal MLA prefills (w = L) on the same inputs")
     return ap.parse_args()
@@ -321,6 +323,9 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    # a cache smaller than twice the 126 MB L2 would be served from L2 on
+    # back-to-back steps: flush L2 before every step and time steps one by one
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if B * L * ROW_BYTES < (256 << 20) else None
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -329,27 +334,63 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(local_rank) if rank == 0 else None
     time.sleep(0.25 if sampler else 0)
     n0 = lca.launch_count()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if sampler:
         sampler.mark()
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total_ms = e0.elapsed_time(e1)
+    else:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a_, b_ in ev:
+            flush.zero_()
+            a_.record(stream)
+            step()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        total_ms = sum(a_.elapsed_time(b_) for a_, b_ in ev)
     if sampler:
         sampler.mark()
     launches = (lca.launch_count() - n0) / args.steps
     barrier()
     torch.cuda.synchronize()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    ms = max_over_ranks(total_ms / args.steps, world, dev)
     if sampler:
         sampler.stop()
+
+    # in-run comparison: the unfused path (condense to stored representatives,
+    # then attention over them), which writes and re-reads the representatives
+    unfused_ms = None
+    if args.unfused_compare and lca.num_groups(L) > 0:
+        rep_u = torch.empty(B, lca.num_groups(L), 576, dtype=torch.bfloat16, device=dev)
+
+        def unfused_step():
+            lca.lca_condense(cache, q_recent, scale=inp.scale, rep=rep_u, ws=ws, stream=stream)
+            lca.lca_decode_attn(cache, rep_u, q, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+
+        for _ in range(3):
+            unfused_step()
+        torch.cuda.synchronize()
+        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        u0.record(stream)
+        for _ in range(args.unfused_compare):
+            unfused_step()
+        u1.record(stream)
+        torch.cuda.synchronize()
+        unfused_ms = max_over_ranks(u0.elapsed_time(u1) / args.unfused_compare, world, dev)
+        del rep_u
 
     # per-kernel durations (CUDA events around each launch, on its stream)
     prof_steps = min(args.steps, 200)
     lca.profile_enable(True)
     for _ in range(prof_steps):
+        if flush is not None:
+            flush.zero_()
         step()
     torch.cuda.synchronize()
     prof = lca.profile_collect()
@@ -400,7 +441,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": args.workload, "B_per_gpu": B, "L": L, "g": 16, "w": 1024,
                    "heads": 16, "d_c": 512, "d_r": 64, "parallelism": f"replicas x{world}",
-                   "l2": "inputs (B*L*1152 B) larger than the 126 MB L2; no flush"},
+                   "l2": ("inputs (B*L*1152 B) larger than the 126 MB L2; no flush" if flush is None else
+                          "flushed (256 MB write) before every step; steps timed one by one")},
         "cache_gbps": gbs, "cache_frac_of_hbm": gbs / world / peak,
         "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA)",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
@@ -413,6 +455,14 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
+    if unfused_ms is not None:
+        m = lca.num_groups(L)
+        line["unfused_path"] = {
+            "ms_per_step": unfused_ms, "tokens_per_s": tokens / (unfused_ms / 1e3),
+            "fused_speedup": unfused_ms / ms,
+            "algorithmic_bytes_per_step": B * (L + 2 * m) * ROW_BYTES,
+            "note": "lca_condense (reads the cache, writes m representatives) then lca_decode_attn "
+                    "(re-reads them and the window)"}
     if world == 1 and not args.no_cpu_baseline:
         tok_s, cores, sample, _ = cpu_baseline(inp, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
