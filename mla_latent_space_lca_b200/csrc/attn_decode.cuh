@@ -67,7 +67,8 @@ constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
 constexpr int AT_NBAR = 24;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
-constexpr int AT_SMEM = AT_OFF_MISC + 256;              // 225792
+constexpr int AT_OFF_ALB = AT_OFF_MISC + 256;           // per softmax warp: alpha [4 sub][16], anchors [4]
+constexpr int AT_SMEM = AT_OFF_ALB + 4 * 68 * 4;         // 226880
 constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
 
 enum { MODE_MLA = 0, MODE_REPS = 1, MODE_LCA = 2 };
@@ -192,6 +193,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
     float *fsc = reinterpret_cast<float *>(smem + AT_OFF_MISC + 128);   // [2][16]
+    float *alb = reinterpret_cast<float *>(smem + AT_OFF_ALB) + 68 * (warp & 3);   // this softmax warp's
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 3; ++s) {
@@ -408,20 +410,42 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         for (int e = 0; e < 4; ++e) al[4 * k4 + e] = sc[e] * inv;
                         anc[k4] = gi;
                     }
-                    // anchors from thread (g=4, sub=0); alpha of my tokens from (g=4, my sub)
+                    // alpha of my tokens from thread (g=4, my sub), anchors from (g=4,
+                    // sub=0), through this warp's shared-memory slot
+                    __syncwarp();
+                    if (g == 4) {
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) anc[k4] = __shfl_sync(0xffffffffu, anc[k4], 16);
+                        for (int v = 0; v < 4; ++v)
+                            *reinterpret_cast<float4 *>(alb + 16 * sub + 4 * v) =
+                                make_float4(al[4 * v], al[4 * v + 1], al[4 * v + 2], al[4 * v + 3]);
+                        if (sub == 0)
+                            *reinterpret_cast<int4 *>(alb + 64) = make_int4(anc[0], anc[1], anc[2], anc[3]);
+                    }
+                    __syncwarp();
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) al[x] = __shfl_sync(0xffffffffu, al[x], 16 + sub);
+                    for (int v = 0; v < 4; ++v) {
+                        const float4 t4 = *reinterpret_cast<const float4 *>(alb + 16 * sub + 4 * v);
+                        al[4 * v] = t4.x;
+                        al[4 * v + 1] = t4.y;
+                        al[4 * v + 2] = t4.z;
+                        al[4 * v + 3] = t4.w;
+                    }
+                    {
+                        const int4 a4 = *reinterpret_cast<const int4 *>(alb + 64);
+                        anc[0] = a4.x;
+                        anc[1] = a4.y;
+                        anc[2] = a4.z;
+                        anc[3] = a4.w;
+                    }
                     if (a.anchor && quad == 0 && lane == 0) {
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4)
                             if (k4 < ti.valid)
                                 a.anchor[size_t(b) * a.m + size_t(k) * 4 + k4] = int32_t((k * 4 + k4) * 16 + anc[k4]);
                     }
-                    // per group: zx = sum alpha X (threads g < 4) and the anchor's
-                    // Y of two heads (threads g = 6, 7), each summed over the 4
-                    // threads of its row
+                    // per group: zx = sum alpha X (threads g < 4, summed over the 4
+                    // threads of the row) and the anchor's Y of two heads (threads
+                    // g = 6, 7: only the thread holding the anchor token keeps it)
                     float zx[4], y0[4], y1[4];
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
@@ -435,19 +459,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         }
                         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                        a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
-                        a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
-                        a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
-                        a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
                         zx[k4] = acc;
                         y0[k4] = a0;
                         y1[k4] = a1;
                     }
-                    // head 4q+g's Y lives in thread g' = 6 + (g&1): ya for g < 2, yb for g >= 2
-                    const int ysrc = 24 + 4 * (g & 1) + sub;
+                    // head 4q+g's Y lives in thread g' = 6 + (g&1) (ya for g < 2,
+                    // yb for g >= 2), in the sub-lane whose tokens hold the anchor
                     float z[4];
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
+                        const int ysrc = 24 + 4 * (g & 1) + ((anc[k4] & 7) >> 1);
                         const float v0 = __shfl_sync(0xffffffffu, y0[k4], ysrc);
                         const float v1 = __shfl_sync(0xffffffffu, y1[k4], ysrc);
                         const float yv = (g & 2) ? v1 : v0;
