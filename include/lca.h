@@ -194,8 +194,8 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
  *   anchor [B][q_len/g][m_last] int32 or NULL, m_last = m of the range's last
  *          block: absolute anchor positions of block k's groups j < m_k in
  *          row (k - q_start/g); the rest of each row is not written.
- * Representatives are rounded to bf16 like cache rows.  Requires g == 16 and
- * L <= 2^27.  ws: lca_workspace_bytes(LCA_OP_PREFILL, B, L, q_len, p) bytes
+ * Representatives are rounded to bf16 like cache rows.  Requires g == 16,
+ * L <= 2^27 and B * q_len / 16 < 2^31 (LCA_ERR_UNSUPPORTED otherwise).  ws: lca_workspace_bytes(LCA_OP_PREFILL, B, L, q_len, p) bytes
  * (enough for any q_start; the blocks are processed in chunks of 256 so the
  * workspace stays near 256 * m_last * 1152 bytes). */
 int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L,

@@ -557,6 +557,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     if (p.g != 16 || p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
     if (q_start < 0 || q_len < 0 || q_start % 16 || q_len % 16 || q_start + q_len > L) return LCA_ERR_INVALID_ARG;
     if (L > (int64_t(1) << 27)) return LCA_ERR_UNSUPPORTED;   // query rows 16 L index a TMA map
+    if (int64_t(B) * (q_len / 16) >= (int64_t(1) << 31)) return LCA_ERR_UNSUPPORTED;   // block index of a TMA map
     if ((o_lat && !aligned16(o_lat)) || (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
         return LCA_ERR_MISALIGNED;
     if (q_len == 0) return LCA_OK;

@@ -105,6 +105,12 @@ def test_other_entry_points_reject_bad_arguments(lcalib):
     pv = LcaParams(16, 1024, 0.07, _lib.VARIANT_SPARSE)
     assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 0, 4096, pv, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
     assert lcalib.lca_decode_noalloc(A, A, A, A, 1, 4096, pv, A, None, None, None) == _lib.LCA_ERR_UNSUPPORTED
+    # prefill size limits: L beyond 2^27, and 2^31 blocks over the batch
+    assert lcalib.lca_prefill_block(A, A, A, 1, (1 << 27) + 16, 0, 16, p, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
+    assert lcalib.lca_prefill_block(A, A, A, 1 << 8, 1 << 27, 0, 1 << 27, p, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
+    # prefill range checks: unaligned start, past the end
+    assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 8, 16, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 4080, 32, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
 
 
 def test_valid_call_without_gpu_reports_no_device(lcalib):
