@@ -209,17 +209,21 @@ def ncu_traffic(workload):
         return None
 
 
-def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0):
+REF_BUDGET_S = 150.0   # whole reference-arm run (all K + W steps), seconds
+
+
+def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0, seqs: int = 0):
     """The oracle as it stands, on host cores, over a bounded sample of the
-    workload (whole sequences).  Returns (tokens/s, cores, sample text,
-    per-step seconds)."""
+    workload (whole sequences; `seqs` per call, else ~2 s worth).  Returns
+    (tokens/s, cores, sample text, per-step seconds)."""
     import oracle
     from mla_latent_space_lca_b200.inputs import bf16_bits
 
     B = inp.cache.shape[0]
     # sample size: sequences whose oracle decode takes ~1-3 s
     per_seq_guess = inp.L * 16 * 576 * 2 / 3e9
-    S = max(1, min(B, int(2.0 / max(per_seq_guess, 1e-6))))
+    S = seqs if seqs > 0 else max(1, min(B, int(2.0 / max(per_seq_guess, 1e-6))))
+    S = min(S, B)
     sl = list(range(S))
     c = bf16_bits(inp.cache[:S])
     qr = bf16_bits(inp.q_recent[:S])
@@ -266,7 +270,11 @@ def run_reference(args, rank, world):
     if wl["kind"] == "prefill":
         import oracle
         inp = make_prefill_inputs(wl["B"], wl["L"], seed=0)
-        n = 2 * oracle.num_threads()
+        # blocks per step so that all K + W steps fit REF_BUDGET_S
+        n0 = oracle.num_threads()
+        _, _, _, t0 = prefill_cpu_baseline(inp, n0, steps=1)
+        per_step = REF_BUDGET_S / max(1, args.steps + args.warmup)
+        n = max(1, min(2 * n0, int(n0 * per_step / max(t0[0], 1e-6))))
         tok_s, cores, sample, times = prefill_cpu_baseline(inp, n, steps=args.steps, warmup=args.warmup)
         ms = 1e3 * statistics.mean(times)
         line = {
@@ -283,7 +291,12 @@ def run_reference(args, rank, world):
         print(json.dumps(line), flush=True)
         return
     inp = make_decode_inputs(wl["B"], wl["L"], seed=0)
-    tok_s, cores, sample, times = cpu_baseline(inp, 0, steps=args.steps, warmup=args.warmup)
+    # size each step's sample so that all K + W steps fit REF_BUDGET_S: time
+    # one single-sequence call first
+    _, _, _, t1 = cpu_baseline(inp, 0, steps=1, warmup=0, seqs=1)
+    per_step = REF_BUDGET_S / max(1, args.steps + args.warmup)
+    seqs = max(1, min(wl["B"], int(per_step / max(t1[0], 1e-6))))
+    tok_s, cores, sample, times = cpu_baseline(inp, 0, steps=args.steps, warmup=args.warmup, seqs=seqs)
     ms = 1e3 * statistics.mean(times)
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
