@@ -67,8 +67,9 @@ constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
 constexpr int AT_NBAR = 24;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
-constexpr int AT_OFF_ALB = AT_OFF_MISC + 256;           // per softmax warp: alpha [4 sub][16], anchors [4]
-constexpr int AT_SMEM = AT_OFF_ALB + 4 * 68 * 4;         // 226880
+constexpr int AT_OFF_ALB = AT_OFF_MISC + 256;           // per softmax warp: e [4 sub][16], anchors [4], 1/den [4]
+constexpr int AT_ALB = 72;                               // floats per softmax warp
+constexpr int AT_SMEM = AT_OFF_ALB + 4 * AT_ALB * 4;     // 226944
 constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
 
 enum { MODE_MLA = 0, MODE_REPS = 1, MODE_LCA = 2 };
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
     float *fsc = reinterpret_cast<float *>(smem + AT_OFF_MISC + 128);   // [2][16]
-    float *alb = reinterpret_cast<float *>(smem + AT_OFF_ALB) + 68 * (warp & 3);   // this softmax warp's
+    float *alb = reinterpret_cast<float *>(smem + AT_OFF_ALB) + AT_ALB * (warp & 3);   // this softmax warp's
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < 3; ++s) {
@@ -374,7 +375,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 float f = 1.f;      // reference-max rescale factor of this head
                 if (MODE == MODE_LCA && ti.hist) {
                     // ---- fused condensation of 4 groups; threads g == 4 own u
-                    float al[16];
+                    float al[16];       // exp(s - group max); alpha = al * rinv
+                    float rinv[4];      // 1 / sum of the group's al
                     int anc[4];
 #pragma unroll
                     for (int x = 0; x < 16; ++x) al[x] = lo[x] + __shfl_down_sync(0xffffffffu, lo[x], 4);
@@ -405,9 +407,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         }
                         den += __shfl_xor_sync(0xffffffffu, den, 1);
                         den += __shfl_xor_sync(0xffffffffu, den, 2);
-                        const float inv = 1.f / den;
+                        rinv[k4] = __fdividef(1.f, den);   // den >= 1 (the maximum's term)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) al[4 * k4 + e] = sc[e] * inv;
+                        for (int e = 0; e < 4; ++e) al[4 * k4 + e] = sc[e];
                         anc[k4] = gi;
                     }
                     // alpha of my tokens from thread (g=4, my sub), anchors from (g=4,
@@ -418,8 +420,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         for (int v = 0; v < 4; ++v)
                             *reinterpret_cast<float4 *>(alb + 16 * sub + 4 * v) =
                                 make_float4(al[4 * v], al[4 * v + 1], al[4 * v + 2], al[4 * v + 3]);
-                        if (sub == 0)
+                        if (sub == 0) {
                             *reinterpret_cast<int4 *>(alb + 64) = make_int4(anc[0], anc[1], anc[2], anc[3]);
+                            *reinterpret_cast<float4 *>(alb + 68) = make_float4(rinv[0], rinv[1], rinv[2], rinv[3]);
+                        }
                     }
                     __syncwarp();
 #pragma unroll
@@ -436,6 +440,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         anc[1] = a4.y;
                         anc[2] = a4.z;
                         anc[3] = a4.w;
+                        const float4 r4 = *reinterpret_cast<const float4 *>(alb + 68);
+                        rinv[0] = r4.x;
+                        rinv[1] = r4.y;
+                        rinv[2] = r4.z;
+                        rinv[3] = r4.w;
                     }
                     if (a.anchor && quad == 0 && lane == 0) {
 #pragma unroll
@@ -459,7 +468,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                         }
                         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                        zx[k4] = acc;
+                        zx[k4] = acc * rinv[k4];
                         y0[k4] = a0;
                         y1[k4] = a1;
                     }
@@ -487,8 +496,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const float p = (k4 < ti.valid) ? fast_exp2(z[k4] - m_use) : 0.f;
                         psum += p;
+                        const float pr = p * rinv[k4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) w[4 * k4 + e] = p * al[4 * k4 + e];
+                        for (int e = 0; e < 4; ++e) w[4 * k4 + e] = pr * al[4 * k4 + e];
                     }
                     l_run += psum;
                 } else {
