@@ -96,11 +96,12 @@ def test_prefill_small(B, L, w, q_start, q_len, peak):
     check_prefill(inp, q_start, q_len, w)
 
 
-def test_prefill_tiles_and_chunks():
+@pytest.mark.parametrize("B", [1, 2])
+def test_prefill_tiles_and_chunks(B):
     """More than one condense block tile (128 blocks), several representative
-    tiles per block and two 256-block chunks; sampled blocks."""
-    B, L, w = 1, 16 * 300, 256
-    inp = make_prefill_inputs(B, L, w=w, seed=41)
+    tiles per block and two 256-block chunks per sequence; sampled blocks."""
+    L, w = 16 * 300, 256
+    inp = make_prefill_inputs(B, L, w=w, seed=41 + B)
     blocks = [0, 1, 15, 16, 17, 30, 127, 128, 129, 200, 255, 256, 257, 298, 299]
     check_prefill(inp, 0, L, w, blocks=blocks)
 
