@@ -229,6 +229,13 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
                        int B, int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor,
                        void *stream);
 
+/* Self-test of the failure path (no counterpart on the page): launches one
+ * kernel whose bounded wait can never be satisfied.  After ~2 s it records
+ * LCA_ERR_DEVICE_TIMEOUT in the device status word (kernel id 8 in bits
+ * 8..15 of lca_device_status's detail, wait site 1 in bits 16..23) and
+ * returns; the context stays usable.  Asynchronous on `stream`. */
+int lca_selftest_wait_timeout(void *stream);
+
 /* Text for a status code (static storage). */
 const char *lca_strerror(int status);
 

@@ -30,7 +30,8 @@ VARIANT_LCA, VARIANT_POOL_POSITION, VARIANT_SPARSE = range(3)
 EXPORTS = ("lca_num_groups", "lca_workspace_bytes", "mla_decode_attn", "lca_condense",
            "lca_decode_attn", "lca_decode", "lca_prefill_block", "lca_strerror",
            "lca_device_status", "lca_profile_enable", "lca_profile_collect", "lca_launch_count",
-           "lca_decode_noalloc", "lca_condense_append", "lca_decode_stored")
+           "lca_decode_noalloc", "lca_condense_append", "lca_decode_stored",
+           "lca_selftest_wait_timeout")
 
 
 class LcaParams(ctypes.Structure):
@@ -69,6 +70,8 @@ def lib():
         L.mla_decode_attn.argtypes = [P, P, P, I, I64, F, P, P, P, SZ, P]
         L.lca_condense.restype = I
         L.lca_condense.argtypes = [P, P, I, I64, LcaParams, P, P, P, P, SZ, P]
+        L.lca_selftest_wait_timeout.restype = I
+        L.lca_selftest_wait_timeout.argtypes = [P]
         L.lca_condense_append.restype = I
         L.lca_condense_append.argtypes = [P, P, I, I64, LcaParams, I64, P, I64, P, P, P, SZ, P]
         L.lca_decode_stored.restype = I

@@ -20,6 +20,7 @@
 #include "attn_decode.cuh"
 #include "wuv_gemm.cuh"
 #include "prefill.cuh"
+#include "selftest.cuh"
 
 using namespace lca;
 
@@ -110,9 +111,9 @@ struct ProfRec {
     cudaEvent_t a, b;
     int kid;
 };
-const char *kKernelNames[] = {"",         "prep_summary", "condense",    "attn_decode",
-                               "combine_wuv", "wuv_gemm",  "attn_prefill", "condense_prefill"};
-constexpr int kNumKernelIds = 8;
+const char *kKernelNames[] = {"",         "prep_summary", "condense",    "attn_decode",      "combine_wuv",
+                               "wuv_gemm", "attn_prefill", "condense_prefill", "selftest_wait"};
+constexpr int kNumKernelIds = 9;
 bool g_prof_on = false;
 std::vector<ProfRec> g_prof_used;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
@@ -657,6 +658,17 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
         }
     }
     return LCA_OK;
+}
+
+int lca_selftest_wait_timeout(void *stream)
+{
+    int rc = LCA_OK;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Launch l(st, K_SELFTEST);
+    selftest_wait_kernel<<<1, 32, 0, st>>>();
+    return l.done();
 }
 
 const char *lca_strerror(int status)
