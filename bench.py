@@ -58,6 +58,8 @@ def parse():
                     help="decode: stored-representative mode (groups condensed once and kept)")
     ap.add_argument("--unfused-compare", type=int, default=0,
                     help="decode: also time N steps of the unfused path (condense, then attend stored reps)")
+    ap.add_argument("--split-l", action="store_true",
+                    help="decode: every sequence's cache split along L over the ranks (strong scaling)")
     ap.add_argument("--mla-compare", type=int, default=0,
                     help="prefill: also time N full causal MLA prefills (w = L) on the same inputs")
     return ap.parse_args()
@@ -603,6 +605,158 @@ def run_ours_stored(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_ours_split(args, rank, world, local_rank):
+    """Decode with every sequence's cache split along L over the ranks: rank r
+    holds rows shard_bounds(L, world)[r] of the same B sequences; a step is
+    its shard record, an all-gather of the records and the merge + W_UV.
+    The whole job decodes B tokens per step whatever the rank count."""
+    import torch.distributed as dist
+
+    import mla_latent_space_lca_b200 as lca
+    from mla_latent_space_lca_b200.split_l import shard_bounds, split_l_decode
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    assert wl["kind"] == "decode"
+    B, L = wl["B"], wl["L"]
+    inp = make_decode_inputs(B, L, seed=0)          # the same sequences on every rank
+    row0, row1 = shard_bounds(L, world)[rank]
+    h_shard = inp.cache[:, row0:row1].contiguous()
+    cache = h_shard.to(dev)
+    q_recent, q, w_uv = inp.q_recent.to(dev), inp.q.to(dev), inp.w_uv.to(dev)
+    ws = lca.workspace(3, B, L, device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(c=cache, qr=q_recent, qq=q):
+        split_l_decode(c, qr, qq, w_uv, L, row0, scale=inp.scale, out=out, ws=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    shard_bytes = B * (row1 - row0) * ROW_BYTES
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if shard_bytes < (256 << 20) else None
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)
+    n0 = lca.launch_count()
+    if sampler:
+        sampler.mark()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a_, b_ in ev:
+        if flush is not None:
+            flush.zero_()
+        a_.record(stream)
+        step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    total_ms = sum(a_.elapsed_time(b_) for a_, b_ in ev)
+    if sampler:
+        sampler.mark()
+    launches = (lca.launch_count() - n0) / args.steps
+    barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(total_ms / args.steps, world, dev)
+    if sampler:
+        sampler.stop()
+
+    prof_steps = min(args.steps, 200)
+    lca.profile_enable(True)
+    for _ in range(prof_steps):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    prof = lca.profile_collect()
+    lca.profile_enable(False)
+
+    # the fused single-device decode of the same sequences, for comparison (one rank)
+    fused_ms = None
+    if world == 1:
+        def fused():
+            lca.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, out=out, ws=ws)
+        for _ in range(3):
+            fused()
+        torch.cuda.synchronize()
+        fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(min(args.steps, 200))]
+        for a_, b_ in fev:
+            if flush is not None:
+                flush.zero_()
+            a_.record(stream)
+            fused()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        fused_ms = sum(a_.elapsed_time(b_) for a_, b_ in fev) / len(fev)
+
+    # end to end: this rank's shard and the queries from pinned host memory
+    pin = [t.pin_memory() for t in (h_shard, inp.q_recent, inp.q)]
+    h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
+    dbuf = [torch.empty_like(t, device=dev) for t in pin]
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+
+    def e2e_step():
+        for d, h in zip(dbuf, pin):
+            d.copy_(h, non_blocking=True)
+        step(*dbuf)
+        h_out.copy_(out, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / args.e2e_steps, world, dev)
+    rc, detail = lca.device_status(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    if rank != 0:
+        return
+    peak, peak_kind = measured_hbm_peak()
+    attn = prof.get("attn_decode")
+    attn_ms = attn[1] / attn[0] if attn else None
+    achieved = shard_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
+    line = {
+        "metric": METRIC, "value": B / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "B": B, "L": L, "g": 16, "w": 1024, "heads": 16,
+                   "d_c": 512, "d_r": 64, "parallelism": f"split-L x{world}",
+                   "rank0_rows": [row0, row1],
+                   "l2": ("shard larger than the 126 MB L2; no flush" if flush is None else
+                          "flushed (256 MB write) before every step")},
+        "cache_gbps": B * L * ROW_BYTES / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA, rank 0's shard)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak if achieved else None,
+                     "traffic": ncu_traffic(args.workload) if world == 1 else None,
+                     "algorithmic_bytes_per_launch": shard_bytes, "launch_ms": attn_ms},
+        "kernels_ms_per_step": {k: v[1] / v[0] for k, v in prof.items()},
+        "gpu_launches": launches,
+        "clocks": sampler.summary() if sampler else None,
+        "e2e": {"value": B / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 4},
+    }
+    if fused_ms is not None:
+        line["fused_decode_ms_per_step"] = fused_ms
+    if world == 1 and not args.no_cpu_baseline:
+        tok_s, cores, sample, _ = cpu_baseline(inp, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+
+
 def run_ours_prefill(args, rank, world, local_rank):
     import torch.distributed as dist
 
@@ -767,7 +921,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        fn = run_ours_prefill if prefill else (run_ours_stored if args.stored else run_ours)
+        if prefill:
+            fn = run_ours_prefill
+        else:
+            fn = run_ours_stored if args.stored else (run_ours_split if args.split_l else run_ours)
         fn(args, rank, world, local_rank)
     finally:
         if world > 1:

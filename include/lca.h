@@ -229,6 +229,43 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
                        int B, int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor,
                        void *stream);
 
+/* Decode split along the sequence across devices.  Every query's attention
+ * over [representatives || window] (整体框架) is a softmax over a set of rows,
+ * so it can be cut into shards of rows.  Each shard yields a partial: o
+ * normalised over its own rows plus the log-sum-exp of its logits.
+ * lca_combine_shards merges the partials by their log-sum-exp and applies
+ * W_UV.  (The page runs on one device; this interface is not part of the
+ * method, and the result equals lca_decode up to fp32 rounding.)
+ *
+ * A shard record is LCA_SHARD_RECORD_PER_HEAD * 16 * B floats, contiguous:
+ *   o    [B][16][512] fp32: the attention output over the shard's rows alone
+ *   lse2 [B][16]      fp32: log2( sum over the shard's rows of exp(z) ),
+ *        z the scaled logit of 整体框架
+ * so a plain all-gather of the records feeds lca_combine_shards.
+ *
+ * lca_decode_shard: cache_shard [B][L_shard][576] bf16 (contiguous) holds
+ * rows row0 .. row0+L_shard-1 of every sequence of a cache of length L.
+ * Shards cut at group boundaries.  row0 % g == 0, and row0 <= m*g with
+ * m = lca_num_groups(L, p).  Either the shard ends at L, which makes it the
+ * last shard and gives it the whole window, or it ends at a multiple of g no
+ * later than m*g.  Each of its groups is condensed with the summary query
+ * of q_recent [B][g][16][576] (NULL allowed only if the shard has no
+ * groups), exactly as in lca_decode.  q [B][16][576] is the current query.
+ *   part   one shard record (required, 16-byte aligned)
+ *   anchor [B][m_shard] int32 or NULL, m_shard = groups in the shard: the
+ *          anchor's row within the shard (add row0 for its position).
+ * Requires g == 16 and variant LCA.  ws: LCA_OP_DECODE bytes for B.
+ *
+ * lca_combine_shards: parts [n_shards] shard records (any order),
+ * w_uv [16][512][128] bf16 -> out [B][16][128] fp32 and, if not NULL,
+ * o_lat [B][16][512] fp32.  No workspace. */
+#define LCA_SHARD_RECORD_PER_HEAD 513
+int lca_decode_shard(const void *cache_shard, const void *q_recent, const void *q, int B, int64_t L,
+                     int64_t row0, int64_t L_shard, lca_params p, float *part, int32_t *anchor,
+                     void *ws, size_t ws_bytes, void *stream);
+int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv, float *out,
+                       float *o_lat, void *stream);
+
 /* Self-test of the failure path (no counterpart on the page): launches one
  * kernel whose bounded wait can never be satisfied.  After ~2 s it records
  * LCA_ERR_DEVICE_TIMEOUT in the device status word (kernel id 8 in bits

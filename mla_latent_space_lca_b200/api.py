@@ -163,6 +163,49 @@ def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     return out
 
 
+def shard_record_floats(B: int) -> int:
+    """Floats in one shard record: o [B][16][512] then lse2 [B][16]."""
+    return B * H * _lib.SHARD_RECORD_PER_HEAD
+
+
+def lca_decode_shard(cache_shard, q_recent, q, L, row0, g=16, w=1024, scale=None, part=None,
+                     anchor=None, ws=None, stream=None):
+    """Partial decode attention over rows row0 .. row0 + L_shard - 1 of a
+    cache of length L (cache_shard [B, L_shard, 576]); returns the shard
+    record (float32 [B*16*513]: o, then lse2)."""
+    B, Ls, _ = cache_shard.shape
+    _need(cache_shard, "cache_shard", torch.bfloat16, (B, Ls, D))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    if q_recent is not None:
+        _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
+    dev = cache_shard.device
+    part = torch.empty(shard_record_floats(B), dtype=torch.float32, device=dev) if part is None else part
+    _need(part, "part", torch.float32, (shard_record_floats(B),))
+    if anchor is not None:
+        _need(anchor, "anchor", torch.int32)
+    ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=dev) if ws is None else ws
+    rc = _lib.lib().lca_decode_shard(_ptr(cache_shard), _ptr(q_recent), _ptr(q), B, L, row0, Ls,
+                                     _params(g, w, scale), _ptr(part), _ptr(anchor), _ptr(ws),
+                                     ws.numel(), _stream(stream))
+    check(rc, "lca_decode_shard")
+    return part
+
+
+def lca_combine_shards(parts, w_uv, B, out=None, o_lat=None, stream=None):
+    """parts [n, B*16*513] float32 shard records -> out [B, 16, 128]."""
+    n = parts.shape[0]
+    _need(parts, "parts", torch.float32, (n, shard_record_floats(B)))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=parts.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V))
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
+    rc = _lib.lib().lca_combine_shards(_ptr(parts), n, B, _ptr(w_uv), _ptr(out), _ptr(o_lat),
+                                       _stream(stream))
+    check(rc, "lca_combine_shards")
+    return out
+
+
 def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, out=None,
                       o_lat=None, anchor=None, ws=None, stream=None):
     B, L, _ = cache.shape

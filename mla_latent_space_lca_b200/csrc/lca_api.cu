@@ -269,7 +269,7 @@ int check_ws(void *ws, size_t ws_bytes, size_t need)
 template <int MODE>
 int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const void *q, const void *w_uv, int B,
                   int64_t L, int64_t m, int64_t win0, float scale, float *out, float *o_lat, int32_t *anchor,
-                  const DecodeWs &w, cudaStream_t st, int64_t rep_stride = 0)
+                  const DecodeWs &w, cudaStream_t st, int64_t rep_stride = 0, float *lse_out = nullptr)
 {
     int rc = get_encode();
     if (rc) return rc;
@@ -311,8 +311,8 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
                                         MODE == MODE_LCA && m > 0, map_cache, map_rep, a);
         if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
-    CUtensorMap map_w;
-    rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
+    CUtensorMap map_w = map_cache;   // unused when out is NULL (a shard's partial)
+    if (out) rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
     if (rc) return rc;
     {
         Launch l(st, K_COMBINE);
@@ -320,7 +320,8 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
         const int rpc = std::max(1, std::min(TD_ROWS, (LCA_HEADS * B + dev->sms - 1) / dev->sms));
         const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + rpc - 1) / rpc), dim3(256),
                                         TD_SMEM_ALLOC, st, true, map_w, (const float *)w.part_o,
-                                        (const float *)w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out, rpc);
+                                        (const float *)w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out, rpc,
+                                        lse_out, 0, int64_t(0));
         if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     return LCA_OK;
@@ -546,6 +547,63 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
     const int64_t m = num_groups(L, p);
     if (m > 0 && (rc = launch_prep(q_recent, B, p, w, st))) return rc;
     return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, anchor, w, st);
+}
+
+int lca_decode_shard(const void *cache_shard, const void *q_recent, const void *q, int B, int64_t L, int64_t row0,
+                     int64_t L_shard, lca_params p, float *part, int32_t *anchor, void *ws, size_t ws_bytes,
+                     void *stream)
+{
+    if (!cache_shard || !q || !part) return LCA_ERR_INVALID_ARG;
+    if (B < 1 || L < 1 || L >= (int64_t(1) << 31) || L_shard < 1 || row0 < 0 || row0 + L_shard > L ||
+        int64_t(B) * L_shard >= (int64_t(1) << 40))
+        return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (p.g != 16 || p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
+    const int64_t m = num_groups(L, p), hist_end = m * p.g, row1 = row0 + L_shard;
+    // whole groups; a shard that does not reach L lies inside the history,
+    // so the window belongs to the last shard alone
+    if (row0 % p.g || row0 > hist_end || (row1 < L && (row1 % p.g || row1 > hist_end))) return LCA_ERR_INVALID_ARG;
+    const int64_t m_loc = (std::min(row1, hist_end) - row0) / p.g;
+    if (m_loc > 0 && !q_recent) return LCA_ERR_INVALID_ARG;
+    if (!aligned16(cache_shard) || !aligned16(q) || !aligned16(part) || (q_recent && !aligned16(q_recent)) ||
+        (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+        return LCA_ERR_MISALIGNED;
+    int rc = LCA_OK;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (m_loc > 0 && (rc = launch_prep(q_recent, B, p, w, st))) return rc;
+    // the shard is an LCA decode of its own L_shard rows: m_loc groups, then
+    // (last shard only) the window; o and lse2 go to the partial record
+    float *lse = part + size_t(B) * LCA_HEADS * LCA_DC;
+    return run_attention<MODE_LCA>(dev, cache_shard, nullptr, q, nullptr, B, L_shard, m_loc, m_loc * p.g, p.scale,
+                                   nullptr, part, anchor, w, st, 0, lse);
+}
+
+int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv, float *out, float *o_lat,
+                       void *stream)
+{
+    if (!parts || !w_uv || !out || n_shards < 1 || B < 1 || B > (1 << 20)) return LCA_ERR_INVALID_ARG;
+    if (!aligned16(parts) || !aligned16(w_uv) || !aligned16(out) || (o_lat && !aligned16(o_lat)))
+        return LCA_ERR_MISALIGNED;
+    int rc = get_encode();
+    if (rc) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap map_w;
+    rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
+    if (rc) return rc;
+    Launch l(st, K_COMBINE);
+    const int rpc = std::max(1, std::min(TD_ROWS, (LCA_HEADS * B + dev->sms - 1) / dev->sms));
+    const int64_t stride = int64_t(B) * LCA_HEADS * LCA_SHARD_RECORD_PER_HEAD;
+    const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + rpc - 1) / rpc), dim3(256),
+                                    TD_SMEM_ALLOC, st, false, map_w, parts, (const float *)nullptr, B, 0,
+                                    int64_t(0), 0, o_lat, out, rpc, (float *)nullptr, n_shards, stride);
+    if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
+    return LCA_OK;
 }
 
 int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B, int64_t L, int64_t q_start,

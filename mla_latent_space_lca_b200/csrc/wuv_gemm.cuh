@@ -136,6 +136,15 @@ __global__ void __launch_bounds__(128, 1)
 // and the warps of a row are merged through shared memory into the bf16
 // K-major B operand.  K = 512 runs as four MMA chains of 8 k-steps, each on
 // its own issuing thread and TMEM accumulator; the epilogue sums them.
+//
+// Two further uses serve a decode split along L across devices:
+//  - out == NULL skips W_UV: the kernel only merges the slots, writes the
+//    normalised o (o_lat) and, through lse_out, each row's base-2
+//    log-sum-exp M + log2(den) -- one shard's partial;
+//  - n_shards > 0 reads n_shards such partials instead of the split-L
+//    workspace: record s starts at part_o + s * shard_stride and holds o
+//    [B][16][512] followed by lse2 [B][16] (part_ml is unused); each acts as
+//    a slot with maximum lse2 and denominator 1.
 constexpr int TD_ROWS = 8;
 constexpr int TD_N = 16;
 constexpr int TD_A = LCA_DC * LCA_DV * 2;               // 131072
@@ -151,7 +160,8 @@ constexpr int TD_SMEM_ALLOC = TD_SMEM + 1024;
 __global__ void __launch_bounds__(256, 1)
     tail_decode_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
                        const float *__restrict__ part_ml, int B, int n_tiles, int64_t T, int G,
-                       float *__restrict__ o_lat, float *__restrict__ out, int rpc)
+                       float *__restrict__ o_lat, float *__restrict__ out, int rpc,
+                       float *__restrict__ lse_out, int n_shards, int64_t shard_stride)
 {
     extern __shared__ uint8_t td_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -162,6 +172,8 @@ __global__ void __launch_bounds__(256, 1)
     const int b0 = blockIdx.y * rpc;           // rpc <= TD_ROWS rows (sequences) per CTA
     const int nb = min(rpc, B - b0);
     const int wpr = max(1, TD_ROWS / nb);     // warps per row
+    const bool gemm = out != nullptr;
+    const size_t lse_off = size_t(B) * LCA_HEADS * LCA_DC;   // lse2 within a shard record
     const uint32_t wbar = sbase + TD_OFF_BAR, accf = wbar + 8, drain0 = wbar + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + TD_OFF_BAR + 128);
     float *scr = reinterpret_cast<float *>(smem + TD_OFF_SCR);
@@ -180,7 +192,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (threadIdx.x == 0) {
+    if (gemm && threadIdx.x == 0) {
         prefetch_tensormap(&map_w);
         const uint64_t pol = policy_evict_last();
         mbar_expect_tx(wbar, TD_A);
@@ -204,17 +216,23 @@ __global__ void __launch_bounds__(256, 1)
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         if (r < nb) {
             const int b = b0 + r;
-            const int c0 = split_owner(int64_t(b) * n_tiles, T, G);
-            const int ns = split_owner(int64_t(b + 1) * n_tiles - 1, T, G) - c0 + 1;
+            const int c0 = n_shards ? 0 : split_owner(int64_t(b) * n_tiles, T, G);
+            const int ns = n_shards ? n_shards : split_owner(int64_t(b + 1) * n_tiles - 1, T, G) - c0 + 1;
             const int mine = (ns - sub + wpr - 1) / wpr;   // slots sub, sub+wpr, ...
             for (int base = 0; base < mine; base += 32) {
                 const int cnt = min(32, mine - base);
                 float m = -INFINITY, l = 0.f;
                 if (lane < cnt) {
-                    const size_t sl = size_t(c0 + sub + wpr * (base + lane) + b) * LCA_HEADS + h;
-                    const float2 ml = *reinterpret_cast<const float2 *>(part_ml + sl * 2);
-                    m = ml.x;
-                    l = ml.y;
+                    const int s = sub + wpr * (base + lane);
+                    if (n_shards) {
+                        m = part_o[size_t(s) * shard_stride + lse_off + size_t(b) * LCA_HEADS + h];
+                        l = 1.f;
+                    } else {
+                        const size_t sl = size_t(c0 + s + b) * LCA_HEADS + h;
+                        const float2 ml = *reinterpret_cast<const float2 *>(part_ml + sl * 2);
+                        m = ml.x;
+                        l = ml.y;
+                    }
                 }
                 float Mc = m;
 #pragma unroll
@@ -233,8 +251,10 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll 4
                 for (int k = 0; k < cnt; ++k) {
                     const float wk = __shfl_sync(0xffffffffu, wl, k);
-                    const size_t sl = size_t(c0 + sub + wpr * (base + k) + b) * LCA_HEADS + h;
-                    const float4 *po = reinterpret_cast<const float4 *>(part_o + sl * LCA_DC + 16 * lane);
+                    const int s = sub + wpr * (base + k);
+                    const float *rec = n_shards ? part_o + size_t(s) * shard_stride + (size_t(b) * LCA_HEADS + h) * LCA_DC
+                                                : part_o + (size_t(c0 + s + b) * LCA_HEADS + h) * LCA_DC;
+                    const float4 *po = reinterpret_cast<const float4 *>(rec + 16 * lane);
                     const float4 x0 = po[0], x1 = po[1], x2 = po[2], x3 = po[3];
                     acc[0] = fmaf(wk, x0.x, acc[0]); acc[1] = fmaf(wk, x0.y, acc[1]);
                     acc[2] = fmaf(wk, x0.z, acc[2]); acc[3] = fmaf(wk, x0.w, acc[3]);
@@ -274,6 +294,7 @@ __global__ void __launch_bounds__(256, 1)
         }
         const float inv = 1.f / dt;
         for (int i = 0; i < wpr; ++i) coef[r * 8 + i] *= inv;
+        if (lse_out) lse_out[size_t(b0 + r) * LCA_HEADS + h] = Mt + log2f(dt);
     }
     __syncthreads();
     // ---- merge the warps of each row; o -> o_lat (fp32) and the B operand (bf16)
@@ -298,7 +319,7 @@ __global__ void __launch_bounds__(256, 1)
     fence_proxy_async();
     __syncthreads();
 
-    if (warp >= 4 && lane == 0) {
+    if (gemm && warp >= 4 && lane == 0) {
         const int j = warp - 4;   // k-chunks 2j, 2j+1
         if (mbar_wait(wbar, 0, nullptr, K_GEMM, 31)) {
             tc_fence_after();
@@ -315,7 +336,7 @@ __global__ void __launch_bounds__(256, 1)
         tc_commit(drain0 + 8 * j);
         mbar_wait(drain0 + 8 * j, 0, nullptr, K_GEMM, 32);
     }
-    if (warp < 4) {
+    if (gemm && warp < 4) {
         bool ok = mbar_wait(accf, 0, nullptr, K_GEMM, 33);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {

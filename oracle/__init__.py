@@ -57,6 +57,8 @@ def _load():
         lib.ora_lca_attend_reps.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P]
         lib.ora_lca_decode_stored.restype = I
         lib.ora_lca_decode_stored.argtypes = [P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
+        lib.ora_lca_decode_shard.restype = I
+        lib.ora_lca_decode_shard.argtypes = [P, P, P, I, Lg, I, I, I, I, I, Dd, Lg, Lg, P, P, P]
         lib.ora_lca_prefill.restype = I
         lib.ora_lca_prefill.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, P, Lg,
                                         P, P, P]
@@ -68,6 +70,11 @@ def _u16(a):
     a = np.ascontiguousarray(a)
     assert a.dtype == np.uint16, a.dtype
     return a
+
+
+def _bf16_to_f64(a):
+    """Exact widening of bf16 bit patterns (the high half of an fp32)."""
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def _ptr(a):
@@ -134,6 +141,41 @@ def lca_decode(cache, q_recent, q, w_uv, g: int, w: int, scale: float, dr: int =
     _load().ora_lca_decode(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L, H, dc, dr,
                            dv, g, w, scale, _ptr(o_lat), _ptr(out), _ptr(anchor))
     return o_lat, out, anchor[:, :m]
+
+
+def lca_decode_shard(cache, q_recent, q, g: int, w: int, scale: float, row0: int, row1: int,
+                     dr: int = 64):
+    """One shard (rows row0 .. row1-1) of the LCA decode attention.
+    -> (o [B,H,dc] normalised over the shard's rows, lse [B,H] = natural
+    log-sum-exp of the shard's logits, anchor [B,m_shard] absolute)."""
+    cache, q_recent, q = _u16(cache), _u16(q_recent), _u16(q)
+    B, L, D = cache.shape
+    H = q.shape[1]
+    dc = D - dr
+    m = num_groups(L, g, w)
+    m_shard = max(0, (min(row1, m * g) - row0) // g)
+    o = np.zeros((B, H, dc))
+    lse = np.zeros((B, H))
+    anchor = np.zeros((B, max(m_shard, 1)), np.int32)
+    rc = _load().ora_lca_decode_shard(_ptr(cache), _ptr(q_recent), _ptr(q), B, L, H, dc, dr, g, w,
+                                      scale, row0, row1, _ptr(o), _ptr(lse), _ptr(anchor))
+    if rc != 0:
+        raise ValueError("shard rows must start at a group boundary and be non-empty")
+    return o, lse, anchor[:, :m_shard]
+
+
+def combine_shards(o_parts, lse_parts, w_uv):
+    """Merge attention outputs over disjoint row sets: with S = log sum_s
+    exp(lse_s), o = sum_s exp(lse_s - S) o_s (each o_s normalised over its
+    rows), then the per-head W_UV up-projection out_h = W_UV[h]^T o_h.
+    o_parts [n,B,H,dc], lse_parts [n,B,H] -> (o_lat [B,H,dc], out [B,H,dv])."""
+    o_parts, lse_parts = np.asarray(o_parts, np.float64), np.asarray(lse_parts, np.float64)
+    top = lse_parts.max(axis=0)
+    wts = np.exp(lse_parts - top)                        # [n,B,H]
+    o_lat = (wts[..., None] * o_parts).sum(axis=0) / wts.sum(axis=0)[..., None]
+    wv = _bf16_to_f64(_u16(w_uv))                        # [H,dc,dv]
+    out = np.einsum("bhk,hkv->bhv", o_lat, wv)
+    return o_lat, out
 
 
 def lca_attend_reps(cache, rep, q, w_uv, g: int, w: int, scale: float, dr: int = 64):

@@ -202,9 +202,9 @@ int ora_lca_condense(const uint16_t *cache, const uint16_t *q_recent, int B, lon
  * form) over n_rep fp64 representative rows followed by n_win cache rows:
  * z_hr = scale * (q_lat,h . c_r + q_rope,h . k_r), p = softmax_r(z),
  * o_lat,h = sum_r p_r c_r.  Representatives carry no extra bias. */
-static void attend_head(const uint16_t *qh, int dc, int dr, double scale, long n_rep,
-                        const double *rep_c, const double *rep_k, const uint16_t *rep_bf,
-                        const uint16_t *win, long n_win, double *o)
+static void attend_head_lse(const uint16_t *qh, int dc, int dr, double scale, long n_rep,
+                            const double *rep_c, const double *rep_k, const uint16_t *rep_bf,
+                            const uint16_t *win, long n_win, double *o, double *lse)
 {
     int D = dc + dr;
     long n = n_rep + n_win;
@@ -244,7 +244,16 @@ static void attend_head(const uint16_t *qh, int dc, int dr, double scale, long n
         }
         o[k] = acc / den;
     }
+    /* log sum_r exp(z_r), for merging attention over disjoint row sets */
+    if (lse) *lse = mx + log(den);
     free(z);
+}
+
+static void attend_head(const uint16_t *qh, int dc, int dr, double scale, long n_rep,
+                        const double *rep_c, const double *rep_k, const uint16_t *rep_bf,
+                        const uint16_t *win, long n_win, double *o)
+{
+    attend_head_lse(qh, dc, dr, scale, n_rep, rep_c, rep_k, rep_bf, win, n_win, o, NULL);
 }
 
 /* Per-head value up-projection out_h = W_UV[h]^T o_lat,h (W_UV [H][dc][dv]). */
@@ -303,6 +312,46 @@ int ora_lca_decode(const uint16_t *cache, const uint16_t *q_recent, const uint16
         if (out) up_project(ol + (size_t)b * H * dc, w_uv, H, dc, dv, out + (size_t)b * H * dv);
     if (o_lat) memcpy(o_lat, ol, sizeof(double) * (size_t)B * H * dc);
     free(ol);
+    free(rc);
+    free(rk);
+    return 0;
+}
+
+/* One shard of the LCA decode attention: the rows row0 .. row1-1 of each
+ * sequence (row0 a multiple of g).  The groups among them (those below
+ * m*g) are condensed exactly as in ora_lca_decode, and the current query
+ * attends [those representatives || the shard's window rows] alone:
+ * o_part [B][H][dc] is normalised over the shard's rows and
+ * lse [B][H] = log sum exp(z) over them.  anchor_out [B][m_shard] (or NULL)
+ * receives absolute positions. */
+int ora_lca_decode_shard(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q, int B,
+                         long L, int H, int dc, int dr, int g, int w, double scale, long row0,
+                         long row1, double *o_part, double *lse, int32_t *anchor_out)
+{
+    int D = dc + dr;
+    long m = ora_num_groups(L, g, w);
+    long hist_end = m * g;
+    long j0 = row0 / g, j1 = (row1 < hist_end ? row1 : hist_end) / g;
+    long n_rep = j1 > j0 ? j1 - j0 : 0;
+    long wstart = row0 > hist_end ? row0 : hist_end;
+    long n_win = row1 > wstart ? row1 - wstart : 0;
+    if (row0 % g != 0 || row1 <= row0 || row1 > L) return -1;
+    double *rc = (double *)malloc(sizeof(double) * (size_t)B * (m > 0 ? m : 1) * dc);
+    double *rk = (double *)malloc(sizeof(double) * (size_t)B * (m > 0 ? m : 1) * dr);
+    int32_t *an = (int32_t *)malloc(sizeof(int32_t) * (size_t)B * (m > 0 ? m : 1));
+    ora_lca_condense(cache, q_recent, B, L, H, dc, dr, g, w, scale, rc, rk, an, NULL, NULL);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; b++)
+        for (int h = 0; h < H; h++)
+            attend_head_lse(q + ((size_t)b * H + h) * D, dc, dr, scale, n_rep,
+                            rc + ((size_t)b * m + j0) * dc, rk + ((size_t)b * m + j0) * dr, NULL,
+                            cache + ((size_t)b * L + wstart) * D, n_win,
+                            o_part + ((size_t)b * H + h) * dc, lse + (size_t)b * H + h);
+    if (anchor_out)
+        for (int b = 0; b < B; b++)
+            for (long j = 0; j < n_rep; j++)
+                anchor_out[(size_t)b * n_rep + j] = an[(size_t)b * m + j0 + j];
+    free(an);
     free(rc);
     free(rk);
     return 0;

@@ -113,6 +113,36 @@ def test_other_entry_points_reject_bad_arguments(lcalib):
     assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 4080, 32, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
 
 
+def test_shard_entry_points_reject_bad_arguments(lcalib):
+    p = LcaParams(16, 1024, 0.07)
+    big = 1 << 30
+    L = 4096 + 21            # m = 193 groups: history rows 0 .. 3087
+
+    def shard(row0, Ls, **kw):
+        a = dict(cache=A, q_recent=A, q=A, B=1, L=L, p=p, part=A, ws_bytes=big)
+        a.update(kw)
+        return lcalib.lca_decode_shard(a["cache"], a["q_recent"], a["q"], a["B"], a["L"], row0, Ls,
+                                       a["p"], a["part"], None, A, a["ws_bytes"], None)
+    INV = _lib.LCA_ERR_INVALID_ARG
+    assert shard(8, 16) == INV                      # not at a group boundary
+    assert shard(0, 24) == INV                      # ends inside a group
+    assert shard(3088 - 16, 32) == INV              # runs into the window without reaching L
+    assert shard(3104, L - 3104) == INV             # starts inside the window
+    assert shard(0, L + 16) == INV                  # past the end
+    assert shard(0, 0) == INV                       # empty
+    assert shard(0, 16, q_recent=None) == INV       # groups need the summary query
+    assert shard(0, 16, part=None) == INV
+    assert shard(0, 16, part=A + 4) == _lib.LCA_ERR_MISALIGNED
+    assert shard(0, 16, ws_bytes=16) == _lib.LCA_ERR_WORKSPACE
+    assert shard(0, 16, p=LcaParams(8, 1024, 0.07)) == _lib.LCA_ERR_UNSUPPORTED
+    assert lcalib.lca_combine_shards(A, 0, 1, A, A, None, None) == INV
+    assert lcalib.lca_combine_shards(None, 2, 1, A, A, None, None) == INV
+    assert lcalib.lca_combine_shards(A, 2, 1, A, A + 8, None, None) == _lib.LCA_ERR_MISALIGNED
+    if not __import__("torch").cuda.is_available():
+        # a valid window-only last shard needs no summary query and gets as far as the device
+        assert shard(3088, L - 3088, q_recent=None) == _lib.LCA_ERR_NO_DEVICE
+
+
 def test_valid_call_without_gpu_reports_no_device(lcalib):
     import torch
     if torch.cuda.is_available():

@@ -1,5 +1,8 @@
-"""Multi-process host logic of the benchmark on CPU (gloo, world size 2): the
-timing reduction takes the slowest rank, and replicas draw distinct batches."""
+"""Multi-process host logic on CPU (gloo, world sizes 2 and 3): the timing
+reduction takes the slowest rank, replicas draw distinct batches, and the
+decode split along the cache gathers and merges every rank's shard record
+(the oracle stands in for the kernels)."""
+import math
 import os
 import sys
 
@@ -46,3 +49,91 @@ def test_single_rank_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(2.0, 1) == 2.0
+
+
+# ------------------------------------------------ decode split along the cache
+def _oracle_shard_fn(cache_shard, q_recent, q, L, row0, g=16, w=1024, scale=None, ws=None):
+    """Stand-in for lca_decode_shard on CPU: the oracle run on this rank's
+    rows alone, packed into the library's shard record (o, then lse2)."""
+    import numpy as np
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits
+    Ls = cache_shard.shape[1]
+    w_loc = w if row0 + Ls == L else 0          # only the last shard holds the window
+    o, lse, _ = oracle.lca_decode_shard(bf16_bits(cache_shard), bf16_bits(q_recent), bf16_bits(q),
+                                        g, w_loc, scale, 0, Ls)
+    rec = np.concatenate([o.ravel(), (lse / math.log(2.0)).ravel()])
+    return torch.from_numpy(rec.astype(np.float32))
+
+
+def _oracle_combine_fn(parts, w_uv, B, out=None):
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits
+    n = parts.shape[0]
+    o = parts[:, : B * 16 * 512].double().numpy().reshape(n, B, 16, 512)
+    lse = parts[:, B * 16 * 512:].double().numpy().reshape(n, B, 16) * math.log(2.0)
+    return torch.from_numpy(oracle.combine_shards(o, lse, bf16_bits(w_uv))[1])
+
+
+def _split_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from mla_latent_space_lca_b200.inputs import make_decode_inputs
+        from mla_latent_space_lca_b200.split_l import shard_bounds, split_l_decode
+        inp = make_decode_inputs(2, 256 + 16 * 9 + 5, w=256, seed=41)
+        row0, row1 = shard_bounds(inp.L, world, 16, 256)[rank]
+        out = split_l_decode(inp.cache[:, row0:row1].contiguous(), inp.q_recent, inp.q, inp.w_uv,
+                             inp.L, row0, w=256, scale=inp.scale, shard_fn=_oracle_shard_fn,
+                             combine_fn=_oracle_combine_fn)
+        q.put((rank, out.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_split_l_decode_gathers_and_merges_shards(world):
+    """Each rank decodes its own rows of the cache, the shard records are
+    all-gathered, and every rank's merge equals the unsplit decode."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits, make_decode_inputs
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 31500 + (os.getpid() + world) % 2000
+    procs = [ctx.Process(target=_split_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    inp = make_decode_inputs(2, 256 + 16 * 9 + 5, w=256, seed=41)
+    _, ref, _ = oracle.lca_decode(bf16_bits(inp.cache), bf16_bits(inp.q_recent), bf16_bits(inp.q),
+                                  bf16_bits(inp.w_uv), 16, 256, inp.scale)
+    for _, out in res:   # float32 records: agreement to fp32 rounding
+        np.testing.assert_allclose(out, ref, rtol=0, atol=2e-6)
+
+
+def test_shard_bounds():
+    sys.path.insert(0, ROOT)
+    from mla_latent_space_lca_b200.split_l import shard_bounds
+    for L, n, g, w in [(1 << 20, 8, 16, 1024), (4096 + 21, 3, 16, 1024), (1024 + 48, 4, 16, 1024),
+                       (81, 5, 16, 0), (80, 5, 16, 0), (32768, 1, 16, 1024), (131072, 7, 16, 1024)]:
+        b = shard_bounds(L, n, g, w)
+        m = max(0, (L - w) // g)
+        assert len(b) == n and b[0][0] == 0 and b[-1][1] == L
+        for (a0, a1), (c0, _) in zip(b[:-1], b[1:]):
+            assert a1 == c0 and a1 % g == 0 and a1 <= m * g   # whole groups, window in the last
+        assert all(r1 > r0 for r0, r1 in b)
+        rows = [r1 - r0 for r0, r1 in b]
+        if m * g >= (n - 1) * (L // n):                       # balanced when the history allows
+            assert max(rows) - min(rows) <= 2 * g
+    assert shard_bounds(1 << 20, 8)[3] == (3 << 17, 4 << 17)
+    with pytest.raises(ValueError):
+        shard_bounds(1024 + 32, 4)      # two groups, four shards
+    with pytest.raises(ValueError):
+        shard_bounds(80, 6, 16, 0)      # five groups and no window row for a sixth shard

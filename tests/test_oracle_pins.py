@@ -428,3 +428,76 @@ def test_ablation_sparse_keeps_the_anchor_row(ora):
             assert np.array_equal(sp["rep_c"][b, j], rows[b, a, :8])
             assert np.array_equal(sp["rep_k"][b, j], rows[b, a, 8:])
     assert np.array_equal(sp["rep_k"], base["rep_k"])
+
+
+# ------------------------------------------------- decode split along the cache
+def _split_cases(L, g, w):
+    m = max(0, (L - w) // g)
+    return [[0, L], [0, g, L], [0, m * g, L], [0, 2 * g, 3 * g, m * g - g, L], [0, g, 2 * g, m * g, L]]
+
+
+@pytest.mark.parametrize("w", [6, 0])
+def test_shard_merge_equals_unsplit_decode(ora, w):
+    """整体框架: one softmax over [representatives || window].  Merging the
+    shards' outputs by their log-sum-exp gives the unsplit decode for every
+    cut, including a shard of one group and a shard of the window alone."""
+    rng = np.random.default_rng(31)
+    g, L = 4, 47
+    cache, q, q_recent, w_uv = small_case(rng, L=L, g=g)
+    ol, out, anchor = ora.lca_decode(cache, q_recent, q, w_uv, g, w, 0.3, dr=4)
+    for cuts in _split_cases(L, g, w):
+        parts = [ora.lca_decode_shard(cache, q_recent, q, g, w, 0.3, a, b, dr=4)
+                 for a, b in zip(cuts[:-1], cuts[1:])]
+        ol2, out2 = ora.combine_shards([p[0] for p in parts], [p[1] for p in parts], w_uv)
+        np.testing.assert_allclose(ol2, ol, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(out2, out, rtol=0, atol=1e-13)
+        assert np.array_equal(np.concatenate([p[2] for p in parts], axis=1), anchor)
+
+
+def test_shard_of_one_window_row_closed_form(ora):
+    """A shard holding a single row: softmax weight 1, so o is that row's
+    latent and the log-sum-exp is its one logit z = scale (q_lat.c + q_rope.k)."""
+    rng = np.random.default_rng(32)
+    g, w, dc, dr, L = 4, 0, 8, 4, 4 * 5 + 1
+    cache, q, q_recent, _ = small_case(rng, L=L, g=g)
+    o, lse, anchor = ora.lca_decode_shard(cache, q_recent, q, g, w, 0.3, L - 1, L, dr=dr)
+    assert anchor.shape == (2, 0)
+    row = from_bits(cache[:, L - 1])                         # [B, dc+dr]
+    qq = from_bits(q)                                        # [B, H, dc+dr]
+    np.testing.assert_array_equal(o, np.broadcast_to(row[:, None, :dc], o.shape))
+    z = 0.3 * np.einsum("bhk,bk->bh", qq, row)
+    np.testing.assert_allclose(lse, z, rtol=0, atol=1e-14)
+
+
+def test_shard_of_one_uniform_group_closed_form(ora):
+    """q_recent = 0 gives a uniform pool: a shard of one group attends one
+    representative, the group's mean latent with its first token's key."""
+    rng = np.random.default_rng(33)
+    g, w, dc, dr, L = 4, 6, 8, 4, 31
+    cache, q, q_recent, _ = small_case(rng, L=L, g=g)
+    q_recent = np.zeros_like(q_recent)
+    j = 2
+    o, lse, anchor = ora.lca_decode_shard(cache, q_recent, q, g, w, 0.3, j * g, (j + 1) * g, dr=dr)
+    assert np.array_equal(anchor, np.full((2, 1), j * g))
+    grp = from_bits(cache[:, j * g:(j + 1) * g])             # [B, g, dc+dr]
+    rep_c, rep_k = grp[:, :, :dc].mean(axis=1), grp[:, 0, dc:]
+    np.testing.assert_allclose(o, np.broadcast_to(rep_c[:, None], o.shape), rtol=0, atol=1e-15)
+    qq = from_bits(q)
+    z = 0.3 * (np.einsum("bhk,bk->bh", qq[..., :dc], rep_c) + np.einsum("bhk,bk->bh", qq[..., dc:], rep_k))
+    np.testing.assert_allclose(lse, z, rtol=0, atol=1e-14)
+
+
+def test_combine_of_two_shards_closed_form(ora):
+    """Two partial outputs with log-sum-exps a and b merge with weights
+    e^a / (e^a + e^b) and e^b / (e^a + e^b); W_UV is the identity on the
+    first dv coordinates here."""
+    B, H, dc, dv = 1, 2, 4, 4
+    o1 = np.arange(B * H * dc, dtype=np.float64).reshape(B, H, dc)
+    o2 = -np.ones((B, H, dc))
+    a, b = np.array([[0.0, 2.0]]), np.array([[math.log(3.0), 2.0]])
+    eye = np.zeros((H, dc, dv))
+    eye[:, np.arange(dv), np.arange(dv)] = 1.0
+    ol, out = ora.combine_shards([o1, o2], [a, b], bf16_bits(eye))
+    np.testing.assert_allclose(ol[0, 0], 0.25 * o1[0, 0] + 0.75 * o2[0, 0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(ol[0, 1], 0.5 * o1[0, 1] + 0.5 * o2[0, 1], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(out, ol, rtol=0, atol=1e-15)
