@@ -235,6 +235,34 @@ def test_reference_max_rescale(where):
     compare(mla.cpu().numpy(), mla_ref, "mla out")
 
 
+def test_reference_max_rescale_on_consecutive_tiles():
+    """Twenty consecutive 64-row tiles, each holding a group whose logit tops
+    everything before it by more than the rescale threshold: the reference
+    maximum moves, and O is rescaled, on every one of them, back to back
+    (and across the CTAs' split points of the longer sequence)."""
+    B, L = 2, 30000
+    inp = make_decode_inputs(B, L, seed=22)
+    for b in range(B):
+        # the logit grows through the RoPE key alone (the latents stay O(1)):
+        # q_rope . k = |q_rope| a, a step of ~11 in log2 units per tile
+        qr0 = inp.q[b, 0, 512:].float()
+        for k in range(20):
+            key = (qr0 / qr0.norm() * (760.0 + 330.0 * k)).to(torch.bfloat16)
+            j = 4 * (300 + k)                  # one group in each of tiles 300..319
+            inp.cache[b, 16 * j: 16 * (j + 1), 512:] = key
+    cache, q_recent, q, w_uv = dev(inp)
+    o_lat = torch.empty(B, 16, 512, device="cuda")
+    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=o_lat)
+    mla = api.mla_decode_attn(cache, q, w_uv, inp.scale)
+    torch.cuda.synchronize()
+    c, qr, qb, wb = bits(inp)
+    ol_ref, out_ref, _ = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
+    compare(out.cpu().numpy(), out_ref, "out")
+    _, mla_ref = oracle.mla_decode(c, qb, wb, inp.scale)
+    compare(mla.cpu().numpy(), mla_ref, "mla out")
+
+
 def test_fused_equals_condense_then_attend():
     """The fused pass and condense -> attend over stored reps agree up to the
     bf16 rounding of stored representatives."""
