@@ -240,6 +240,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         if (lane == 0) {
             prefetch_tensormap(&map_cache);
             if (MODE == MODE_REPS && a.m > 0) prefetch_tensormap(&map_rep);
+            // rows may come from a kernel earlier in the stream: read them only
+            // once the preceding grid (and so everything before it) is complete
+            griddep_wait();
             const uint64_t pol = policy_evict_first();
             int last[3] = {-1, -1, -1};
             int i = 0;

@@ -16,7 +16,17 @@ namespace lca {
 // unit per sequence (nbs = 1), blockwise prefill one per block of g queries.
 // Grid (units, 9): a block owns 64 columns of one unit; its 256 threads are
 // 8 column groups (16-byte loads) x 32 row slices of the g*16 (t, h) query
-// rows, combined through shared memory.
+// rows, with all of a thread's loads in flight at once (one round trip for
+// g = 16), reduced by shuffles within a warp and through 2 KB of shared
+// memory across the 8 warps.
+//
+// Ordering: the kernel lets its dependent (the attention kernel) launch at
+// once, then waits for its own predecessor in the stream (whose output may
+// be q_recent) before reading.  The attention kernel reads nothing before
+// it has waited for this grid to complete, which covers that predecessor
+// too; meanwhile its launch and prologue overlap the predecessor's tail.
+// Every CTA of this grid is resident before the dependent can launch (each
+// triggers first thing), so the dependent never starves it of an SM.
 constexpr int PREP_THREADS = 256;
 
 __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16_t *__restrict__ q_recent,
@@ -24,9 +34,12 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16
                                                                     float coef, float *__restrict__ u,
                                                                     uint16_t *__restrict__ uhl)
 {
-    __shared__ float part[32][64 + 1];
+    __shared__ float part[8][64];
+    griddep_launch_dependents();
+    griddep_wait();
     const int b = blockIdx.x;
-    const int cg = threadIdx.x & 7, sl = threadIdx.x >> 3;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cg = threadIdx.x & 7, sl = threadIdx.x >> 3;   // 32 slices
     const int col0 = blockIdx.y * 64 + 8 * cg;
     const int rows = g * LCA_HEADS;
     const uint16_t *base =
@@ -48,14 +61,22 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16
             acc[6] += bf_lo(x[e].w); acc[7] += bf_hi(x[e].w);
         }
     }
+    // the warp's 4 slices of each column group (lane bits 3 and 4)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[sl][8 * cg + e] = acc[e];
+    for (int e = 0; e < 8; ++e) {
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane < 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[warp][8 * lane + e] = acc[e];
+    }
     __syncthreads();
     if (threadIdx.x < 64) {
         const int c = threadIdx.x;
         float t = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < 32; ++k) t += part[k][c];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += part[w][c];
         const int col = blockIdx.y * 64 + c;
         const float uu = t * coef;
         if (u) u[size_t(b) * LCA_D + col] = uu;
@@ -64,12 +85,6 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16
         uhl[(size_t(b) * 2 + 0) * LCA_D + col] = __bfloat16_as_ushort(hi);
         uhl[(size_t(b) * 2 + 1) * LCA_D + col] = __bfloat16_as_ushort(lo);
     }
-    // This kernel may overlap the previous step's tail (it reads only its
-    // own inputs); the attention kernel that follows must not start before
-    // that tail has finished reading the split-L partials.
-    griddep_wait();
-    __syncthreads();
-    griddep_launch_dependents();
 }
 
 }  // namespace lca
