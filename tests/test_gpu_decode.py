@@ -74,7 +74,7 @@ def bits(inp):
 
 
 # ---------------------------------------------------------------- MLA decode
-@pytest.mark.parametrize("B,L", [(1, 1), (2, 63), (3, 64), (2, 65), (3, 1000), (2, 4096)])
+@pytest.mark.parametrize("B,L", [(1, 1), (2, 63), (3, 64), (2, 65), (3, 1000), (2, 4096), (200, 300)])
 def test_mla_decode_parity(B, L):
     inp = make_decode_inputs(B, L, seed=100 + L)
     cache, _, q, w_uv = dev(inp)
@@ -190,6 +190,10 @@ def test_decode_attn_over_stored_reps(B, L):
     (1, 5000, 30.0),
     (5, 2100, 30.0),
     (70, 1100, 1.0),                  # more rows than one combine CTA holds
+    # more sequences than SMs: a CTA's split-L piece spans several sequences
+    (300, 1040, 1.0),                 # one group each, 17 tiles per sequence
+    (200, 700, 1.0),                  # nothing condensed, one tile per sequence
+    (150, 1024 + 16 * 16, 30.0),      # exactly one full history tile
 ])
 def test_lca_decode_fused_parity(B, L, peak):
     inp = make_decode_inputs(B, L, seed=400 + L, peak=peak)
