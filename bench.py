@@ -61,7 +61,8 @@ def parse():
     ap.add_argument("--split-l", action="store_true",
                     help="decode: every sequence's cache split along L over the ranks (strong scaling)")
     ap.add_argument("--mla-compare", type=int, default=0,
-                    help="prefill: also time N full causal MLA prefills (w = L) on the same inputs")
+                    help="decode: also time N plain MLA decode steps (g = 1, every row attended) on the "
+                         "same inputs; prefill: N full causal MLA prefills (w = L)")
     return ap.parse_args()
 
 
@@ -400,6 +401,37 @@ def run_ours(args, rank, world, local_rank):
         unfused_ms = max_over_ranks(u0.elapsed_time(u1) / args.unfused_compare, world, dev)
         del rep_u
 
+    # in-run comparison: plain MLA decode (g = 1) over the whole cache, the
+    # same inputs, timed the same way
+    mla = None
+    if args.mla_compare:
+        def mla_step():
+            lca.mla_decode_attn(cache, q, w_uv, inp.scale, out=out, ws=ws, stream=stream)
+
+        for _ in range(3):
+            mla_step()
+        torch.cuda.synchronize()
+        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.mla_compare)]
+        for a_, b_ in mev:
+            if flush is not None:
+                flush.zero_()
+            a_.record(stream)
+            mla_step()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        mla_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in mev) / args.mla_compare, world, dev)
+        lca.profile_enable(True)
+        for _ in range(min(args.mla_compare, 200)):
+            if flush is not None:
+                flush.zero_()
+            mla_step()
+        torch.cuda.synchronize()
+        mprof = lca.profile_collect()
+        lca.profile_enable(False)
+        mattn = mprof.get("attn_decode")
+        mla = {"ms_per_step": mla_ms, "attn_ms": mattn[1] / mattn[0] if mattn else None}
+
     # per-kernel durations (CUDA events around each launch, on its stream)
     prof_steps = min(args.steps, 200)
     lca.profile_enable(True)
@@ -470,6 +502,14 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
     }
+    if mla is not None:
+        line["mla_path"] = {
+            "ms_per_step": mla["ms_per_step"], "tokens_per_s": tokens / (mla["ms_per_step"] / 1e3),
+            "lca_speedup": mla["ms_per_step"] / ms,
+            "attn_ms": mla["attn_ms"],
+            "attn_frac_of_hbm": (algo_bytes / (mla["attn_ms"] / 1e3) / 1e9 / peak) if mla["attn_ms"] else None,
+            "note": "mla_decode_attn (g = 1): every cached row attended, same inputs and timing; "
+                    "reads the same bytes as the fused LCA step, with 16x the attention rows"}
     if unfused_ms is not None:
         m = lca.num_groups(L)
         line["unfused_path"] = {
