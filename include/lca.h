@@ -85,11 +85,20 @@ extern "C" {
 #define LCA_VARIANT_LCA 0
 #define LCA_VARIANT_POOL_POSITION 1
 #define LCA_VARIANT_SPARSE 2
+/* cache_pitch: rows from the first row of one sequence's cache to the
+ * next one's.  0 means the packed layout [B][L][576] (pitch L).  A decoder
+ * that keeps a preallocated cache [B][L_max][576] and lets L grow passes
+ * L_max here, and rows L .. L_max-1 of each sequence are never read.
+ * Otherwise it must satisfy cache_pitch >= L and B * cache_pitch < 2^40.
+ * It applies to every entry point taking lca_params (the cache_shard of
+ * lca_decode_shard, rows L_shard); mla_decode_attn takes the packed layout,
+ * and lca_decode with g = 1 is MLA decode with a pitch. */
 typedef struct {
     int g;
     int w;
     float scale;
     int variant;
+    int64_t cache_pitch;
 } lca_params;
 
 /* Operation ids for lca_workspace_bytes. */

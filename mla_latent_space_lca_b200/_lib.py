@@ -38,7 +38,7 @@ SHARD_RECORD_PER_HEAD = 513
 
 class LcaParams(ctypes.Structure):
     _fields_ = [("g", ctypes.c_int), ("w", ctypes.c_int), ("scale", ctypes.c_float),
-                ("variant", ctypes.c_int)]
+                ("variant", ctypes.c_int), ("cache_pitch", ctypes.c_int64)]
 
 
 class KernelTime(ctypes.Structure):

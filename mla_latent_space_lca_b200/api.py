@@ -23,8 +23,9 @@ def default_scale() -> float:
     return 1.0 / math.sqrt(192.0)
 
 
-def _params(g: int, w: int, scale: float | None, variant: int = 0) -> LcaParams:
-    return LcaParams(int(g), int(w), float(default_scale() if scale is None else scale), int(variant))
+def _params(g: int, w: int, scale: float | None, variant: int = 0, pitch: int = 0) -> LcaParams:
+    return LcaParams(int(g), int(w), float(default_scale() if scale is None else scale), int(variant),
+                     int(pitch))
 
 
 def _ptr(t):
@@ -47,6 +48,26 @@ def _need(t, name, dtype, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _cache(t, name="cache"):
+    """A cache tensor [B, L, 576] bf16, either packed or rows 0 .. L-1 of each
+    sequence of a larger [B, L_max, 576] buffer (a view such as
+    buf[:, :L]).  Returns the pitch in rows to pass to the library (0 when
+    packed)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if t.dim() != 3 or t.shape[2] != D:
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected (B, L, {D})")
+    if t.is_contiguous():
+        return 0
+    B, L, _ = t.shape
+    s0, s1, s2 = t.stride()
+    if s2 != 1 or s1 != D or s0 % D or s0 < L * D:
+        raise ValueError(f"{name} must hold each sequence's rows contiguously (strides {t.stride()})")
+    return s0 // D
+
+
 def num_groups(L: int, g: int = 16, w: int = 1024) -> int:
     return int(_lib.lib().lca_num_groups(L, _params(g, w, None)))
 
@@ -63,11 +84,16 @@ def workspace(op: int, B: int, L: int, q_len: int = 0, g: int = 16, w: int = 102
 
 def mla_decode_attn(cache, q, w_uv, scale=None, out=None, o_lat=None, ws=None, stream=None):
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q, "q", torch.bfloat16, (B, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
     ws = workspace(_lib.OP_MLA_DECODE, B, L, device=cache.device) if ws is None else ws
+    if pitch:   # a strided cache: MLA decode through lca_decode with g = 1
+        rc = _lib.lib().lca_decode(_ptr(cache), None, _ptr(q), _ptr(w_uv), B, L, _params(1, 0, scale, 0, pitch),
+                                   _ptr(out), _ptr(o_lat), None, _ptr(ws), ws.numel(), _stream(stream))
+        check(rc, "mla_decode_attn")
+        return out
     rc = _lib.lib().mla_decode_attn(_ptr(cache), _ptr(q), _ptr(w_uv), B, L,
                                     float(default_scale() if scale is None else scale), _ptr(out),
                                     _ptr(o_lat), _ptr(ws), ws.numel(), _stream(stream))
@@ -78,13 +104,13 @@ def mla_decode_attn(cache, q, w_uv, scale=None, out=None, o_lat=None, ws=None, s
 def lca_condense(cache, q_recent, g=16, w=1024, scale=None, rep=None, anchor=None, alpha=None,
                  ws=None, stream=None, variant=0):
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
     m = num_groups(L, g, w)
     dev = cache.device
     rep = torch.empty(B, m, D, dtype=torch.bfloat16, device=dev) if rep is None else rep
     ws = workspace(_lib.OP_CONDENSE, B, L, g=g, w=w, device=dev) if ws is None else ws
-    rc = _lib.lib().lca_condense(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale, variant),
+    rc = _lib.lib().lca_condense(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale, variant, pitch),
                                  _ptr(rep) if m > 0 else None, _ptr(anchor), _ptr(alpha), _ptr(ws),
                                  ws.numel(), _stream(stream))
     check(rc, "lca_condense")
@@ -94,7 +120,7 @@ def lca_condense(cache, q_recent, g=16, w=1024, scale=None, rep=None, anchor=Non
 def lca_decode_attn(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None, ws=None,
                     stream=None):
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q, "q", torch.bfloat16, (B, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     m = num_groups(L, g, w)
@@ -103,7 +129,7 @@ def lca_decode_attn(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
     ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_attn(_ptr(cache), _ptr(rep) if m > 0 else None, _ptr(q), _ptr(w_uv),
-                                    B, L, _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(ws),
+                                    B, L, _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(ws),
                                     ws.numel(), _stream(stream))
     check(rc, "lca_decode_attn")
     return out
@@ -114,14 +140,14 @@ def lca_condense_append(cache, q_recent, rep, j0, g=16, w=1024, scale=None, anch
     """Condense groups j0 .. m-1 into rows j0 .. of the representative cache
     rep [B, rep_cap, 576] (bf16); returns m, the number of groups now held."""
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
     _need(rep, "rep", torch.bfloat16)
     if rep.dim() != 3 or rep.shape[0] != B or rep.shape[2] != D:
         raise ValueError(f"rep has shape {tuple(rep.shape)}, expected ({B}, rep_cap, {D})")
     m = num_groups(L, g, w)
     ws = workspace(_lib.OP_CONDENSE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
-    rc = _lib.lib().lca_condense_append(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale, variant), int(j0),
+    rc = _lib.lib().lca_condense_append(_ptr(cache), _ptr(q_recent), B, L, _params(g, w, scale, variant, pitch), int(j0),
                                         _ptr(rep), rep.shape[1], _ptr(anchor), _ptr(alpha), _ptr(ws),
                                         ws.numel(), _stream(stream))
     check(rc, "lca_condense_append")
@@ -133,14 +159,14 @@ def lca_decode_stored(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o
     """Attention over the kept representatives rep [B, rep_cap, 576] (rows
     0 .. m-1) and the window, then W_UV."""
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q, "q", torch.bfloat16, (B, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     _need(rep, "rep", torch.bfloat16)
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
     ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_stored(_ptr(cache), _ptr(rep), rep.shape[1], _ptr(q), _ptr(w_uv), B, L,
-                                      _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(ws), ws.numel(),
+                                      _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(ws), ws.numel(),
                                       _stream(stream))
     check(rc, "lca_decode_stored")
     return out
@@ -149,7 +175,7 @@ def lca_decode_stored(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o
 def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None,
                anchor=None, ws=None, stream=None):
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q, "q", torch.bfloat16, (B, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     if g != 1:
@@ -157,7 +183,7 @@ def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
     ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
-                               _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(anchor), _ptr(ws),
+                               _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor), _ptr(ws),
                                ws.numel(), _stream(stream))
     check(rc, "lca_decode")
     return out
@@ -174,7 +200,7 @@ def lca_decode_shard(cache_shard, q_recent, q, L, row0, g=16, w=1024, scale=None
     cache of length L (cache_shard [B, L_shard, 576]); returns the shard
     record (float32 [B*16*513]: o, then lse2)."""
     B, Ls, _ = cache_shard.shape
-    _need(cache_shard, "cache_shard", torch.bfloat16, (B, Ls, D))
+    pitch = _cache(cache_shard, "cache_shard")
     _need(q, "q", torch.bfloat16, (B, H, D))
     if q_recent is not None:
         _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
@@ -185,7 +211,7 @@ def lca_decode_shard(cache_shard, q_recent, q, L, row0, g=16, w=1024, scale=None
         _need(anchor, "anchor", torch.int32)
     ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=dev) if ws is None else ws
     rc = _lib.lib().lca_decode_shard(_ptr(cache_shard), _ptr(q_recent), _ptr(q), B, L, row0, Ls,
-                                     _params(g, w, scale), _ptr(part), _ptr(anchor), _ptr(ws),
+                                     _params(g, w, scale, 0, pitch), _ptr(part), _ptr(anchor), _ptr(ws),
                                      ws.numel(), _stream(stream))
     check(rc, "lca_decode_shard")
     return part
@@ -209,7 +235,7 @@ def lca_combine_shards(parts, w_uv, B, out=None, o_lat=None, stream=None):
 def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, out=None,
                       o_lat=None, anchor=None, ws=None, stream=None):
     B, L, _ = cache.shape
-    _need(cache, "cache", torch.bfloat16, (B, L, D))
+    pitch = _cache(cache)
     _need(q, "q", torch.bfloat16, (B, L, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     out = (torch.empty(B, q_len, H, D_V, dtype=torch.float32, device=cache.device)
@@ -221,7 +247,7 @@ def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, 
         _need(anchor, "anchor", torch.int32)
     ws = workspace(_lib.OP_PREFILL, B, L, q_len, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_prefill_block(_ptr(cache), _ptr(q), _ptr(w_uv), B, L, q_start, q_len,
-                                      _params(g, w, scale), _ptr(out), _ptr(o_lat), _ptr(anchor),
+                                      _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
                                       _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "lca_prefill_block")
     return out

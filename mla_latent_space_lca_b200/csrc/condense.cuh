@@ -27,9 +27,9 @@ constexpr int CD_GROUP_BYTES = 16 * LCA_D * 2;                      // 18432
 constexpr int CD_SMEM = CD_WARPS * CD_SLOTS * CD_GROUP_BYTES + CD_WARPS * CD_SLOTS * 8;
 
 struct CondenseArgs {
-    const uint16_t *cache;   // [B][L][576]
+    const uint16_t *cache;   // [B][pitch][576], rows 0 .. L-1 of each sequence used
     const float *u;          // [B][576]
-    int64_t L;
+    int64_t pitch;           // rows between consecutive sequences
     int64_t m;               // groups condensed per sequence: j0 .. j0+m-1
     int64_t j0;              // first group
     int64_t stride;          // rows per sequence of rep / anchor / alpha
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
 
     auto issue = [&](int64_t gi, int s) {
         const int64_t b = gi / a.m, j = a.j0 + (gi - b * a.m);
-        const uint16_t *src = a.cache + (size_t(b) * a.L + size_t(j) * 16) * LCA_D;
+        const uint16_t *src = a.cache + (size_t(b) * a.pitch + size_t(j) * 16) * LCA_D;
         const uint32_t bar = smem_u32(&bars[s]);
         mbar_expect_tx(bar, CD_GROUP_BYTES);
         bulk_load(smem_u32(ring + s * CD_GROUP_BYTES), src, CD_GROUP_BYTES, bar, pol);

@@ -241,7 +241,17 @@ PrefillWs prefill_ws_layout(void *ws, int B, int64_t nb, int64_t m_bound)
 bool params_ok(const lca_params &p)
 {
     return p.g >= 1 && p.w >= 0 && std::isfinite(p.scale) && p.scale > 0.f && p.variant >= LCA_VARIANT_LCA &&
-           p.variant <= LCA_VARIANT_SPARSE;
+           p.variant <= LCA_VARIANT_SPARSE && p.cache_pitch >= 0;
+}
+
+// Rows between consecutive sequences of the cache (the packed layout when
+// the caller leaves cache_pitch at 0), and whether it fits sequences of L rows.
+int64_t cache_pitch(const lca_params &p, int64_t L) { return p.cache_pitch > 0 ? p.cache_pitch : L; }
+
+bool pitch_ok(const lca_params &p, int B, int64_t L)
+{
+    const int64_t pitch = cache_pitch(p, L);
+    return pitch >= L && int64_t(B) * pitch < (int64_t(1) << 40);
 }
 
 int64_t num_groups(int64_t L, const lca_params &p)
@@ -268,7 +278,8 @@ int check_ws(void *ws, size_t ws_bytes, size_t need)
 // Shared tail of the decode paths: split-L attention, combine, W_UV GEMM.
 template <int MODE>
 int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const void *q, const void *w_uv, int B,
-                  int64_t L, int64_t m, int64_t win0, float scale, float *out, float *o_lat, int32_t *anchor,
+                  int64_t L, int64_t pitch, int64_t m, int64_t win0, float scale, float *out, float *o_lat,
+                  int32_t *anchor,
                   const DecodeWs &w, cudaStream_t st, int64_t rep_stride = 0, float *lse_out = nullptr)
 {
     int rc = get_encode();
@@ -292,7 +303,7 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
 
     CUtensorMap map_cache, map_rep;
     rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
-                   uint64_t(L) * LCA_D * 2, 64, AT_TILE, 1);
+                   uint64_t(pitch) * LCA_D * 2, 64, AT_TILE, 1);
     if (rc) return rc;
     if (MODE == MODE_REPS && m > 0) {
         // rows per sequence: m, or the capacity of a representative cache
@@ -412,7 +423,7 @@ int mla_decode_attn(const void *cache, const void *q, const void *w_uv, int B, i
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
-    return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, 0, 0, scale, out, o_lat, nullptr, w,
+    return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, L, 0, 0, scale, out, o_lat, nullptr, w,
                                    static_cast<cudaStream_t>(stream));
 }
 
@@ -429,7 +440,7 @@ int lca_condense_append(const void *cache, const void *q_recent, int B, int64_t 
 {
     if (!cache || !q_recent) return LCA_ERR_INVALID_ARG;
     if (B < 1 || L < 1 || L >= (int64_t(1) << 31)) return LCA_ERR_INVALID_ARG;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
     if (p.g != 16) return LCA_ERR_UNSUPPORTED;
     const int64_t m = num_groups(L, p);
     if (j0 < 0 || j0 > m || rep_cap < m) return LCA_ERR_INVALID_ARG;
@@ -448,7 +459,7 @@ int lca_condense_append(const void *cache, const void *q_recent, int B, int64_t 
     CondenseArgs a{};
     a.cache = static_cast<const uint16_t *>(cache);
     a.u = w.u;
-    a.L = L;
+    a.pitch = cache_pitch(p, L);
     a.m = m - j0;
     a.j0 = j0;
     a.stride = rep_cap;
@@ -469,7 +480,7 @@ int lca_decode_stored(const void *cache, const void *rep, int64_t rep_cap, const
 {
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
     if (p.g != 16) return LCA_ERR_UNSUPPORTED;
     const int64_t m = num_groups(L, p);
     if (rep_cap < m || (m > 0 && !rep)) return LCA_ERR_INVALID_ARG;
@@ -478,8 +489,8 @@ int lca_decode_stored(const void *cache, const void *rep, int64_t rep_cap, const
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
-    return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, nullptr, w,
-                                    static_cast<cudaStream_t>(stream), rep_cap);
+    return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, cache_pitch(p, L), m, m * p.g, p.scale, out,
+                                    o_lat, nullptr, w, static_cast<cudaStream_t>(stream), rep_cap);
 }
 
 int lca_decode_attn(const void *cache, const void *rep, const void *q, const void *w_uv, int B, int64_t L,
@@ -487,7 +498,7 @@ int lca_decode_attn(const void *cache, const void *rep, const void *q, const voi
 {
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
     if (p.g != 16) return LCA_ERR_UNSUPPORTED;
     const int64_t m = num_groups(L, p);
     if (m > 0 && !rep) return LCA_ERR_INVALID_ARG;
@@ -496,8 +507,8 @@ int lca_decode_attn(const void *cache, const void *rep, const void *q, const voi
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
-    return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, nullptr, w,
-                                    static_cast<cudaStream_t>(stream));
+    return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, cache_pitch(p, L), m, m * p.g, p.scale, out,
+                                    o_lat, nullptr, w, static_cast<cudaStream_t>(stream));
 }
 
 int lca_decode(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B, int64_t L,
@@ -505,21 +516,26 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
 {
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
     if (p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;   // ablations: lca_condense + lca_decode_attn
-    if (p.g == 1) return mla_decode_attn(cache, q, w_uv, B, L, p.scale, out, o_lat, ws, ws_bytes, stream);
-    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
-    if (!q_recent) return LCA_ERR_INVALID_ARG;
-    if (!aligned16(q_recent) || (o_lat && !aligned16(o_lat)) || (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+    if (p.g != 1 && p.g != 16) return LCA_ERR_UNSUPPORTED;
+    if (p.g != 1 && !q_recent) return LCA_ERR_INVALID_ARG;
+    if ((p.g != 1 && !aligned16(q_recent)) || (o_lat && !aligned16(o_lat)) ||
+        (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
         return LCA_ERR_MISALIGNED;
-    const int64_t m = num_groups(L, p);
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t pitch = cache_pitch(p, L);
+    if (p.g == 1)   // every token its own representative: MLA decode
+        return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, pitch, 0, 0, p.scale, out, o_lat, nullptr,
+                                       w, st);
+    const int64_t m = num_groups(L, p);
     if (m > 0 && (rc = launch_prep(q_recent, B, p, w, st))) return rc;
-    return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, anchor, w, st);
+    return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, pitch, m, m * p.g, p.scale, out, o_lat, anchor,
+                                   w, st);
 }
 
 int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B, int64_t L,
@@ -527,7 +543,7 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
 {
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
     if (p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
     if (B > LCA_NOALLOC_MAX_BATCH) return LCA_ERR_SCRATCH_LIMIT;
     if (p.g != 1 && p.g != 16) return LCA_ERR_UNSUPPORTED;
@@ -542,11 +558,14 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
     DeviceInfo *dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t pitch = cache_pitch(p, L);
     if (p.g == 1)
-        return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, 0, 0, p.scale, out, o_lat, nullptr, w, st);
+        return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, pitch, 0, 0, p.scale, out, o_lat, nullptr,
+                                       w, st);
     const int64_t m = num_groups(L, p);
     if (m > 0 && (rc = launch_prep(q_recent, B, p, w, st))) return rc;
-    return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, m, m * p.g, p.scale, out, o_lat, anchor, w, st);
+    return run_attention<MODE_LCA>(dev, cache, nullptr, q, w_uv, B, L, pitch, m, m * p.g, p.scale, out, o_lat, anchor,
+                                   w, st);
 }
 
 int lca_decode_shard(const void *cache_shard, const void *q_recent, const void *q, int B, int64_t L, int64_t row0,
@@ -557,7 +576,7 @@ int lca_decode_shard(const void *cache_shard, const void *q_recent, const void *
     if (B < 1 || L < 1 || L >= (int64_t(1) << 31) || L_shard < 1 || row0 < 0 || row0 + L_shard > L ||
         int64_t(B) * L_shard >= (int64_t(1) << 40))
         return LCA_ERR_INVALID_ARG;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L_shard)) return LCA_ERR_INVALID_ARG;
     if (p.g != 16 || p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
     const int64_t m = num_groups(L, p), hist_end = m * p.g, row1 = row0 + L_shard;
     // whole groups; a shard that does not reach L lies inside the history,
@@ -578,8 +597,8 @@ int lca_decode_shard(const void *cache_shard, const void *q_recent, const void *
     // the shard is an LCA decode of its own L_shard rows: m_loc groups, then
     // (last shard only) the window; o and lse2 go to the partial record
     float *lse = part + size_t(B) * LCA_HEADS * LCA_DC;
-    return run_attention<MODE_LCA>(dev, cache_shard, nullptr, q, nullptr, B, L_shard, m_loc, m_loc * p.g, p.scale,
-                                   nullptr, part, anchor, w, st, 0, lse);
+    return run_attention<MODE_LCA>(dev, cache_shard, nullptr, q, nullptr, B, L_shard, cache_pitch(p, L_shard), m_loc,
+                                   m_loc * p.g, p.scale, nullptr, part, anchor, w, st, 0, lse);
 }
 
 int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv, float *out, float *o_lat,
@@ -612,7 +631,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
 {
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
-    if (!params_ok(p)) return LCA_ERR_INVALID_ARG;
+    if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
     if (p.g != 16 || p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
     if (q_start < 0 || q_len < 0 || q_start % 16 || q_len % 16 || q_start + q_len > L) return LCA_ERR_INVALID_ARG;
     if (L > (int64_t(1) << 27)) return LCA_ERR_UNSUPPORTED;   // query rows 16 L index a TMA map
@@ -632,12 +651,13 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     const uint16_t *qv = static_cast<const uint16_t *>(q);
 
     CUtensorMap map_cache, map_rows, map_q, map_u, map_w;
-    if ((rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
-                        uint64_t(L) * LCA_D * 2, 64, 64, 1)))
+    const uint64_t seq_bytes = uint64_t(cache_pitch(p, L)) * LCA_D * 2;
+    if ((rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2, seq_bytes, 64, 64,
+                        1)))
         return rc;
     // the condensation's history tiles: CP_ROWS rows
-    if ((rc = make_map3(&map_rows, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
-                        uint64_t(L) * LCA_D * 2, 64, CP_ROWS, 1)))
+    if ((rc = make_map3(&map_rows, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2, seq_bytes, 64,
+                        CP_ROWS, 1)))
         return rc;
     if ((rc = make_map3(&map_q, q, LCA_D, uint64_t(L) * LCA_HEADS, uint64_t(B), uint64_t(LCA_D) * 2,
                         uint64_t(L) * LCA_HEADS * LCA_D * 2, 64, 64, 1)))

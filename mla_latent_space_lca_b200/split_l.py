@@ -51,7 +51,8 @@ def split_l_decode(cache_shard, q_recent, q, w_uv, L: int, row0: int, *, g: int 
                    scale=None, group=None, out=None, ws=None, shard_fn=None, combine_fn=None):
     """One decode step of B sequences whose caches are split across the
     ranks of `group`.  This rank holds rows row0 .. row0 + L_shard - 1 of
-    every sequence (cache_shard [B, L_shard, 576]); q_recent and q are the
+    every sequence (cache_shard [B, L_shard, 576], packed or a view into a
+    larger buffer such as full[:, row0:row1]); q_recent and q are the
     same on every rank.  Returns out [B, 16, 128] (the same on every rank).
     Without an initialised process group (or with one rank) the shard is
     the whole cache and no exchange takes place.

@@ -113,6 +113,23 @@ def test_other_entry_points_reject_bad_arguments(lcalib):
     assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 4080, 32, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
 
 
+def test_cache_pitch_is_checked(lcalib):
+    big = 1 << 30
+    bad = [LcaParams(16, 1024, 0.07, 0, 4000),          # pitch below L = 4096
+           LcaParams(16, 1024, 0.07, 0, -1),            # negative
+           LcaParams(16, 1024, 0.07, 0, 1 << 39)]       # B * pitch beyond 2^40
+    for p in bad:
+        assert call_decode(lcalib, p=p) == _lib.LCA_ERR_INVALID_ARG
+        assert lcalib.lca_condense(A, A, 2, 4096, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+        assert lcalib.lca_decode_attn(A, A, A, A, 2, 4096, p, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+        assert lcalib.lca_prefill_block(A, A, A, 2, 4096, 0, 16, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
+    assert lcalib.lca_workspace_bytes(3, 2, 4096, 0, LcaParams(16, 1024, 0.07, 0, -5)) == 0
+    if not __import__("torch").cuda.is_available():
+        # a valid pitch gets as far as the device check
+        assert call_decode(lcalib, p=LcaParams(16, 1024, 0.07, 0, 5000)) == _lib.LCA_ERR_NO_DEVICE
+        assert call_decode(lcalib, p=LcaParams(1, 0, 0.07, 0, 5000)) == _lib.LCA_ERR_NO_DEVICE
+
+
 def test_shard_entry_points_reject_bad_arguments(lcalib):
     p = LcaParams(16, 1024, 0.07)
     big = 1 << 30
