@@ -51,7 +51,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=None, help="default 20 (decode), 3 (prefill)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_b32_l32k")
-    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-full-copy", type=int, default=2,
+                    help="decode: also time N steps that copy the whole cache in from the host")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stored", action="store_true",
@@ -443,29 +445,59 @@ def run_ours(args, rank, world, local_rank):
     prof = lca.profile_collect()
     lca.profile_enable(False)
 
-    # end to end through the public API: pinned host inputs -> device -> result -> host
-    pin = [t.pin_memory() for t in (inp.cache, inp.q_recent, inp.q)]
+    # end to end through the public API, as a decode loop runs: the cache is
+    # state resident on the device (the prefill wrote it); every step brings
+    # the new token's row (into row L-1 of each sequence), the recent queries
+    # and the query from pinned host memory, decodes, and reads the result
+    # back.  Steps are timed one by one, with the L2 flush between them when
+    # the cache would otherwise stay in L2.
+    pin_row = inp.cache[:, L - 1].contiguous().pin_memory()
+    pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
     h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
     dbuf = [torch.empty_like(t, device=dev) for t in pin]
-    h2d = sum(t.numel() * t.element_size() for t in pin)
+    h2d = pin_row.numel() * 2 + sum(t.numel() * t.element_size() for t in pin)
     d2h = h_out.numel() * 4
-    for _ in range(1):
+
+    def e2e_step():
+        cache[:, L - 1].copy_(pin_row, non_blocking=True)
         for d, h in zip(dbuf, pin):
             d.copy_(h, non_blocking=True)
-        lca.lca_decode(dbuf[0], dbuf[1], dbuf[2], w_uv, scale=inp.scale, out=out, ws=ws)
+        lca.lca_decode(cache, dbuf[0], dbuf[1], w_uv, scale=inp.scale, out=out, ws=ws)
         h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
     torch.cuda.synchronize()
     barrier()
-    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    x0.record(stream)
-    for _ in range(args.e2e_steps):
-        for d, h in zip(dbuf, pin):
-            d.copy_(h, non_blocking=True)
-        lca.lca_decode(dbuf[0], dbuf[1], dbuf[2], w_uv, scale=inp.scale, out=out, ws=ws)
-        h_out.copy_(out, non_blocking=True)
-    x1.record(stream)
+    n_e2e = max(1, args.e2e_steps)
+    xev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+    for a_, b_ in xev:
+        if flush is not None:
+            flush.zero_()
+        a_.record(stream)
+        e2e_step()
+        b_.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / args.e2e_steps, world, dev)
+    e2e_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in xev) / n_e2e, world, dev)
+    assert torch.equal(h_out, out.cpu())
+
+    # for reference: the same step with the whole cache copied in from the host
+    full_ms = None
+    if args.e2e_full_copy:
+        pin_cache = inp.cache.pin_memory()
+        dcache = torch.empty_like(pin_cache, device=dev)
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(args.e2e_full_copy):
+            dcache.copy_(pin_cache, non_blocking=True)
+            for d, h in zip(dbuf, pin):
+                d.copy_(h, non_blocking=True)
+            lca.lca_decode(dcache, dbuf[0], dbuf[1], w_uv, scale=inp.scale, out=out, ws=ws)
+            h_out.copy_(out, non_blocking=True)
+        x1.record(stream)
+        torch.cuda.synchronize()
+        full_ms = max_over_ranks(x0.elapsed_time(x1) / args.e2e_full_copy, world, dev)
+        del dcache, pin_cache
     rc, detail = lca.device_status(clear=True)
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail:#x})")
@@ -500,8 +532,15 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches,
         "clocks": sampler.summary() if sampler else None,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "note": "lca_decode in a decode loop: cache resident on the device; per step the new "
+                        "token's row, q_recent and q in from pinned host memory, out back"},
     }
+    if full_ms is not None:
+        line["e2e_full_cache_copy"] = {
+            "value": tokens / (full_ms / 1e3), "unit": "tokens/s", "ms_per_step": full_ms,
+            "h2d_bytes_per_step": h2d - pin_row.numel() * 2 + B * L * ROW_BYTES, "d2h_bytes_per_step": d2h,
+            "note": "the whole cache copied in from the host every step (bounded by the host link)"}
     if mla is not None:
         line["mla_path"] = {
             "ms_per_step": mla["ms_per_step"], "tokens_per_s": tokens / (mla["ms_per_step"] / 1e3),
@@ -593,23 +632,35 @@ def run_ours_stored(args, rank, world, local_rank):
     prof = lca.profile_collect()
     lca.profile_enable(False)
 
-    # end to end: the step's query and recent queries from pinned memory, out back
+    # end to end, as a decode loop runs: cache and kept representatives
+    # resident on the device; per step the new token's row (into row L-1),
+    # the recent queries and the query from pinned memory, out back; steps
+    # timed one by one with the L2 flush between them
+    pin_row = inp.cache[:, L - 1].contiguous().pin_memory()
     pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
     h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
     dbuf = [torch.empty_like(t, device=dev) for t in pin]
-    h2d = sum(t.numel() * t.element_size() for t in pin)
-    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    x0.record(stream)
-    n_e2e = max(1, args.e2e_steps)
-    for i in range(n_e2e):
+    h2d = pin_row.numel() * 2 + sum(t.numel() * t.element_size() for t in pin)
+
+    def e2e_step():
+        cache[:, L - 1].copy_(pin_row, non_blocking=True)
         for d, h in zip(dbuf, pin):
             d.copy_(h, non_blocking=True)
         lca.lca_decode_stored(cache, rep, dbuf[1], w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
         h_out.copy_(out, non_blocking=True)
-    x1.record(stream)
+
+    for _ in range(3):
+        e2e_step()
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / n_e2e, world, dev)
+    n_e2e = max(1, args.e2e_steps)
+    xev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+    for a_, b_ in xev:
+        flush.zero_()
+        a_.record(stream)
+        e2e_step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in xev) / n_e2e, world, dev)
     rc, detail = lca.device_status(clear=True)
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail:#x})")
@@ -640,7 +691,8 @@ def run_ours_stored(args, rank, world, local_rank):
         "clocks": sampler.summary() if sampler else None,
         "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 4,
-                "note": "cache and representative cache resident on the device (a decode server's state)"},
+                "note": "decode loop: cache and kept representatives resident on the device; per step the new "
+                        "token's row, q_recent and q in from pinned host memory, out back"},
     }
     print(json.dumps(line), flush=True)
 
@@ -736,27 +788,36 @@ def run_ours_split(args, rank, world, local_rank):
         torch.cuda.synchronize()
         fused_ms = sum(a_.elapsed_time(b_) for a_, b_ in fev) / len(fev)
 
-    # end to end: this rank's shard and the queries from pinned host memory
-    pin = [t.pin_memory() for t in (h_shard, inp.q_recent, inp.q)]
+    # end to end, as a decode loop runs: each rank's shard stays resident;
+    # per step the rank holding row L-1 takes the new token's row, every rank
+    # the recent queries and the query, from pinned host memory; out back
+    last = row1 == L
+    pin_row = inp.cache[:, L - 1].contiguous().pin_memory() if last else None
+    pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
     h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
     dbuf = [torch.empty_like(t, device=dev) for t in pin]
-    h2d = sum(t.numel() * t.element_size() for t in pin)
+    h2d = (pin_row.numel() * 2 if last else 0) + sum(t.numel() * t.element_size() for t in pin)
 
     def e2e_step():
+        if last:
+            cache[:, L - 1 - row0].copy_(pin_row, non_blocking=True)
         for d, h in zip(dbuf, pin):
             d.copy_(h, non_blocking=True)
-        step(*dbuf)
+        step(cache, *dbuf)
         h_out.copy_(out, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize()
     barrier()
-    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    x0.record(stream)
-    for _ in range(args.e2e_steps):
+    n_e2e = max(1, args.e2e_steps)
+    xev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+    for a_, b_ in xev:
+        if flush is not None:
+            flush.zero_()
+        a_.record(stream)
         e2e_step()
-    x1.record(stream)
+        b_.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / args.e2e_steps, world, dev)
+    e2e_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in xev) / n_e2e, world, dev)
     rc, detail = lca.device_status(clear=True)
     if rc != 0:
         raise RuntimeError(f"device status {rc} ({detail:#x})")
