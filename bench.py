@@ -446,23 +446,27 @@ def run_ours(args, rank, world, local_rank):
     lca.profile_enable(False)
 
     # end to end through the public API, as a decode loop runs: the cache is
-    # state resident on the device (the prefill wrote it); every step brings
-    # the new token's row (into row L-1 of each sequence), the recent queries
-    # and the query from pinned host memory, decodes, and reads the result
-    # back.  Steps are timed one by one, with the L2 flush between them when
-    # the cache would otherwise stay in L2.
+    # state resident on the device (the prefill wrote it), and so are the
+    # recent queries, kept as a ring (only their mean is used); every step
+    # brings the new token's row (into row L-1 of each sequence) and its
+    # query from pinned host memory, puts the query into the ring's oldest
+    # slot, decodes, and reads the result back.  Steps are timed one by one,
+    # with the L2 flush between them when the cache would otherwise stay in L2.
     pin_row = inp.cache[:, L - 1].contiguous().pin_memory()
-    pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
+    pin_q = inp.q.pin_memory()
+    ring = inp.q_recent.to(dev)
     h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
-    dbuf = [torch.empty_like(t, device=dev) for t in pin]
-    h2d = pin_row.numel() * 2 + sum(t.numel() * t.element_size() for t in pin)
+    dq = torch.empty_like(pin_q, device=dev)
+    h2d = pin_row.numel() * 2 + pin_q.numel() * 2
     d2h = h_out.numel() * 4
+    slot = [0]
 
     def e2e_step():
         cache[:, L - 1].copy_(pin_row, non_blocking=True)
-        for d, h in zip(dbuf, pin):
-            d.copy_(h, non_blocking=True)
-        lca.lca_decode(cache, dbuf[0], dbuf[1], w_uv, scale=inp.scale, out=out, ws=ws)
+        dq.copy_(pin_q, non_blocking=True)
+        ring[:, slot[0]].copy_(dq)
+        slot[0] = (slot[0] + 1) % ring.shape[1]
+        lca.lca_decode(cache, ring, dq, w_uv, scale=inp.scale, out=out, ws=ws)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -481,10 +485,13 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in xev) / n_e2e, world, dev)
     assert torch.equal(h_out, out.cpu())
 
-    # for reference: the same step with the whole cache copied in from the host
+    # for reference: the same step with the whole cache and all recent
+    # queries copied in from the host
     full_ms = None
     if args.e2e_full_copy:
         pin_cache = inp.cache.pin_memory()
+        pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
+        dbuf = [torch.empty_like(t, device=dev) for t in pin]
         dcache = torch.empty_like(pin_cache, device=dev)
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record(stream)
@@ -533,13 +540,14 @@ def run_ours(args, rank, world, local_rank):
         "clocks": sampler.summary() if sampler else None,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "lca_decode in a decode loop: cache resident on the device; per step the new "
-                        "token's row, q_recent and q in from pinned host memory, out back"},
+                "note": "lca_decode in a decode loop: cache and recent-query ring resident on the device; "
+                        "per step the new token's row and query in from pinned host memory, out back"},
     }
     if full_ms is not None:
         line["e2e_full_cache_copy"] = {
             "value": tokens / (full_ms / 1e3), "unit": "tokens/s", "ms_per_step": full_ms,
-            "h2d_bytes_per_step": h2d - pin_row.numel() * 2 + B * L * ROW_BYTES, "d2h_bytes_per_step": d2h,
+            "h2d_bytes_per_step": B * L * ROW_BYTES + (inp.q_recent.numel() + inp.q.numel()) * 2,
+            "d2h_bytes_per_step": d2h,
             "note": "the whole cache copied in from the host every step (bounded by the host link)"}
     if mla is not None:
         line["mla_path"] = {
@@ -632,21 +640,29 @@ def run_ours_stored(args, rank, world, local_rank):
     prof = lca.profile_collect()
     lca.profile_enable(False)
 
-    # end to end, as a decode loop runs: cache and kept representatives
-    # resident on the device; per step the new token's row (into row L-1),
-    # the recent queries and the query from pinned memory, out back; steps
-    # timed one by one with the L2 flush between them
+    # end to end, as a decode loop runs: cache, kept representatives and the
+    # recent-query ring resident on the device; per step the new token's row
+    # (into row L-1) and its query from pinned memory, the query into the
+    # ring's oldest slot, every 16th step the append of the group that left
+    # the window, the decode, out back; steps timed one by one with the L2
+    # flush between them
     pin_row = inp.cache[:, L - 1].contiguous().pin_memory()
-    pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
+    pin_q = inp.q.pin_memory()
+    ring = q_recent.clone()
+    dq = torch.empty_like(pin_q, device=dev)
     h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
-    dbuf = [torch.empty_like(t, device=dev) for t in pin]
-    h2d = pin_row.numel() * 2 + sum(t.numel() * t.element_size() for t in pin)
+    h2d = pin_row.numel() * 2 + pin_q.numel() * 2
+    n_step = [0]
 
     def e2e_step():
+        i = n_step[0]
+        n_step[0] += 1
         cache[:, L - 1].copy_(pin_row, non_blocking=True)
-        for d, h in zip(dbuf, pin):
-            d.copy_(h, non_blocking=True)
-        lca.lca_decode_stored(cache, rep, dbuf[1], w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+        dq.copy_(pin_q, non_blocking=True)
+        ring[:, i % ring.shape[1]].copy_(dq)
+        if i % 16 == 15 and m > 0:
+            lca.lca_condense_append(cache, ring, rep, m - 1, scale=inp.scale, ws=ws, stream=stream)
+        lca.lca_decode_stored(cache, rep, dq, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -691,8 +707,9 @@ def run_ours_stored(args, rank, world, local_rank):
         "clocks": sampler.summary() if sampler else None,
         "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 4,
-                "note": "decode loop: cache and kept representatives resident on the device; per step the new "
-                        "token's row, q_recent and q in from pinned host memory, out back"},
+                "note": "decode loop: cache, kept representatives and recent-query ring resident on the "
+                        "device; per step the new token's row and query in from pinned host memory (every "
+                        "16th step also the append of one group), out back"},
     }
     print(json.dumps(line), flush=True)
 
@@ -788,22 +805,26 @@ def run_ours_split(args, rank, world, local_rank):
         torch.cuda.synchronize()
         fused_ms = sum(a_.elapsed_time(b_) for a_, b_ in fev) / len(fev)
 
-    # end to end, as a decode loop runs: each rank's shard stays resident;
-    # per step the rank holding row L-1 takes the new token's row, every rank
-    # the recent queries and the query, from pinned host memory; out back
+    # end to end, as a decode loop runs: each rank's shard and its
+    # recent-query ring stay resident; per step the rank holding row L-1
+    # takes the new token's row, every rank the query (into the ring's oldest
+    # slot), from pinned host memory; out back
     last = row1 == L
     pin_row = inp.cache[:, L - 1].contiguous().pin_memory() if last else None
-    pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
+    pin_q = inp.q.pin_memory()
+    ring = q_recent.clone()
+    dq = torch.empty_like(pin_q, device=dev)
     h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
-    dbuf = [torch.empty_like(t, device=dev) for t in pin]
-    h2d = (pin_row.numel() * 2 if last else 0) + sum(t.numel() * t.element_size() for t in pin)
+    h2d = (pin_row.numel() * 2 if last else 0) + pin_q.numel() * 2
+    n_step = [0]
 
     def e2e_step():
         if last:
             cache[:, L - 1 - row0].copy_(pin_row, non_blocking=True)
-        for d, h in zip(dbuf, pin):
-            d.copy_(h, non_blocking=True)
-        step(cache, *dbuf)
+        dq.copy_(pin_q, non_blocking=True)
+        ring[:, n_step[0] % ring.shape[1]].copy_(dq)
+        n_step[0] += 1
+        step(cache, ring, dq)
         h_out.copy_(out, non_blocking=True)
     e2e_step()
     torch.cuda.synchronize()

@@ -130,7 +130,10 @@ int mla_decode_attn(const void *cache, const void *q, const void *w_uv, int B, i
 /* LCA condensation (关键设计 1 and 2) of the m history groups of each
  * sequence with the summary query qbar = mean of q_recent:
  *   cache    [B][L][576] bf16
- *   q_recent [B][g][16][576] bf16 (the last g queries, current one last)
+ *   q_recent [B][g][16][576] bf16: the last g queries (current one
+ *            included).  Only their mean is used, so the order of the g
+ *            slots does not matter: a decode loop may keep q_recent on the
+ *            device as a ring and overwrite the oldest slot each step.
  *   rep      [B][m][576] bf16  out: [c_rep (512) | k^R of the anchor (64)],
  *            the latent rounded to bf16 like a cache row, the key copied
  *            bit for bit

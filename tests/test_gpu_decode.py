@@ -267,6 +267,24 @@ def test_reference_max_rescale_on_consecutive_tiles():
     compare(mla.cpu().numpy(), mla_ref, "mla out")
 
 
+def test_q_recent_slot_order_is_irrelevant():
+    """The summary query is the mean of the g recent queries, so a ring
+    buffer (any rotation or order of the slots) gives the same decode up to
+    the fp32 summation order."""
+    inp = make_decode_inputs(3, 7000, seed=23, peak=10.0)
+    cache, q_recent, q, w_uv = dev(inp)
+    ring = torch.roll(q_recent, shifts=5, dims=1).contiguous()
+    perm = q_recent[:, torch.randperm(16, generator=torch.Generator().manual_seed(3))].contiguous()
+    outs = [api.lca_decode(cache, qr, q, w_uv, scale=inp.scale) for qr in (q_recent, ring, perm)]
+    torch.cuda.synchronize()
+    c, qr, qb, wb = bits(inp)
+    _, out_ref, _ = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    for o in outs:
+        compare(o.cpu().numpy(), out_ref, "out")
+        a, b = o.double().cpu().numpy(), outs[0].double().cpu().numpy()
+        assert np.linalg.norm(a - b) / np.linalg.norm(b) <= 1e-3
+
+
 def test_fused_equals_condense_then_attend():
     """The fused pass and condense -> attend over stored reps agree up to the
     bf16 rounding of stored representatives."""
