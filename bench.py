@@ -62,6 +62,8 @@ def parse():
                     help="decode: also time N steps of the unfused path (condense, then attend stored reps)")
     ap.add_argument("--split-l", action="store_true",
                     help="decode: every sequence's cache split along L over the ranks (strong scaling)")
+    ap.add_argument("--split-blocks", action="store_true",
+                    help="prefill: one prompt's query blocks split over the ranks by work (strong scaling)")
     ap.add_argument("--mla-compare", type=int, default=0,
                     help="decode: also time N plain MLA decode steps (g = 1, every row attended) on the "
                          "same inputs; prefill: N full causal MLA prefills (w = L)")
@@ -77,20 +79,22 @@ def measured_tensor_peak():
         return 1400.0, "fallback (sustained)"
 
 
-def prefill_flops(L: int, w: int, g: int = 16):
+def prefill_flops(L: int, w: int, k0: int = 0, k1: int | None = None, g: int = 16):
     """Algorithmic flops of a blockwise prefill over [0, L): block k has
     m_k = max(0, floor((16k - w)/16)) representatives; its query t attends
     m_k + (t - 16 m_k + 1) keys, each 16 heads x (576 + 512) x 2 flops; the
     condensation scores (folded summary query, 576 x 2) and pools (512 x 2)
-    every history row of the block; W_UV is 16 x 512 x 128 x 2 per query."""
+    every history row of the block; W_UV is 16 x 512 x 128 x 2 per query.
+    Blocks k0 .. k1-1 (default: all)."""
     cw = -(-w // 16)
     att = cond = 0
-    for k in range(L // 16):
+    k1 = L // 16 if k1 is None else k1
+    for k in range(k0, k1):
         m = max(0, k - cw)
         keys = 16 * m + sum(16 * k + tt - 16 * m + 1 for tt in range(16))
         att += keys * 16 * (576 + 512) * 2
         cond += 16 * m * (576 + 512) * 2
-    wuv = L * 16 * 512 * 128 * 2
+    wuv = 16 * (k1 - k0) * 16 * 512 * 128 * 2
     return {"attention": att, "condense": cond, "wuv": wuv}
 
 
@@ -880,22 +884,29 @@ def run_ours_split(args, rank, world, local_rank):
 
 
 def run_ours_prefill(args, rank, world, local_rank):
+    """Blockwise prefill of B prompts of L tokens.  Replicas by default (each
+    rank its own prompts); with --split-blocks every rank holds the same
+    prompt and computes its work-balanced range of query blocks (strong
+    scaling, no data-path collective)."""
     import torch.distributed as dist
 
     import mla_latent_space_lca_b200 as lca
+    from mla_latent_space_lca_b200.split_blocks import prefill_block_ranges
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     wl = WORKLOADS[args.workload]
     B, L = wl["B"], wl["L"]
-    inp = make_prefill_inputs(B, L, seed=replica_seed(rank))
+    split = args.split_blocks
+    inp = make_prefill_inputs(B, L, seed=0 if split else replica_seed(rank))
+    qs, ql = prefill_block_ranges(L, world)[rank] if split else (0, L)
     cache, q, w_uv = inp.cache.to(dev), inp.q.to(dev), inp.w_uv.to(dev)
-    ws = lca.workspace(4, B, L, L, device=dev)
-    out = torch.empty(B, L, 16, 128, dtype=torch.float32, device=dev)
+    ws = lca.workspace(4, B, L, ql, device=dev)
+    out = torch.empty(B, ql, 16, 128, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        lca.lca_prefill_block(cache, q, w_uv, 0, L, scale=inp.scale, out=out, ws=ws, stream=stream)
+        lca.lca_prefill_block(cache, q, w_uv, qs, ql, scale=inp.scale, out=out, ws=ws, stream=stream)
 
     def barrier():
         if world > 1:
@@ -933,17 +944,19 @@ def run_ours_prefill(args, rank, world, local_rank):
     prof = lca.profile_collect()
     lca.profile_enable(False)
 
-    # end to end: cache and queries from pinned host memory, out back to host
-    pin = [t.pin_memory() for t in (inp.cache, inp.q)]
-    h_out = torch.empty(B, L, 16, 128, dtype=torch.float32).pin_memory()
-    dbuf = [torch.empty_like(t, device=dev) for t in pin]
+    # end to end: the cache rows the range reads (0 .. qs+ql-1) and its
+    # queries from pinned host memory, its output rows back to host
+    pin = [inp.cache[:, :qs + ql].pin_memory(), inp.q[:, qs:qs + ql].pin_memory()]
+    h_out = torch.empty(B, ql, 16, 128, dtype=torch.float32).pin_memory()
+    dcache = torch.empty_like(inp.cache, device=dev)
+    dq = torch.empty_like(inp.q, device=dev)
     h2d = sum(t.numel() * t.element_size() for t in pin)
     d2h = h_out.numel() * 4
 
     def e2e_step():
-        for d, h in zip(dbuf, pin):
-            d.copy_(h, non_blocking=True)
-        lca.lca_prefill_block(dbuf[0], dbuf[1], w_uv, 0, L, scale=inp.scale, out=out, ws=ws)
+        dcache[:, :qs + ql].copy_(pin[0], non_blocking=True)
+        dq[:, qs:qs + ql].copy_(pin[1], non_blocking=True)
+        lca.lca_prefill_block(dcache, dq, w_uv, qs, ql, scale=inp.scale, out=out, ws=ws)
         h_out.copy_(out, non_blocking=True)
 
     e2e_step()
@@ -960,7 +973,7 @@ def run_ours_prefill(args, rank, world, local_rank):
     # in-run comparison: full causal MLA prefill over the same inputs (the same
     # path with a window covering the whole sequence, so nothing is condensed)
     mla_ms = None
-    if args.mla_compare:
+    if args.mla_compare and not split:
         ws_mla = lca.workspace(4, B, L, L, w=L, device=dev)
 
         def mla_step():
@@ -982,9 +995,11 @@ def run_ours_prefill(args, rank, world, local_rank):
         raise RuntimeError(f"device status {rc} ({detail:#x})")
     if rank != 0:
         return
-    tokens = B * L * world
-    fl = prefill_flops(L, inp.w)
-    step_flops = B * sum(fl.values())
+    tokens = B * L * (1 if split else world)
+    fl = prefill_flops(L, inp.w, qs // 16, (qs + ql) // 16)   # rank 0's blocks
+    step_flops = B * sum(fl.values()) * (1 if split else world)
+    if split:   # the whole job's flops: every rank's range
+        step_flops = B * sum(prefill_flops(L, inp.w).values())
     peak, peak_kind = measured_tensor_peak()
     attn = prof.get("attn_prefill")
     attn_ms = attn[1] / attn[0] if attn else None
@@ -993,10 +1008,12 @@ def run_ours_prefill(args, rank, world, local_rank):
     line = {
         "metric": PREFILL_METRIC, "value": tokens / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if split else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "B_per_gpu": B, "L": L, "q_len": L, "g": 16, "w": 1024,
-                   "heads": 16, "d_c": 512, "d_r": 64, "parallelism": f"replicas x{world}",
+                   "heads": 16, "d_c": 512, "d_r": 64,
+                   "parallelism": f"split-blocks x{world}" if split else f"replicas x{world}",
+                   "rank0_queries": [qs, qs + ql],
                    "l2": "queries (B*L*16*1152 B) and representatives far larger than the 126 MB L2; no flush"},
         "step_tflops": step_flops / (ms / 1e3) / 1e12,
         "roofline": {"bound": "tensor", "kernel": "attn_prefill", "achieved": achieved, "peak": peak,

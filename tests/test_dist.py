@@ -1,7 +1,8 @@
 """Multi-process host logic on CPU (gloo, world sizes 2 and 3): the timing
 reduction takes the slowest rank, replicas draw distinct batches, and the
-decode split along the cache gathers and merges every rank's shard record
-(the oracle stands in for the kernels)."""
+decode split along the cache gathers and merges every rank's shard record,
+and a prefill split over query blocks reassembles the whole prefill (the
+oracle stands in for the kernels)."""
 import math
 import os
 import sys
@@ -137,3 +138,66 @@ def test_shard_bounds():
         shard_bounds(1024 + 32, 4)      # two groups, four shards
     with pytest.raises(ValueError):
         shard_bounds(80, 6, 16, 0)      # five groups and no window row for a sixth shard
+
+
+# ------------------------------------------------ prefill split over query blocks
+def test_prefill_block_ranges():
+    sys.path.insert(0, ROOT)
+    from mla_latent_space_lca_b200.split_blocks import block_flops, prefill_block_ranges
+    for L, n, w in [(131072, 8, 1024), (16384, 4, 1024), (2048, 3, 256), (4096 + 7, 5, 100), (64, 4, 0)]:
+        r = prefill_block_ranges(L, n, w=w)
+        assert len(r) == n and r[0][0] == 0 and sum(ql for _, ql in r) == 16 * (L // 16)
+        for (s0, l0), (s1, _) in zip(r[:-1], r[1:]):
+            assert s0 + l0 == s1 and l0 > 0 and s0 % 16 == 0 and l0 % 16 == 0
+        work = [sum(block_flops(k, w=w) for k in range(s // 16, (s + ql) // 16)) for s, ql in r]
+        if L // 16 >= 64 * n:      # enough blocks: balanced to a block's work
+            assert max(work) - min(work) <= 2 * max(block_flops(k, w=w) for k in range(L // 16))
+    with pytest.raises(ValueError):
+        prefill_block_ranges(48, 4)
+
+
+def _prefill_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from mla_latent_space_lca_b200.inputs import bf16_bits, make_prefill_inputs
+        from mla_latent_space_lca_b200.split_blocks import prefill_block_ranges
+        inp = make_prefill_inputs(1, 384, w=64, seed=51)
+        qs, ql = prefill_block_ranges(384, world, w=64)[rank]
+        _, out, _ = oracle.lca_prefill(bf16_bits(inp.cache), bf16_bits(inp.q), bf16_bits(inp.w_uv), qs, ql,
+                                       16, 64, inp.scale, want_olat=False)
+        rows = [None] * world
+        dist.all_gather_object(rows, (qs, out))
+        q.put((rank, rows))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_prefill_ranges_reassemble_the_full_prefill():
+    """Each rank prefills its work-balanced range of query blocks (the oracle
+    stands in for the kernels); the gathered rows equal one prefill of the
+    whole prompt."""
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits, make_prefill_inputs
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 33500 + os.getpid() % 2000
+    procs = [ctx.Process(target=_prefill_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=300) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    inp = make_prefill_inputs(1, 384, w=64, seed=51)
+    _, full, _ = oracle.lca_prefill(bf16_bits(inp.cache), bf16_bits(inp.q), bf16_bits(inp.w_uv), 0, 384,
+                                    16, 64, inp.scale, want_olat=False)
+    for _, rows in res:
+        got = np.concatenate([out for _, out in sorted(rows, key=lambda x: x[0])], axis=1)
+        np.testing.assert_allclose(got, full, rtol=0, atol=1e-12)

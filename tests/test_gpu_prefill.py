@@ -123,6 +123,17 @@ def test_prefill_range_split_consistency():
     torch.testing.assert_close(torch.cat([a, b], dim=1), full, rtol=0, atol=0)
 
 
+def test_prefill_split_over_ranks_by_work():
+    """The work-balanced ranges a split over three devices would take (with
+    chunk edges inside them) give, concatenated, the rows of one call."""
+    from mla_latent_space_lca_b200.split_blocks import prefill_block_ranges
+    B, L, w = 2, 16 * 700, 512
+    inp = make_prefill_inputs(B, L, w=w, seed=48)
+    full, _, _ = run_gpu(inp, 0, L, w)
+    parts = [run_gpu(inp, qs, ql, w)[0] for qs, ql in prefill_block_ranges(L, 3, w=w)]
+    torch.testing.assert_close(torch.cat(parts, dim=1), full, rtol=0, atol=0)
+
+
 def test_prefill_full_size_sampled():
     """The 128K-token prefill (B = 1, L = 131072, w = 1024) in one call, the
     launch configuration the benchmark times; the oracle checks sampled
