@@ -191,6 +191,23 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
                int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor, void *ws,
                size_t ws_bytes, void *stream);
 
+/* lca_decode for a ragged batch: sequence b holds lens[b] cached rows
+ * (1 <= lens[b] <= L; values outside are clamped), at rows 0 .. lens[b]-1
+ * of its cache, [B][pitch][576] with pitch = cache_pitch or L.  Each
+ * sequence is decoded exactly as lca_decode would decode it alone: its own
+ * m_b = lca_num_groups(lens[b], p) groups and window; its query sits at
+ * position lens[b]-1.  (Not part of the page's method: a serving batch holds
+ * sequences of different lengths.)
+ *   lens   [B] int32, a DEVICE array (4-byte aligned), read by the kernels
+ *   anchor [B][m] int32 or NULL with m = lca_num_groups(L, p): row b holds
+ *          sequence b's m_b anchors (the rest of the row is not written)
+ * g == 1 is MLA decode of each sequence's lens[b] rows.  Otherwise requires
+ * g == 16 and variant LCA.  B * (L / 64 + 2) < 2^31 (LCA_ERR_UNSUPPORTED
+ * otherwise).  ws: LCA_OP_DECODE bytes for (B, L). */
+int lca_decode_varlen(const void *cache, const int32_t *lens, const void *q_recent, const void *q,
+                      const void *w_uv, int B, int64_t L, lca_params p, float *out, float *o_lat,
+                      int32_t *anchor, void *ws, size_t ws_bytes, void *stream);
+
 /* Blockwise LCA prefill of query positions [q_start, q_start + q_len) (both
  * multiples of g).  The page reports prefill speed but does not spell out the
  * procedure; this is its plainest reading.  Block k covers t0 = k*g ..

@@ -189,6 +189,27 @@ def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     return out
 
 
+def lca_decode_varlen(cache, lens, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None,
+                      anchor=None, ws=None, stream=None):
+    """Decode of a ragged batch: sequence b holds lens[b] rows (int32 CUDA
+    tensor [B]) at rows 0 .. lens[b]-1 of cache [B, L, 576] (packed, or a
+    view into a larger buffer); L is the largest length the buffer holds."""
+    B, L, _ = cache.shape
+    pitch = _cache(cache)
+    _need(lens, "lens", torch.int32, (B,))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    if g != 1:
+        _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_decode_varlen(_ptr(cache), _ptr(lens), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
+                                      _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
+                                      _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "lca_decode_varlen")
+    return out
+
+
 def shard_record_floats(B: int) -> int:
     """Floats in one shard record: o [B][16][512] then lse2 [B][16]."""
     return B * H * _lib.SHARD_RECORD_PER_HEAD

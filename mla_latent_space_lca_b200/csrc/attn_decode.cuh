@@ -77,8 +77,9 @@ enum { MODE_MLA = 0, MODE_REPS = 1, MODE_LCA = 2 };
 struct AttnArgs {
     const uint16_t *q;     // [B][16][576]
     const uint16_t *uhl;   // [B][2][576] (LCA)
-    int64_t L;
-    int64_t m;             // representatives / groups per sequence (0 for MLA)
+    int64_t L;             // rows per sequence (varlen: the largest length)
+    int64_t m;             // representatives / groups per sequence (0 for MLA); varlen: the
+                           // anchor row stride (groups of the largest length)
     int64_t win0;          // first window row (m*g), 0 for MLA
     int n_hist;            // tiles before the window per sequence
     int n_tiles;           // tiles per sequence
@@ -88,7 +89,85 @@ struct AttnArgs {
     float *part_o;         // [G+B][16][512]
     float *part_ml;        // [G+B][16][2]
     int32_t *anchor;       // [B][m] or NULL (LCA)
+    // ragged batches only: sequence b holds lens[b] rows (clamped to
+    // [1, L]) and tiles tile_start[b] .. tile_start[b+1]-1 of the batch's
+    // tile list; T = tile_start[B]
+    const int32_t *lens;
+    const int32_t *tile_start;
+    int B;
+    int w;
 };
+
+// Geometry of one sequence of L rows: its groups m, first window row and
+// tiles before the window (history tiles of 4 groups, or stored
+// representative tiles of 64 rows), and its tile count.
+struct SeqGeom {
+    int64_t L, m, win0;
+    int n_hist, n_tiles;
+};
+
+template <int MODE>
+__host__ __device__ __forceinline__ SeqGeom seq_geom(int64_t L, int w)
+{
+    SeqGeom g;
+    g.L = L;
+    g.m = (MODE == MODE_MLA || L <= w) ? 0 : (L - w) / 16;
+    g.win0 = 16 * g.m;
+    g.n_hist = MODE == MODE_MLA ? 0 : MODE == MODE_REPS ? int((g.m + AT_TILE - 1) / AT_TILE) : int((g.m + 3) / 4);
+    g.n_tiles = g.n_hist + int((L - g.win0 + AT_TILE - 1) / AT_TILE);
+    return g;
+}
+
+// The tiles [t0, t1) of sequence b, with its geometry.
+struct SeqTiles {
+    int64_t b, t0, t1;
+    SeqGeom g;
+};
+
+__device__ __forceinline__ int64_t clamp_len(int32_t len, int64_t L)
+{
+    return len < 1 ? 1 : (int64_t(len) > L ? L : int64_t(len));
+}
+
+// The sequence that tile t belongs to.  Each role walks its tiles in
+// increasing order, so a ragged batch advances from the previous answer
+// (cur.b < 0 the first time: a binary search over tile_start).
+template <int MODE, bool VARLEN>
+__device__ __forceinline__ SeqTiles seq_of(const AttnArgs &a, int64_t t, const SeqTiles &cur)
+{
+    SeqTiles s;
+    if constexpr (!VARLEN) {
+        s.b = t / a.n_tiles;
+        s.t0 = s.b * a.n_tiles;
+        s.t1 = s.t0 + a.n_tiles;
+        s.g.L = a.L;
+        s.g.m = a.m;
+        s.g.win0 = a.win0;
+        s.g.n_hist = a.n_hist;
+        s.g.n_tiles = a.n_tiles;
+        return s;
+    } else {
+        if (cur.b >= 0 && t >= cur.t0 && t < cur.t1) return cur;
+        int64_t b;
+        if (cur.b < 0) {
+            int lo = 0, hi = a.B - 1;   // the last b with tile_start[b] <= t
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (a.tile_start[mid] <= t) lo = mid;
+                else hi = mid - 1;
+            }
+            b = lo;
+        } else {
+            b = cur.b;
+            while (b + 1 < a.B && a.tile_start[b + 1] <= t) ++b;
+        }
+        s.b = b;
+        s.t0 = a.tile_start[b];
+        s.t1 = a.tile_start[b + 1];
+        s.g = seq_geom<MODE>(clamp_len(a.lens[b], a.L), a.w);
+        return s;
+    }
+}
 
 struct TileInfo {
     int from_rep;   // 1: rows come from the representative tensor
@@ -98,7 +177,7 @@ struct TileInfo {
 };
 
 template <int MODE>
-__device__ __forceinline__ TileInfo tile_info(const AttnArgs &a, int k)
+__device__ __forceinline__ TileInfo tile_info(const SeqGeom &a, int k)
 {
     TileInfo ti;
     ti.from_rep = 0;
@@ -169,7 +248,7 @@ __device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int qu
     }
 }
 
-template <int MODE>
+template <int MODE, bool VARLEN = false>
 __global__ void __launch_bounds__(AT_THREADS, 1)
     attn_decode_kernel(const __grid_constant__ CUtensorMap map_cache,
                        const __grid_constant__ CUtensorMap map_rep, const AttnArgs a)
@@ -230,10 +309,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const uint32_t tmem = *tmem_slot;
     griddep_launch_dependents();
 
+    // a ragged batch's tile list comes from the kernel before: wait for it
+    // (and so for everything earlier in the stream) before reading it
+    if constexpr (VARLEN) griddep_wait();
+    const int64_t T = VARLEN ? int64_t(a.tile_start[a.B]) : a.T;
     const int c = blockIdx.x;
-    const int64_t t_begin = split_begin(c, a.T, a.G);
-    const int64_t t_end = split_begin(c + 1, a.T, a.G);
-    const int n_tiles = a.n_tiles;
+    const int64_t t_begin = split_begin(c, T, a.G);
+    const int64_t t_end = split_begin(c + 1, T, a.G);
 
     if (warp == 5) {
         // ------------------------------------------------------------ TMA producer
@@ -246,11 +328,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             const uint64_t pol = policy_evict_first();
             int last[3] = {-1, -1, -1};
             int i = 0;
+            SeqTiles sq{};
+            sq.b = -1;
             for (int64_t t = t_begin; t < t_end; ++t, ++i) {
                 const int s = i % 3;
                 if (!mbar_wait(empty(s), ((i / 3) & 1) ^ 1, abort_flag, K_ATTN, 1)) break;
-                const int64_t b = t / n_tiles;
-                const TileInfo ti = tile_info<MODE>(a, int(t - b * n_tiles));
+                sq = seq_of<MODE, VARLEN>(a, t, sq);
+                const int64_t b = sq.b;
+                const TileInfo ti = tile_info<MODE>(sq.g, int(t - sq.t0));
                 mbar_expect_tx(full(s), AT_STAGE);
                 const CUtensorMap *mp = ti.from_rep ? &map_rep : &map_cache;
                 const uint32_t dst = sbase + s * AT_STAGE;
@@ -269,8 +354,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             const int half = (warp == 7) ? 1 : 0;
             constexpr uint32_t IDESC_S = idesc_bf16(64, AT_TILE, 0, 0);
             int i = 0, seg = 0;
+            SeqTiles sq{};
+            sq.b = -1;
             for (int64_t t = t_begin; t < t_end; ++t, ++i) {
-                const bool first = (i == 0) || (t % n_tiles == 0);
+                sq = seq_of<MODE, VARLEN>(a, t, sq);
+                const bool first = (i == 0) || (t == sq.t0);
                 if (first && !mbar_wait(segready, seg++ & 1, abort_flag, K_ATTN, 3)) break;
                 if (!mbar_wait(full(i % 3), (i / 3) & 1, abort_flag, K_ATTN, 4)) break;
                 if (!mbar_wait(sempty(i & 1), ((i >> 1) & 1) ^ 1, abort_flag, K_ATTN, 5)) break;
@@ -298,9 +386,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             const int cc = (warp == 6) ? 0 : warp - 7;
             constexpr uint32_t IDESC_PV = idesc_bf16(128, LCA_HEADS, 1, 0);
             int j = 0, first_j = 0;
+            SeqTiles sq{};
+            sq.b = -1;
             for (int64_t t = t_begin; t < t_end; ++t, ++j) {
-                if (j == 0 || t % n_tiles == 0) first_j = j;
-                const bool last = (t + 1 == t_end) || ((t + 1) % n_tiles == 0);
+                sq = seq_of<MODE, VARLEN>(a, t, sq);
+                if (j == 0 || t == sq.t0) first_j = j;
+                const bool last = (t + 1 == t_end) || (t + 1 == sq.t1);
                 if (!mbar_wait(pfull(j & 1), (j >> 1) & 1, abort_flag, K_ATTN, 7)) break;
                 tc_fence_after();
                 const uint32_t stage = sbase + (j % 3) * AT_STAGE;
@@ -329,9 +420,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         bool ok = true;
         float m_use = NEG_INF, l_run = 0.f;   // threads with lane/4 < 4: head 4*quad + lane/4
         griddep_wait();   // the folded summary query comes from the previous kernel
+        SeqTiles sq{};
+        sq.b = -1;
         while (ok && t < t_end) {
-            const int64_t b = t / n_tiles;
-            const int64_t seg_end = min64(t_end, (b + 1) * int64_t(n_tiles));
+            sq = seq_of<MODE, VARLEN>(a, t, sq);
+            const int64_t b = sq.b;
+            const int64_t seg_end = min64(t_end, sq.t1);
             load_q_rows<MODE>(a, b, quad, lane, tmem);
             tc_fence_before();
             __syncwarp();
@@ -340,9 +434,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             l_run = 0.f;
             const int first = i;
             for (; t < seg_end; ++t, ++i) {
-                const int k = int(t - b * n_tiles);
+                const int k = int(t - sq.t0);
                 const int sb = i & 1;
-                const TileInfo ti = tile_info<MODE>(a, k);
+                const TileInfo ti = tile_info<MODE>(sq.g, k);
                 ok = mbar_wait(sfull(sb), (i >> 1) & 1, abort_flag, K_ATTN, 8);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
@@ -373,6 +467,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sempty(sb));
+                if constexpr (VARLEN) {
+                    // Rows past this sequence's end lie inside the tensor map
+                    // (it spans the longest sequence) and may hold anything.
+                    // Their P weights are 0, but 0 * NaN is NaN in the PV MMA,
+                    // so zero them in the stage's 8 latent boxes; S has read
+                    // the stage, and the proxy fence before pfull orders these
+                    // stores before PV.
+                    const int ok_rows = int(min64(AT_TILE, sq.g.L - ti.row));
+                    if (ok_rows < AT_TILE) {
+                        const int nr = AT_TILE - ok_rows;
+                        uint8_t *stg = smem + (i % 3) * AT_STAGE;
+                        for (int x = 32 * quad + lane; x < 8 * nr * 8; x += 128) {
+                            const int box = x / (8 * nr), r = ok_rows + (x / 8) % nr, ch = x % 8;
+                            *reinterpret_cast<uint4 *>(stg + box * AT_CHUNK + r * 128 + ch * 16) =
+                                make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                }
 
                 float w[16];        // P^T weights of this thread's head and tokens (g < 4)
                 float f = 1.f;      // reference-max rescale factor of this head

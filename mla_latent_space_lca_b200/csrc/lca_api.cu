@@ -21,6 +21,7 @@
 #include "wuv_gemm.cuh"
 #include "prefill.cuh"
 #include "selftest.cuh"
+#include "varlen.cuh"
 
 using namespace lca;
 
@@ -63,6 +64,8 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_MLA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_REPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_MLA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
         good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(tail_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TD_SMEM_ALLOC) == cudaSuccess;
@@ -180,6 +183,7 @@ struct DecodeWs {
     float *part_o;
     float *part_ml;
     uint16_t *o_bf16;
+    int32_t *tile_start;   // [B+1], ragged batches only
     size_t bytes;
 };
 
@@ -187,14 +191,15 @@ DecodeWs decode_ws_layout(void *ws, int B)
 {
     DecodeWs w{};
     const size_t slots = size_t(kMaxCtas) + size_t(B);
-    size_t off[6];
+    size_t off[7];
     off[0] = 0;
     off[1] = off[0] + align_up(size_t(B) * LCA_D * 4);                 // u
     off[2] = off[1] + align_up(size_t(B) * 2 * LCA_D * 2);             // uhl
     off[3] = off[2] + align_up(slots * LCA_HEADS * LCA_DC * 4);         // part_o
     off[4] = off[3] + align_up(slots * LCA_HEADS * 2 * 4);              // part_ml
     off[5] = off[4] + align_up(size_t(B) * LCA_HEADS * LCA_DC * 2);     // o_bf16
-    w.bytes = off[5];
+    off[6] = off[5] + align_up((size_t(B) + 1) * 4);                    // tile_start
+    w.bytes = off[6];
     if (ws) {
         uint8_t *p = static_cast<uint8_t *>(ws);
         w.u = reinterpret_cast<float *>(p + off[0]);
@@ -202,6 +207,7 @@ DecodeWs decode_ws_layout(void *ws, int B)
         w.part_o = reinterpret_cast<float *>(p + off[2]);
         w.part_ml = reinterpret_cast<float *>(p + off[3]);
         w.o_bf16 = reinterpret_cast<uint16_t *>(p + off[4]);
+        w.tile_start = reinterpret_cast<int32_t *>(p + off[5]);
     }
     return w;
 }
@@ -276,11 +282,16 @@ int check_ws(void *ws, size_t ws_bytes, size_t need)
 }
 
 // Shared tail of the decode paths: split-L attention, combine, W_UV GEMM.
-template <int MODE>
+// Ragged batches (VARLEN): `lens` holds each sequence's length on the device,
+// L and m are the largest length and its group count (the anchor row
+// stride), and the tile offsets in w.tile_start were written by
+// varlen_tiles_kernel just before; `window` is the local window w.
+template <int MODE, bool VARLEN = false>
 int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const void *q, const void *w_uv, int B,
                   int64_t L, int64_t pitch, int64_t m, int64_t win0, float scale, float *out, float *o_lat,
                   int32_t *anchor,
-                  const DecodeWs &w, cudaStream_t st, int64_t rep_stride = 0, float *lse_out = nullptr)
+                  const DecodeWs &w, cudaStream_t st, int64_t rep_stride = 0, float *lse_out = nullptr,
+                  const int32_t *lens = nullptr, int window = 0)
 {
     int rc = get_encode();
     if (rc) return rc;
@@ -295,11 +306,17 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     else a.n_hist = int((m + 3) / 4);
     a.n_tiles = a.n_hist + int((L - win0 + AT_TILE - 1) / AT_TILE);
     a.T = int64_t(B) * a.n_tiles;
-    a.G = int(std::min<int64_t>(std::min<int64_t>(dev->sms, kMaxCtas), a.T));
+    // a ragged batch's tile count is known on the device only: one CTA per
+    // SM, each reading its range of the tile list
+    a.G = int(std::min<int64_t>(std::min<int64_t>(dev->sms, kMaxCtas), VARLEN ? int64_t(kMaxCtas) : a.T));
     a.sl2 = scale * 1.4426950408889634f;
     a.part_o = w.part_o;
     a.part_ml = w.part_ml;
     a.anchor = anchor;
+    a.lens = lens;
+    a.tile_start = VARLEN ? w.tile_start : nullptr;
+    a.B = B;
+    a.w = window;
 
     CUtensorMap map_cache, map_rep;
     rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
@@ -318,8 +335,8 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
         Launch l(st, K_ATTN);
         // after the summary-query kernel (LCA) the attention prologue and its
         // first cache loads overlap it
-        const cudaError_t e = launch_ex(attn_decode_kernel<MODE>, dim3(a.G), dim3(AT_THREADS), AT_SMEM_ALLOC, st,
-                                        MODE == MODE_LCA && m > 0, map_cache, map_rep, a);
+        const cudaError_t e = launch_ex(attn_decode_kernel<MODE, VARLEN>, dim3(a.G), dim3(AT_THREADS), AT_SMEM_ALLOC,
+                                        st, VARLEN || (MODE == MODE_LCA && m > 0), map_cache, map_rep, a);
         if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     CUtensorMap map_w = map_cache;   // unused when out is NULL (a shard's partial)
@@ -332,7 +349,7 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
         const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + rpc - 1) / rpc), dim3(256),
                                         TD_SMEM_ALLOC, st, true, map_w, (const float *)w.part_o,
                                         (const float *)w.part_ml, B, a.n_tiles, a.T, a.G, o_lat, out, rpc,
-                                        lse_out, 0, int64_t(0));
+                                        lse_out, 0, int64_t(0), (const int32_t *)a.tile_start);
         if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     return LCA_OK;
@@ -359,7 +376,7 @@ constexpr size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 constexpr size_t noalloc_scratch_bytes(size_t B)
 {
     return al256(B * LCA_D * 4) + al256(B * 2 * LCA_D * 2) + al256((kMaxCtas + B) * LCA_HEADS * LCA_DC * 4) +
-           al256((kMaxCtas + B) * LCA_HEADS * 2 * 4) + al256(B * LCA_HEADS * LCA_DC * 2);
+           al256((kMaxCtas + B) * LCA_HEADS * 2 * 4) + al256(B * LCA_HEADS * LCA_DC * 2) + al256((B + 1) * 4);
 }
 constexpr size_t kNoAllocBytes = noalloc_scratch_bytes(LCA_NOALLOC_MAX_BATCH);
 
@@ -538,6 +555,44 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
                                    w, st);
 }
 
+int lca_decode_varlen(const void *cache, const int32_t *lens, const void *q_recent, const void *q, const void *w_uv,
+                      int B, int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor, void *ws,
+                      size_t ws_bytes, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!lens || !params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
+    if (p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
+    if (p.g != 1 && p.g != 16) return LCA_ERR_UNSUPPORTED;
+    if (p.g != 1 && !q_recent) return LCA_ERR_INVALID_ARG;
+    // tile offsets are int32: the whole batch's tiles must stay below 2^31
+    if (int64_t(B) * (L / AT_TILE + 2) >= (int64_t(1) << 31)) return LCA_ERR_UNSUPPORTED;
+    if ((p.g != 1 && !aligned16(q_recent)) || (o_lat && !aligned16(o_lat)) ||
+        (reinterpret_cast<uintptr_t>(lens) & 3u) || (anchor && (reinterpret_cast<uintptr_t>(anchor) & 3u)))
+        return LCA_ERR_MISALIGNED;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t pitch = cache_pitch(p, L);
+    {
+        Launch l(st, K_PREP);
+        if (p.g == 1)
+            varlen_tiles_kernel<MODE_MLA><<<1, VT_THREADS, 0, st>>>(lens, B, L, p.w, w.tile_start);
+        else
+            varlen_tiles_kernel<MODE_LCA><<<1, VT_THREADS, 0, st>>>(lens, B, L, p.w, w.tile_start);
+        if ((rc = l.done())) return rc;
+    }
+    if (p.g == 1)
+        return run_attention<MODE_MLA, true>(dev, cache, nullptr, q, w_uv, B, L, pitch, 0, 0, p.scale, out, o_lat,
+                                             nullptr, w, st, 0, nullptr, lens, p.w);
+    const int64_t m = num_groups(L, p);   // the anchor row stride
+    if ((rc = launch_prep(q_recent, B, p, w, st))) return rc;
+    return run_attention<MODE_LCA, true>(dev, cache, nullptr, q, w_uv, B, L, pitch, m, m * p.g, p.scale, out, o_lat,
+                                         anchor, w, st, 0, nullptr, lens, p.w);
+}
+
 int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B, int64_t L,
                        lca_params p, float *out, float *o_lat, int32_t *anchor, void *stream)
 {
@@ -620,7 +675,8 @@ int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv
     const int64_t stride = int64_t(B) * LCA_HEADS * LCA_SHARD_RECORD_PER_HEAD;
     const cudaError_t e = launch_ex(tail_decode_kernel, dim3(LCA_HEADS, (B + rpc - 1) / rpc), dim3(256),
                                     TD_SMEM_ALLOC, st, false, map_w, parts, (const float *)nullptr, B, 0,
-                                    int64_t(0), 0, o_lat, out, rpc, (float *)nullptr, n_shards, stride);
+                                    int64_t(0), 0, o_lat, out, rpc, (float *)nullptr, n_shards, stride,
+                                    (const int32_t *)nullptr);
     if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     return LCA_OK;
 }

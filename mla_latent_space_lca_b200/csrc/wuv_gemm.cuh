@@ -145,6 +145,8 @@ __global__ void __launch_bounds__(128, 1)
 //    workspace: record s starts at part_o + s * shard_stride and holds o
 //    [B][16][512] followed by lse2 [B][16] (part_ml is unused); each acts as
 //    a slot with maximum lse2 and denominator 1.
+// For a ragged batch tile_start (B+1 offsets into the batch's tile list)
+// replaces the uniform b * n_tiles.
 constexpr int TD_ROWS = 8;
 constexpr int TD_N = 16;
 constexpr int TD_A = LCA_DC * LCA_DV * 2;               // 131072
@@ -161,7 +163,8 @@ __global__ void __launch_bounds__(256, 1)
     tail_decode_kernel(const __grid_constant__ CUtensorMap map_w, const float *__restrict__ part_o,
                        const float *__restrict__ part_ml, int B, int n_tiles, int64_t T, int G,
                        float *__restrict__ o_lat, float *__restrict__ out, int rpc,
-                       float *__restrict__ lse_out, int n_shards, int64_t shard_stride)
+                       float *__restrict__ lse_out, int n_shards, int64_t shard_stride,
+                       const int32_t *__restrict__ tile_start)
 {
     extern __shared__ uint8_t td_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -216,8 +219,14 @@ __global__ void __launch_bounds__(256, 1)
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         if (r < nb) {
             const int b = b0 + r;
-            const int c0 = n_shards ? 0 : split_owner(int64_t(b) * n_tiles, T, G);
-            const int ns = n_shards ? n_shards : split_owner(int64_t(b + 1) * n_tiles - 1, T, G) - c0 + 1;
+            int64_t s0 = int64_t(b) * n_tiles, s1 = int64_t(b + 1) * n_tiles, TT = T;
+            if (tile_start) {
+                s0 = tile_start[b];
+                s1 = tile_start[b + 1];
+                TT = tile_start[B];
+            }
+            const int c0 = n_shards ? 0 : split_owner(s0, TT, G);
+            const int ns = n_shards ? n_shards : split_owner(s1 - 1, TT, G) - c0 + 1;
             const int mine = (ns - sub + wpr - 1) / wpr;   // slots sub, sub+wpr, ...
             for (int base = 0; base < mine; base += 32) {
                 const int cnt = min(32, mine - base);

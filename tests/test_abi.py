@@ -113,6 +113,27 @@ def test_other_entry_points_reject_bad_arguments(lcalib):
     assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 4080, 32, p, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
 
 
+def test_varlen_rejects_bad_arguments(lcalib):
+    p = LcaParams(16, 1024, 0.07)
+    big = 1 << 30
+
+    def call(**kw):
+        a = dict(cache=A, lens=A, q_recent=A, q=A, w_uv=A, B=2, L=4096, p=p, out=A, ws_bytes=big)
+        a.update(kw)
+        return lcalib.lca_decode_varlen(a["cache"], a["lens"], a["q_recent"], a["q"], a["w_uv"], a["B"], a["L"],
+                                        a["p"], a["out"], None, None, A, a["ws_bytes"], None)
+    assert call(lens=None) == _lib.LCA_ERR_INVALID_ARG
+    assert call(q_recent=None) == _lib.LCA_ERR_INVALID_ARG
+    assert call(lens=A + 2) == _lib.LCA_ERR_MISALIGNED
+    assert call(p=LcaParams(8, 1024, 0.07)) == _lib.LCA_ERR_UNSUPPORTED
+    assert call(p=LcaParams(16, 1024, 0.07, _lib.VARIANT_SPARSE)) == _lib.LCA_ERR_UNSUPPORTED
+    assert call(B=1 << 17, L=1 << 20) == _lib.LCA_ERR_UNSUPPORTED     # tile offsets past 2^31
+    assert call(ws_bytes=16) == _lib.LCA_ERR_WORKSPACE
+    if not __import__("torch").cuda.is_available():
+        assert call() == _lib.LCA_ERR_NO_DEVICE
+        assert call(q_recent=None, p=LcaParams(1, 0, 0.07)) == _lib.LCA_ERR_NO_DEVICE
+
+
 def test_cache_pitch_is_checked(lcalib):
     big = 1 << 30
     bad = [LcaParams(16, 1024, 0.07, 0, 4000),          # pitch below L = 4096
