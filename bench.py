@@ -60,6 +60,8 @@ def parse():
                     help="decode: stored-representative mode (groups condensed once and kept)")
     ap.add_argument("--unfused-compare", type=int, default=0,
                     help="decode: also time N steps of the unfused path (condense, then attend stored reps)")
+    ap.add_argument("--varlen", action="store_true",
+                    help="decode: a ragged batch, lengths drawn uniformly from [L/8, 15L/8] (mean L)")
     ap.add_argument("--split-l", action="store_true",
                     help="decode: every sequence's cache split along L over the ranks (strong scaling)")
     ap.add_argument("--split-blocks", action="store_true",
@@ -718,6 +720,139 @@ def run_ours_stored(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_ours_varlen(args, rank, world, local_rank):
+    """Decode of a ragged batch (lca_decode_varlen): B sequences whose
+    lengths are drawn, seeded, uniformly from [L/8, 15L/8] (mean L), held in
+    one [B, 15L/8, 576] buffer.  Algorithmic bytes: the rows each sequence
+    holds, read once."""
+    import torch.distributed as dist
+
+    import mla_latent_space_lca_b200 as lca
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = WORKLOADS[args.workload]
+    assert wl["kind"] == "decode"
+    B, L = wl["B"], wl["L"]
+    L_max = L // 8 * 15
+    gen = torch.Generator().manual_seed(1000 + replica_seed(rank))
+    lens = torch.randint(L // 8, L_max + 1, (B,), generator=gen, dtype=torch.int32)
+    inp = make_decode_inputs(B, L_max, seed=replica_seed(rank))
+    cache, q_recent, q, w_uv = (inp.cache.to(dev), inp.q_recent.to(dev), inp.q.to(dev), inp.w_uv.to(dev))
+    lens_d = lens.to(dev)
+    rows = int(lens.sum())
+    ws = lca.workspace(3, B, L_max, device=dev)
+    out = torch.empty(B, 16, 128, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        lca.lca_decode_varlen(cache, lens_d, q_recent, q, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    time.sleep(0.25 if sampler else 0)
+    n0 = lca.launch_count()
+    if sampler:
+        sampler.mark()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark()
+    launches = (lca.launch_count() - n0) / args.steps
+    barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    if sampler:
+        sampler.stop()
+    lca.profile_enable(True)
+    for _ in range(min(args.steps, 200)):
+        step()
+    torch.cuda.synchronize()
+    prof = lca.profile_collect()
+    lca.profile_enable(False)
+
+    # end to end, as a decode loop runs: cache and recent-query ring resident;
+    # per step each sequence's new row (at its own last position) and its
+    # query in from pinned host memory, out back
+    idx = torch.arange(B, device=dev)
+    last_row = (lens_d - 1).long()
+    pin_rows = inp.cache[torch.arange(B), (lens - 1).long()].contiguous().pin_memory()
+    pin_q = inp.q.pin_memory()
+    ring = q_recent.clone()
+    drows = torch.empty_like(pin_rows, device=dev)
+    dq = torch.empty_like(pin_q, device=dev)
+    h_out = torch.empty(B, 16, 128, dtype=torch.float32).pin_memory()
+    h2d = pin_rows.numel() * 2 + pin_q.numel() * 2
+    n_step = [0]
+
+    def e2e_step():
+        drows.copy_(pin_rows, non_blocking=True)
+        cache[idx, last_row] = drows
+        dq.copy_(pin_q, non_blocking=True)
+        ring[:, n_step[0] % ring.shape[1]].copy_(dq)
+        n_step[0] += 1
+        lca.lca_decode_varlen(cache, lens_d, ring, dq, w_uv, scale=inp.scale, out=out, ws=ws)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    n_e2e = max(1, args.e2e_steps)
+    for _ in range(n_e2e):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1) / n_e2e, world, dev)
+    rc, detail = lca.device_status(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} ({detail:#x})")
+    if rank != 0:
+        return
+    peak, peak_kind = measured_hbm_peak()
+    attn = prof.get("attn_decode")
+    attn_ms = attn[1] / attn[0] if attn else None
+    algo_bytes = rows * ROW_BYTES
+    achieved = algo_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
+    line = {
+        "metric": METRIC, "value": B * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "mode": "ragged batch", "B_per_gpu": B,
+                   "lengths": f"uniform in [{L // 8}, {L_max}] (seeded), total {rows} rows",
+                   "g": 16, "w": 1024, "parallelism": f"replicas x{world}",
+                   "l2": "cache rows far larger than the 126 MB L2; no flush"},
+        "cache_gbps": algo_bytes * world / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA, ragged)", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / peak if achieved else None, "traffic": None,
+                     "algorithmic_bytes_per_launch": algo_bytes, "launch_ms": attn_ms},
+        "kernels_ms_per_step": {k: v[1] / v[0] for k, v in prof.items()},
+        "gpu_launches": launches,
+        "clocks": sampler.summary() if sampler else None,
+        "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 4,
+                "note": "decode loop: cache and recent-query ring resident; per step each sequence's new row "
+                        "and query in from pinned host memory, out back"},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ours_split(args, rank, world, local_rank):
     """Decode with every sequence's cache split along L over the ranks: rank r
     holds rows shard_bounds(L, world)[r] of the same B sequences; a step is
@@ -1063,7 +1198,8 @@ def main():
         if prefill:
             fn = run_ours_prefill
         else:
-            fn = run_ours_stored if args.stored else (run_ours_split if args.split_l else run_ours)
+            fn = (run_ours_stored if args.stored else run_ours_split if args.split_l else
+                  run_ours_varlen if args.varlen else run_ours)
         fn(args, rank, world, local_rank)
     finally:
         if world > 1:
