@@ -208,6 +208,18 @@ int lca_decode_varlen(const void *cache, const int32_t *lens, const void *q_rece
                       const void *w_uv, int B, int64_t L, lca_params p, float *out, float *o_lat,
                       int32_t *anchor, void *ws, size_t ws_bytes, void *stream);
 
+/* lca_decode_stored for a ragged batch: sequence b holds lens[b] cached rows
+ * (clamped to [1, L]) and its first m_b = lca_num_groups(lens[b], p)
+ * representatives in rep [B][rep_cap][576] (rep_cap >= lca_num_groups(L,
+ * p)); its query attends [rep rows 0 .. m_b-1 || cache rows 16 m_b ..
+ * lens[b]-1], then W_UV.  lens is a DEVICE int32 array [B].  A decode loop
+ * appends a sequence's groups with lca_condense_append on that sequence's
+ * views when its length crosses a group boundary.  Requires g == 16 and
+ * B * (L / 64 + 2) < 2^31.  ws: LCA_OP_DECODE_ATTN bytes for (B, L). */
+int lca_decode_stored_varlen(const void *cache, const void *rep, int64_t rep_cap, const int32_t *lens,
+                             const void *q, const void *w_uv, int B, int64_t L, lca_params p, float *out,
+                             float *o_lat, void *ws, size_t ws_bytes, void *stream);
+
 /* Blockwise LCA prefill of query positions [q_start, q_start + q_len) (both
  * multiples of g).  The page reports prefill speed but does not spell out the
  * procedure; this is its plainest reading.  Block k covers t0 = k*g ..

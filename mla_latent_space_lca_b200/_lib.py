@@ -31,7 +31,8 @@ EXPORTS = ("lca_num_groups", "lca_workspace_bytes", "mla_decode_attn", "lca_cond
            "lca_decode_attn", "lca_decode", "lca_prefill_block", "lca_strerror",
            "lca_device_status", "lca_profile_enable", "lca_profile_collect", "lca_launch_count",
            "lca_decode_noalloc", "lca_condense_append", "lca_decode_stored",
-           "lca_selftest_wait_timeout", "lca_decode_shard", "lca_combine_shards", "lca_decode_varlen")
+           "lca_selftest_wait_timeout", "lca_decode_shard", "lca_combine_shards", "lca_decode_varlen",
+           "lca_decode_stored_varlen")
 # floats per head in a shard record: o (512) and its base-2 log-sum-exp
 SHARD_RECORD_PER_HEAD = 513
 
@@ -72,6 +73,8 @@ def lib():
         L.mla_decode_attn.argtypes = [P, P, P, I, I64, F, P, P, P, SZ, P]
         L.lca_condense.restype = I
         L.lca_condense.argtypes = [P, P, I, I64, LcaParams, P, P, P, P, SZ, P]
+        L.lca_decode_stored_varlen.restype = I
+        L.lca_decode_stored_varlen.argtypes = [P, P, I64, P, P, P, I, I64, LcaParams, P, P, P, SZ, P]
         L.lca_decode_varlen.restype = I
         L.lca_decode_varlen.argtypes = [P, P, P, P, P, I, I64, LcaParams, P, P, P, P, SZ, P]
         L.lca_decode_shard.restype = I

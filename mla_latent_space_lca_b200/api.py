@@ -210,6 +210,26 @@ def lca_decode_varlen(cache, lens, q_recent, q, w_uv, g=16, w=1024, scale=None, 
     return out
 
 
+def lca_decode_stored_varlen(cache, rep, lens, q, w_uv, g=16, w=1024, scale=None, out=None, o_lat=None,
+                             ws=None, stream=None):
+    """Stored-representative decode of a ragged batch: sequence b holds
+    lens[b] rows of cache [B, L, 576] and its first num_groups(lens[b])
+    representatives in rep [B, rep_cap, 576]."""
+    B, L, _ = cache.shape
+    pitch = _cache(cache)
+    _need(lens, "lens", torch.int32, (B,))
+    _need(q, "q", torch.bfloat16, (B, H, D))
+    _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
+    _need(rep, "rep", torch.bfloat16)
+    out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
+    rc = _lib.lib().lca_decode_stored_varlen(_ptr(cache), _ptr(rep), rep.shape[1], _ptr(lens), _ptr(q),
+                                             _ptr(w_uv), B, L, _params(g, w, scale, 0, pitch), _ptr(out),
+                                             _ptr(o_lat), _ptr(ws), ws.numel(), _stream(stream))
+    check(rc, "lca_decode_stored_varlen")
+    return out
+
+
 def shard_record_floats(B: int) -> int:
     """Floats in one shard record: o [B][16][512] then lse2 [B][16]."""
     return B * H * _lib.SHARD_RECORD_PER_HEAD

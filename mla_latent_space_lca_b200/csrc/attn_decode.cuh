@@ -468,13 +468,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(sempty(sb));
                 if constexpr (VARLEN) {
-                    // Rows past this sequence's end lie inside the tensor map
-                    // (it spans the longest sequence) and may hold anything.
+                    // Rows past this sequence's end (or past its kept
+                    // representatives) lie inside the tensor map, which spans
+                    // the longest sequence, and may hold anything.
                     // Their P weights are 0, but 0 * NaN is NaN in the PV MMA,
                     // so zero them in the stage's 8 latent boxes; S has read
                     // the stage, and the proxy fence before pfull orders these
                     // stores before PV.
-                    const int ok_rows = int(min64(AT_TILE, sq.g.L - ti.row));
+                    const int ok_rows = ti.from_rep ? ti.valid : int(min64(AT_TILE, sq.g.L - ti.row));
                     if (ok_rows < AT_TILE) {
                         const int nr = AT_TILE - ok_rows;
                         uint8_t *stg = smem + (i % 3) * AT_STAGE;

@@ -66,6 +66,7 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_MLA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
+        good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_REPS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
         good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(tail_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TD_SMEM_ALLOC) == cudaSuccess;
@@ -591,6 +592,33 @@ int lca_decode_varlen(const void *cache, const int32_t *lens, const void *q_rece
     if ((rc = launch_prep(q_recent, B, p, w, st))) return rc;
     return run_attention<MODE_LCA, true>(dev, cache, nullptr, q, w_uv, B, L, pitch, m, m * p.g, p.scale, out, o_lat,
                                          anchor, w, st, 0, nullptr, lens, p.w);
+}
+
+int lca_decode_stored_varlen(const void *cache, const void *rep, int64_t rep_cap, const int32_t *lens, const void *q,
+                             const void *w_uv, int B, int64_t L, lca_params p, float *out, float *o_lat, void *ws,
+                             size_t ws_bytes, void *stream)
+{
+    int rc = check_common(cache, q, w_uv, B, L, out);
+    if (rc) return rc;
+    if (!lens || !params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
+    const int64_t m = num_groups(L, p);   // the longest sequence's groups
+    if (rep_cap < m || (m > 0 && !rep)) return LCA_ERR_INVALID_ARG;
+    if (int64_t(B) * (L / AT_TILE + 2) >= (int64_t(1) << 31)) return LCA_ERR_UNSUPPORTED;
+    if ((rep && !aligned16(rep)) || (o_lat && !aligned16(o_lat)) || (reinterpret_cast<uintptr_t>(lens) & 3u))
+        return LCA_ERR_MISALIGNED;
+    const DecodeWs w = decode_ws_layout(ws, B);
+    if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
+    DeviceInfo *dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    {
+        Launch l(st, K_PREP);
+        varlen_tiles_kernel<MODE_REPS><<<1, VT_THREADS, 0, st>>>(lens, B, L, p.w, w.tile_start);
+        if ((rc = l.done())) return rc;
+    }
+    return run_attention<MODE_REPS, true>(dev, cache, rep, q, w_uv, B, L, cache_pitch(p, L), m, m * p.g, p.scale,
+                                          out, o_lat, nullptr, w, st, rep_cap, nullptr, lens, p.w);
 }
 
 int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, const void *w_uv, int B, int64_t L,

@@ -236,7 +236,9 @@ __global__ void __launch_bounds__(256, 1)
                     if (n_shards) {
                         m = part_o[size_t(s) * shard_stride + lse_off + size_t(b) * LCA_HEADS + h];
                         l = 1.f;
-                    } else {
+                    } else if (split_begin(c0 + s + 1, TT, G) > split_begin(c0 + s, TT, G)) {
+                        // (a ragged batch can have fewer tiles than CTAs: a CTA
+                        // owning none wrote no slot, and its slot is skipped)
                         const size_t sl = size_t(c0 + s + b) * LCA_HEADS + h;
                         const float2 ml = *reinterpret_cast<const float2 *>(part_ml + sl * 2);
                         m = ml.x;
@@ -246,6 +248,7 @@ __global__ void __launch_bounds__(256, 1)
                 float Mc = m;
 #pragma unroll
                 for (int off = 16; off; off >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, off));
+                if (Mc == -INFINITY) continue;   // every slot of the chunk skipped (warp-uniform)
                 const float Mn = fmaxf(M, Mc);
                 const float sc = fast_exp2(M - Mn);   // rescale the earlier chunks (0 at first)
                 den *= sc;
@@ -260,6 +263,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll 4
                 for (int k = 0; k < cnt; ++k) {
                     const float wk = __shfl_sync(0xffffffffu, wl, k);
+                    if (wk == 0.f) continue;   // warp-uniform: skipped slots contribute nothing
                     const int s = sub + wpr * (base + k);
                     const float *rec = n_shards ? part_o + size_t(s) * shard_stride + (size_t(b) * LCA_HEADS + h) * LCA_DC
                                                 : part_o + (size_t(c0 + s + b) * LCA_HEADS + h) * LCA_DC;

@@ -11,7 +11,9 @@ would show. Checks:
 - equal lengths reproduce lca_decode bit for bit;
 - g = 1 is MLA decode of each sequence's rows;
 - a batch with more sequences than SMs and lengths from 1 to 3000 matches
-  the single-sequence GPU calls.
+  the single-sequence GPU calls;
+- the stored-representative mode (lca_decode_stored_varlen), with NaN in the
+  representative cache past each sequence's groups.
 """
 import numpy as np
 import pytest
@@ -121,3 +123,56 @@ def test_many_sequences_match_single_calls():
         # its attention weights to bf16 (2^-9 relative) independently
         assert np.linalg.norm(a - r) / np.linalg.norm(r) <= 2.0 ** -8, (b, n)
         compare(out[b:b + 1], one.cpu().numpy(), f"seq {b} (len {n}) vs its own call")
+
+
+def test_ragged_stored_decode():
+    """Stored representatives for a ragged batch: each sequence's groups are
+    appended by a call on its own views (as a decode loop does when its
+    length crosses a group boundary); rows of the representative cache past
+    each sequence's groups hold NaN."""
+    L = 6000
+    lens = [1, 900, 1040, 3017, 6000, 2222]
+    B = len(lens)
+    inp = make_decode_inputs(B, L, seed=105, peak=10.0)
+    cache = ragged(inp, lens)
+    q_recent, q, w_uv = inp.q_recent.cuda(), inp.q.cuda(), inp.w_uv.cuda()
+    cap = api.num_groups(L) + 7
+    rep = torch.empty(B, cap, 576, dtype=torch.bfloat16, device="cuda")
+    rep.view(torch.int16).fill_(NAN_BF16)
+    for b, n in enumerate(lens):
+        if api.num_groups(n) > 0:
+            api.lca_condense_append(cache[b:b + 1, :n], q_recent[b:b + 1], rep[b:b + 1], 0, scale=inp.scale)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    o_lat = torch.empty(B, 16, 512, device="cuda")
+    out = api.lca_decode_stored_varlen(cache, rep, lens_d, q, w_uv, scale=inp.scale, o_lat=o_lat)
+    torch.cuda.synchronize()
+    for b, n in enumerate(lens):
+        mb = api.num_groups(n)
+        c = bf16_bits(inp.cache[b:b + 1, :n])
+        rep_bits = rep[b:b + 1, :mb].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        ol_ref, out_ref = oracle.lca_attend_reps(c, rep_bits, bf16_bits(inp.q[b:b + 1]), bf16_bits(inp.w_uv), 16,
+                                                 1024, inp.scale)
+        compare(o_lat[b:b + 1].cpu().numpy(), ol_ref, f"stored o_lat seq {b} (len {n})")
+        compare(out[b:b + 1].cpu().numpy(), out_ref, f"stored out seq {b} (len {n})")
+        one = api.lca_decode_stored(cache[b:b + 1, :n], rep[b:b + 1], q[b:b + 1], w_uv, scale=inp.scale)
+        torch.cuda.synchronize()
+        compare(out[b:b + 1].cpu().numpy(), one.cpu().numpy(), f"stored seq {b} vs its own call")
+
+
+@pytest.mark.parametrize("g", [16, 1])
+def test_fewer_tiles_than_ctas(g):
+    """A ragged batch whose whole tile list is shorter than the grid: CTAs
+    that own no tile write no partial slot, and the merge must skip them."""
+    L = 1200
+    lens = [5, 700, 1100, 64, 1200]
+    inp = make_decode_inputs(len(lens), L, seed=106, peak=10.0)
+    out, o_lat, _ = run(inp, lens, g=g)
+    for b, n in enumerate(lens):
+        c = bf16_bits(inp.cache[b:b + 1, :n])
+        qb, wb = bf16_bits(inp.q[b:b + 1]), bf16_bits(inp.w_uv)
+        if g == 1:
+            ol_ref, out_ref = oracle.mla_decode(c, qb, wb, inp.scale)
+        else:
+            ol_ref, out_ref, _ = oracle.lca_decode(c, bf16_bits(inp.q_recent[b:b + 1]), qb, wb, 16, 1024, inp.scale)
+        compare(o_lat[b:b + 1], ol_ref, f"o_lat seq {b} (len {n})")
+        compare(out[b:b + 1], out_ref, f"out seq {b} (len {n})")
