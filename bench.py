@@ -536,6 +536,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": ("inputs (B*L*1152 B) larger than the 126 MB L2; no flush" if flush is None else
                           "flushed (256 MB write) before every step; steps timed one by one")},
         "cache_gbps": gbs, "cache_frac_of_hbm": gbs / world / peak,
+        "cache_frac_of_nominal_8tbs": gbs / world / 8000.0,
         "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA)",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak if achieved else None, "traffic": traffic,
@@ -838,6 +839,7 @@ def run_ours_varlen(args, rank, world, local_rank):
                    "g": 16, "w": 1024, "parallelism": f"replicas x{world}",
                    "l2": "cache rows far larger than the 126 MB L2; no flush"},
         "cache_gbps": algo_bytes * world / (ms / 1e3) / 1e9,
+        "cache_frac_of_nominal_8tbs": algo_bytes / (ms / 1e3) / 1e9 / 8000.0,
         "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA, ragged)", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak if achieved else None, "traffic": None,
