@@ -21,10 +21,19 @@
 
 namespace lca {
 
-constexpr int CD_WARPS = 4;
-constexpr int CD_SLOTS = 3;
-constexpr int CD_GROUP_BYTES = 16 * LCA_D * 2;                      // 18432
-constexpr int CD_SMEM = CD_WARPS * CD_SLOTS * CD_GROUP_BYTES + CD_WARPS * CD_SLOTS * 8;
+// Each warp owns S group slots and issues its own copies, so no slot
+// is ever shared between warps.  The per-group arithmetic is a chain of
+// dependent shared-memory loads, FMAs and shuffles; one warp per scheduler
+// cannot hide its latency, so a CTA runs several warps per scheduler.
+template <int W, int S>
+struct CondenseShape {
+    static constexpr int kWarps = W;
+    static constexpr int kSlots = S;
+    static constexpr int kGroupBytes = 16 * LCA_D * 2;                          // 18432
+    static constexpr int kSmem = W * S * kGroupBytes + W * S * 8;
+};
+constexpr int CD_GROUP_BYTES = 16 * LCA_D * 2;
+using CdShape = CondenseShape<12, 1>;    // the shape the library launches
 
 struct CondenseArgs {
     const uint16_t *cache;   // [B][pitch][576], rows 0 .. L-1 of each sequence used
@@ -40,34 +49,44 @@ struct CondenseArgs {
     int variant;             // LCA_VARIANT_*: the method or one of its ablations
 };
 
-__device__ __forceinline__ float dot8(const uint4 x, const float *u)
+// acc + x . u over one 16-byte slice (8 bf16) of a row
+__device__ __forceinline__ float dot8(const uint4 x, const float *u, float acc)
 {
-    float a = bf_lo(x.x) * u[0];
-    a = fmaf(bf_hi(x.x), u[1], a);
-    a = fmaf(bf_lo(x.y), u[2], a);
-    a = fmaf(bf_hi(x.y), u[3], a);
-    a = fmaf(bf_lo(x.z), u[4], a);
-    a = fmaf(bf_hi(x.z), u[5], a);
-    a = fmaf(bf_lo(x.w), u[6], a);
-    a = fmaf(bf_hi(x.w), u[7], a);
-    return a;
+    acc = fmaf(bf_lo(x.x), u[0], acc);
+    acc = fmaf(bf_hi(x.x), u[1], acc);
+    acc = fmaf(bf_lo(x.y), u[2], acc);
+    acc = fmaf(bf_hi(x.y), u[3], acc);
+    acc = fmaf(bf_lo(x.z), u[4], acc);
+    acc = fmaf(bf_hi(x.z), u[5], acc);
+    acc = fmaf(bf_lo(x.w), u[6], acc);
+    acc = fmaf(bf_hi(x.w), u[7], acc);
+    return acc;
 }
 
-__global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const CondenseArgs a)
+__device__ __forceinline__ void load_u8(const float *p, float *uu)
 {
+    const float4 x0 = __ldg(reinterpret_cast<const float4 *>(p)), x1 = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+    uu[0] = x0.x, uu[1] = x0.y, uu[2] = x0.z, uu[3] = x0.w;
+    uu[4] = x1.x, uu[5] = x1.y, uu[6] = x1.z, uu[7] = x1.w;
+}
+
+template <int W, int S>
+__global__ void __launch_bounds__(W * 32, 1) condense_kernel(const CondenseArgs a)
+{
+    using Shape = CondenseShape<W, S>;
     extern __shared__ __align__(128) uint8_t cd_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint8_t *ring = cd_smem + size_t(warp) * CD_SLOTS * CD_GROUP_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(cd_smem + CD_WARPS * CD_SLOTS * CD_GROUP_BYTES) +
-                     warp * CD_SLOTS;
+    uint8_t *ring = cd_smem + size_t(warp) * S * CD_GROUP_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(cd_smem + W * S * CD_GROUP_BYTES) + warp * S;
     if (lane == 0) {
-        for (int s = 0; s < CD_SLOTS; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        for (int s = 0; s < S; ++s) mbar_init(smem_u32(&bars[s]), 1);
         fence_mbar_init();
     }
     __syncwarp();
+    static_assert(Shape::kSmem <= 227 * 1024, "slots exceed shared memory");
 
-    const int64_t nw = int64_t(gridDim.x) * CD_WARPS;
-    const int64_t gw = int64_t(blockIdx.x) * CD_WARPS + warp;
+    const int64_t nw = int64_t(gridDim.x) * W;
+    const int64_t gw = int64_t(blockIdx.x) * W + warp;
     const uint64_t pol = policy_evict_first();
 
     auto issue = [&](int64_t gi, int s) {
@@ -78,45 +97,57 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
         bulk_load(smem_u32(ring + s * CD_GROUP_BYTES), src, CD_GROUP_BYTES, bar, pol);
     };
 
-    int issued_last[CD_SLOTS] = {-1, -1, -1};
+    // the cache rows and u may come from the previous kernel in the stream
+    griddep_wait();
     if (lane == 0) {
-        for (int s = 0; s < CD_SLOTS; ++s) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
             const int64_t gi = gw + s * nw;
-            if (gi < a.total) {
-                issue(gi, s);
-                issued_last[s] = s;
-            }
+            if (gi < a.total) issue(gi, s);
         }
     }
+
+    // this lane's 16-byte column slices of u: lane, lane + 32 (for all 16
+    // rows) and 64 + lane % 8 (for rows 4 (lane / 8) .. + 3), so that the
+    // 16 x 72 slices of a group split evenly, 36 per lane
+    float u0[8], u1[8], u2[8];
+    int64_t ub = -1;
+    const int xrow = 4 * (lane >> 3), xslice = 64 + (lane & 7);
 
     bool ok = true;
     int it = 0;
     for (int64_t gi = gw; gi < a.total; gi += nw, ++it) {
-        const int s = it % CD_SLOTS;
-        ok = mbar_wait(smem_u32(&bars[s]), (it / CD_SLOTS) & 1, nullptr, K_CONDENSE, 1);
+        const int s = it % S;
+        ok = mbar_wait(smem_u32(&bars[s]), (it / S) & 1, nullptr, K_CONDENSE, 1);
         if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
         }
         const int64_t b = gi / a.m, j = a.j0 + (gi - b * a.m);
         const uint8_t *tile = ring + s * CD_GROUP_BYTES;
+        if (b != ub) {
+            const float *ur = a.u + size_t(b) * LCA_D;
+            load_u8(ur + 8 * lane, u0);
+            load_u8(ur + 8 * (lane + 32), u1);
+            load_u8(ur + 8 * xslice, u2);
+            ub = b;
+        }
 
-        // importance: partial dots over this lane's 16-byte column slices
-        // (lane, lane+32 and, for lanes < 8, lane+64 of the 72 slices)
+        // importance: partial dots of the 16 rows over this lane's slices
         float acc[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-#pragma unroll 1
-        for (int r = 0; r < 3; ++r) {
-            const int v = lane + 32 * r;
-            if (v < 72) {
-                const float4 *up = reinterpret_cast<const float4 *>(a.u + size_t(b) * LCA_D + 8 * v);
-                const float4 x0 = __ldg(up), x1 = __ldg(up + 1);
-                const float uu[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        for (int i = 0; i < 16; ++i) {
+            const uint8_t *row = tile + i * (LCA_D * 2);
+            acc[i] = dot8(*reinterpret_cast<const uint4 *>(row + lane * 16), u0, 0.f);
+            acc[i] = dot8(*reinterpret_cast<const uint4 *>(row + (lane + 32) * 16), u1, acc[i]);
+        }
+        {
+            float e[4];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    acc[i] += dot8(*reinterpret_cast<const uint4 *>(tile + i * (LCA_D * 2) + v * 16), uu);
-            }
+            for (int t = 0; t < 4; ++t)
+                e[t] = dot8(*reinterpret_cast<const uint4 *>(tile + (xrow + t) * (LCA_D * 2) + xslice * 16), u2, 0.f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) acc[i] += ((i >> 2) == (lane >> 3)) ? e[i & 3] : 0.f;
         }
         // halving transpose-reduce: after it lanes 2t and 2t+1 hold token t
 #pragma unroll
@@ -223,19 +254,23 @@ __global__ void __launch_bounds__(CD_WARPS * 32, 1) condense_kernel(const Conden
         // release the slot and refill it
         __syncwarp();
         if (lane == 0) {
-            const int64_t nxt = gi + CD_SLOTS * nw;
+            const int64_t nxt = gi + S * nw;
             if (nxt < a.total) {
                 fence_proxy_async();
                 issue(nxt, s);
-                issued_last[s] = it + CD_SLOTS;
             }
         }
     }
     if (!ok && lane == 0) {
-        // a wait expired: let every copy already issued land before exiting
-        for (int s = 0; s < CD_SLOTS; ++s)
-            if (issued_last[s] >= 0)
-                mbar_wait(smem_u32(&bars[s]), (issued_last[s] / CD_SLOTS) & 1, nullptr, K_CONDENSE, 2);
+        // a wait expired at item `it`: items 0 .. it - 1 + S of this warp had
+        // been issued; let the last one of each slot land before exiting
+        const int64_t n = (a.total - gw + nw - 1) / nw;
+        const int64_t hi = min64(int64_t(it) - 1 + S, n - 1);
+        for (int s = 0; s < S; ++s) {
+            if (hi < s) continue;
+            const int64_t i = hi - (hi - s) % S;
+            mbar_wait(smem_u32(&bars[s]), uint32_t(i / S) & 1u, nullptr, K_CONDENSE, 2);
+        }
     }
 }
 

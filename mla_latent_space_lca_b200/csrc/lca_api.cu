@@ -67,7 +67,8 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_MLA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_LCA, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_decode_kernel<MODE_REPS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM_ALLOC) == cudaSuccess;
-        good &= cudaFuncSetAttribute(condense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CD_SMEM) == cudaSuccess;
+        good &= cudaFuncSetAttribute(condense_kernel<CdShape::kWarps, CdShape::kSlots>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, CdShape::kSmem) == cudaSuccess;
         good &= cudaFuncSetAttribute(wuv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GM_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(tail_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TD_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(condense_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CP_SMEM_ALLOC) == cudaSuccess;
@@ -486,10 +487,12 @@ int lca_condense_append(const void *cache, const void *q_recent, int B, int64_t 
     a.anchor = anchor;
     a.alpha = alpha;
     a.variant = p.variant;
-    const int64_t want = (a.total + CD_WARPS - 1) / CD_WARPS;
+    const int64_t want = (a.total + CdShape::kWarps - 1) / CdShape::kWarps;
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(dev->sms, want)));
     Launch l(st, K_CONDENSE);
-    condense_kernel<<<grid, CD_WARPS * 32, CD_SMEM, st>>>(a);
+    if (launch_ex(condense_kernel<CdShape::kWarps, CdShape::kSlots>, dim3(grid), dim3(CdShape::kWarps * 32),
+                  CdShape::kSmem, st, true, a) != cudaSuccess)
+        return LCA_ERR_CUDA;
     return l.done();
 }
 
