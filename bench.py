@@ -389,7 +389,7 @@ def run_ours(args, rank, world, local_rank):
 
     # in-run comparison: the unfused path (condense to stored representatives,
     # then attention over them), which writes and re-reads the representatives
-    unfused_ms = None
+    unfused_ms = condense_ms = None
     if args.unfused_compare and lca.num_groups(L) > 0:
         rep_u = torch.empty(B, lca.num_groups(L), 576, dtype=torch.bfloat16, device=dev)
 
@@ -407,6 +407,14 @@ def run_ours(args, rank, world, local_rank):
         u1.record(stream)
         torch.cuda.synchronize()
         unfused_ms = max_over_ranks(u0.elapsed_time(u1) / args.unfused_compare, world, dev)
+        lca.profile_enable(True)
+        for _ in range(min(args.unfused_compare, 200)):
+            unfused_step()
+        torch.cuda.synchronize()
+        uprof = lca.profile_collect()
+        lca.profile_enable(False)
+        ucond = uprof.get("condense")
+        condense_ms = ucond[1] / ucond[0] if ucond else None
         del rep_u
 
     # in-run comparison: plain MLA decode (g = 1) over the whole cache, the
@@ -572,6 +580,13 @@ def run_ours(args, rank, world, local_rank):
             "algorithmic_bytes_per_step": B * (L + 2 * m) * ROW_BYTES,
             "note": "lca_condense (reads the cache, writes m representatives) then lca_decode_attn "
                     "(re-reads them and the window)"}
+        if condense_ms:
+            # condense_kernel alone: the 16 m history rows read, the m representatives written
+            cbytes = B * 17 * m * ROW_BYTES
+            line["unfused_path"]["condense_kernel"] = {
+                "launch_ms": condense_ms, "algorithmic_bytes_per_launch": cbytes,
+                "achieved_gbs": cbytes / (condense_ms / 1e3) / 1e9,
+                "frac_of_measured_hbm": cbytes / (condense_ms / 1e3) / 1e9 / peak}
     if world == 1 and not args.no_cpu_baseline:
         tok_s, cores, sample, _ = cpu_baseline(inp, args.cpu_seconds)
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
