@@ -59,9 +59,9 @@ def _load():
         lib.ora_lca_decode_stored.argtypes = [P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
         lib.ora_lca_decode_shard.restype = I
         lib.ora_lca_decode_shard.argtypes = [P, P, P, I, Lg, I, I, I, I, I, Dd, Lg, Lg, P, P, P]
-        lib.ora_lca_prefill.restype = I
-        lib.ora_lca_prefill.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, P, Lg,
-                                        P, P, P]
+        lib.ora_lca_prefill_v.restype = I
+        lib.ora_lca_prefill_v.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, I, P, Lg,
+                                          P, P, P]
         _lib = lib
     return _lib
 
@@ -213,9 +213,11 @@ def lca_decode_stored(cache, q_all, w_uv, g: int, w: int, scale: float, dr: int 
 
 
 def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, scale: float,
-                blocks=None, dr: int = 64, want_anchor: bool = False, want_olat: bool = True):
+                blocks=None, dr: int = 64, want_anchor: bool = False, want_olat: bool = True,
+                variant: int = LCA):
     """Blockwise LCA prefill.  -> (o_lat [B,q_len,H,dc] | None, out [B,q_len,H,dv], anchor|None).
-    `blocks` = absolute block indices to evaluate (others left as NaN)."""
+    `blocks` = absolute block indices to evaluate (others left as NaN).
+    `variant`: the method (LCA) or an ablation (POOL_POSITION, SPARSE)."""
     cache, qpre, w_uv = _u16(cache), _u16(qpre), _u16(w_uv)
     B, L, D = cache.shape
     H = qpre.shape[2]
@@ -230,9 +232,9 @@ def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, sca
         nbl = len(bl)
     m_max = num_groups(q_start + q_len - g, g, w)
     anchor = np.full((B, q_len // g, max(m_max, 1)), -1, np.int32) if want_anchor else None
-    rc = _load().ora_lca_prefill(_ptr(cache), _ptr(qpre), _ptr(w_uv), B, L, q_start, q_len, H,
-                                 dc, dr, dv, g, w, scale, _ptr(bl), nbl, _ptr(o_lat), _ptr(out),
-                                 _ptr(anchor))
+    rc = _load().ora_lca_prefill_v(_ptr(cache), _ptr(qpre), _ptr(w_uv), B, L, q_start, q_len, H,
+                                   dc, dr, dv, g, w, scale, int(variant), _ptr(bl), nbl, _ptr(o_lat),
+                                   _ptr(out), _ptr(anchor))
     if rc != 0:
         raise ValueError("bad prefill range")
     return o_lat, out, anchor

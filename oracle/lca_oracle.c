@@ -392,11 +392,12 @@ int ora_lca_attend_reps(const uint16_t *cache, const uint16_t *rep, const uint16
  * o_lat [B][q_len][H][dc], out [B][q_len][H][dv]; rows of blocks that are
  * not processed are left untouched.  anchor_out, if not NULL, receives
  * [B][q_len/g][m_max] absolute anchor positions (m_max = max m_k over the
- * range, unused slots untouched). */
-int ora_lca_prefill(const uint16_t *cache, const uint16_t *qpre, const uint16_t *w_uv, int B,
-                    long L, long q_start, long q_len, int H, int dc, int dr, int dv, int g, int w,
-                    double scale, const int64_t *blocks, long n_blocks, double *o_lat,
-                    double *out, int32_t *anchor_out)
+ * range, unused slots untouched).  `variant` selects the representative as
+ * in condense_group_v: the method or one of the two ablations. */
+int ora_lca_prefill_v(const uint16_t *cache, const uint16_t *qpre, const uint16_t *w_uv, int B,
+                      long L, long q_start, long q_len, int H, int dc, int dr, int dv, int g, int w,
+                      double scale, int variant, const int64_t *blocks, long n_blocks, double *o_lat,
+                      double *out, int32_t *anchor_out)
 {
     int D = dc + dr;
     if (q_start % g || q_len % g || q_start < 0 || q_start + q_len > L) return -1;
@@ -417,8 +418,8 @@ int ora_lca_prefill(const uint16_t *cache, const uint16_t *qpre, const uint16_t 
             double *rc = (double *)malloc(sizeof(double) * (m > 0 ? m : 1) * dc);
             double *rk = (double *)malloc(sizeof(double) * (m > 0 ? m : 1) * dr);
             for (long j = 0; j < m; j++) {
-                int I = condense_group(qbar, seq + (size_t)j * g * D, g, H, dc, dr, scale,
-                                       rc + (size_t)j * dc, rk + (size_t)j * dr, NULL, NULL);
+                int I = condense_group_v(qbar, seq + (size_t)j * g * D, g, H, dc, dr, scale, variant,
+                                         rc + (size_t)j * dc, rk + (size_t)j * dr, NULL, NULL);
                 if (anchor_out)
                     anchor_out[((size_t)b * nb_range + (k - q_start / g)) * (m_max > 0 ? m_max : 1) + j] =
                         (int32_t)(j * g + I);
@@ -440,6 +441,16 @@ int ora_lca_prefill(const uint16_t *cache, const uint16_t *qpre, const uint16_t 
             free(qbar);
         }
     return 0;
+}
+
+/* The method's prefill (variant ORA_LCA). */
+int ora_lca_prefill(const uint16_t *cache, const uint16_t *qpre, const uint16_t *w_uv, int B,
+                    long L, long q_start, long q_len, int H, int dc, int dr, int dv, int g, int w,
+                    double scale, const int64_t *blocks, long n_blocks, double *o_lat,
+                    double *out, int32_t *anchor_out)
+{
+    return ora_lca_prefill_v(cache, qpre, w_uv, B, L, q_start, q_len, H, dc, dr, dv, g, w, scale,
+                             ORA_LCA, blocks, n_blocks, o_lat, out, anchor_out);
 }
 
 /* Stored-representative decode: the reading of the page's "90% KV-cache

@@ -310,6 +310,64 @@ def test_prefill_block_subset_matches_full(ora):
     assert np.isnan(out2[:, 0]).all()
 
 
+def test_prefill_sparse_is_mla_over_anchor_rows(ora):
+    """"纯稀疏" prefill: every representative is its anchor token's own row, so
+    query t of block k is exact MLA attention over the cache rows
+    [anchors of groups 0 .. m_k - 1 || m_k g .. t].  The anchors are the
+    method's (the same argmax)."""
+    rng = np.random.default_rng(14)
+    g, w = 4, 8
+    cache, qpre, w_uv = prefill_case(rng)
+    qs, ql = 32, 40
+    ol, out, anc = ora.lca_prefill(cache, qpre, w_uv, qs, ql, g, w, 0.3, dr=4, want_anchor=True,
+                                   variant=ora.SPARSE)
+    _, _, anc_lca = ora.lca_prefill(cache, qpre, w_uv, qs, ql, g, w, 0.3, dr=4, want_anchor=True)
+    assert np.array_equal(anc, anc_lca)
+    for t in range(qs, qs + ql):
+        t0 = t - t % g
+        mb = max(0, (t0 - w) // g)
+        rows = np.concatenate([anc[0, (t0 - qs) // g, :mb], np.arange(mb * g, t + 1)])
+        ol2, o2 = ora.mla_decode(cache[:, rows], qpre[:, t], w_uv, 0.3, dr=4)
+        np.testing.assert_allclose(ol[:, t - qs], ol2, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(out[:, t - qs], o2, rtol=0, atol=1e-13)
+
+
+def test_prefill_pool_position_attends_pooled_keys(ora):
+    """"纯池化（含位置）" prefill, on a cache built so that the pooled rows are
+    known exactly.  The rows of each history group share everything but one
+    RoPE coordinate. The block's queries are identical, and their two heads'
+    dots cancel on that coordinate. So the group's importance scores are
+    equal, alpha = 1/g, and the representative is the group's mean row.
+    Attending stored bf16 representatives equal to those means must then
+    give the block's outputs.  The method (anchor key = the group's first
+    row, which is not the mean) gives something else."""
+    rng = np.random.default_rng(15)
+    g, w, dc, dr = 4, 8, 8, 4
+    cache, qpre, w_uv = prefill_case(rng)
+    t0 = 40
+    m = (t0 - w) // g
+    rows = from_bits(cache).copy()
+    for j in range(m):
+        rows[0, j * g:(j + 1) * g] = rows[0, j * g]
+        rows[0, j * g:(j + 1) * g, dc + 2] = rng.integers(-3, 4, size=g)
+    cache = bf16_bits(rows)
+    q = np.zeros((2, dc + dr))
+    q[0, dc + 2] = 1.0
+    q[1, 0], q[1, dc + 2] = 1.0, -1.0
+    qpre = qpre.copy()
+    qpre[0, t0:t0 + g] = bf16_bits(q)
+    pooled = from_bits(cache)[0, :m * g].reshape(m, g, dc + dr).mean(axis=1)
+    rep = bf16_bits(pooled)[None]
+    assert np.array_equal(from_bits(rep)[0], pooled)
+    ol, out, _ = ora.lca_prefill(cache, qpre, w_uv, t0, g, g, w, 0.3, dr=dr, variant=ora.POOL_POSITION)
+    ol_m, _, _ = ora.lca_prefill(cache, qpre, w_uv, t0, g, g, w, 0.3, dr=dr)
+    for t in range(t0, t0 + g - 1):
+        ol2, o2 = ora.lca_attend_reps(cache[:, :t + 1], rep, qpre[:, t], w_uv, g, w, 0.3, dr=dr)
+        np.testing.assert_allclose(ol[:, t - t0], ol2, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(out[:, t - t0], o2, rtol=0, atol=1e-13)
+        assert not np.allclose(ol_m[:, t - t0], ol2, rtol=0, atol=1e-6)
+
+
 # ----------------------------------------------------------------- stored representatives
 def stored_case(rng, B=2, L=61, H=3, dc=8, dr=4, dv=5, peak=3.0):
     cache = rand_bits(rng, (B, L, dc + dr))
