@@ -74,10 +74,11 @@ extern "C" {
  * own representative, which is exactly MLA).  w: local window (>= 0).
  * scale: logit scale (1/sqrt(192) for the 128+64 per-head MLA width).
  * variant: LCA_VARIANT_LCA (0) is the method; the other two are the
- * ablations of the page's 消融实验 table, accepted by lca_condense and
- * lca_condense_append only (other entry points that condense return
- * LCA_ERR_UNSUPPORTED for them; the attention over stored representatives
- * is the same for all three):
+ * ablations of the page's 消融实验 table, accepted by lca_condense,
+ * lca_condense_append and lca_prefill_block (the decode entry points that
+ * condense on the fly return LCA_ERR_UNSUPPORTED for them: decode an
+ * ablation with lca_condense + lca_decode_attn, since the attention over
+ * stored representatives is the same for all three):
  *   LCA_VARIANT_POOL_POSITION: the RoPE key is pooled with the same weights
  *     as the latent, k_rep = sum_i alpha_i k^R_i ("纯池化（含位置）");
  *   LCA_VARIANT_SPARSE: the representative is the most important token's row,
@@ -235,7 +236,8 @@ int lca_decode_stored_varlen(const void *cache, const void *rep, int64_t rep_cap
  *   anchor [B][q_len/g][m_last] int32 or NULL, m_last = m of the range's last
  *          block: absolute anchor positions of block k's groups j < m_k in
  *          row (k - q_start/g); the rest of each row is not written.
- * Representatives are rounded to bf16 like cache rows.  Requires g == 16,
+ * Representatives are rounded to bf16 like cache rows.  p.variant selects
+ * the method or one of its two ablations (see lca_params).  Requires g == 16,
  * L <= 2^27 and B * q_len / 16 < 2^31 (LCA_ERR_UNSUPPORTED otherwise).  ws: lca_workspace_bytes(LCA_OP_PREFILL, B, L, q_len, p) bytes
  * (enough for any q_start; the blocks are processed in chunks of 256 so the
  * workspace stays near 256 * m_last * 1152 bytes). */

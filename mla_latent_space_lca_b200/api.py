@@ -204,7 +204,7 @@ def lca_decode_varlen(cache, lens, q_recent, q, w_uv, g=16, w=1024, scale=None, 
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
     ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_varlen(_ptr(cache), _ptr(lens), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
-                                      _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
+                                      _params(g, w, scale, variant, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
                                       _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "lca_decode_varlen")
     return out
@@ -274,7 +274,7 @@ def lca_combine_shards(parts, w_uv, B, out=None, o_lat=None, stream=None):
 
 
 def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, out=None,
-                      o_lat=None, anchor=None, ws=None, stream=None):
+                      o_lat=None, anchor=None, ws=None, stream=None, variant=0):
     B, L, _ = cache.shape
     pitch = _cache(cache)
     _need(q, "q", torch.bfloat16, (B, L, H, D))
@@ -288,7 +288,7 @@ def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, 
         _need(anchor, "anchor", torch.int32)
     ws = workspace(_lib.OP_PREFILL, B, L, q_len, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_prefill_block(_ptr(cache), _ptr(q), _ptr(w_uv), B, L, q_start, q_len,
-                                      _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
+                                      _params(g, w, scale, variant, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
                                       _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "lca_prefill_block")
     return out

@@ -719,7 +719,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     int rc = check_common(cache, q, w_uv, B, L, out);
     if (rc) return rc;
     if (!params_ok(p) || !pitch_ok(p, B, L)) return LCA_ERR_INVALID_ARG;
-    if (p.g != 16 || p.variant != LCA_VARIANT_LCA) return LCA_ERR_UNSUPPORTED;
+    if (p.g != 16) return LCA_ERR_UNSUPPORTED;
     if (q_start < 0 || q_len < 0 || q_start % 16 || q_len % 16 || q_start + q_len > L) return LCA_ERR_INVALID_ARG;
     if (L > (int64_t(1) << 27)) return LCA_ERR_UNSUPPORTED;   // query rows 16 L index a TMA map
     if (int64_t(B) * (q_len / 16) >= (int64_t(1) << 31)) return LCA_ERR_UNSUPPORTED;   // block index of a TMA map
@@ -786,6 +786,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
                 c.k0 = k0;
                 c.m_ld = m_ld;
                 c.anchor = anchor ? anchor + size_t(b) * size_t(nb) * size_t(m_ld) : nullptr;
+                c.variant = p.variant;
                 const int n_bt = (nbc + 127) / 128;
                 Launch l(st, K_PREFILL_CONDENSE);
                 const cudaError_t e = launch_ex(condense_prefill_kernel, dim3(unsigned(n_bt * c.n_gt)),

@@ -96,6 +96,7 @@ struct CondPreArgs {
     int64_t k0;        // first block of the call (anchor rows)
     int64_t m_ld;      // anchor row length
     int32_t *anchor;   // this sequence's anchor rows [(k - k0)][m_ld], or NULL
+    int variant;       // LCA_VARIANT_*: the method or one of its ablations
 };
 
 __global__ void __launch_bounds__(CP_THREADS, 2)
@@ -195,16 +196,23 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
                 // rep_j[128 x 128c..] = alpha_j (A, K-major, K = 16 at column 16 jj of
                 // the alpha tile) * rows 16 jj.. of the tile (B, MN-major, N = 128
                 // spanning boxes 2c and 2c+1); one TMEM buffer, drained in turn
+                // (pooled-key ablation: a fifth N = 64 MMA pools the RoPE box)
                 constexpr uint32_t IDESC_P = idesc_bf16(128, 128, 0, 1);
+                constexpr uint32_t IDESC_PK = idesc_bf16(128, 64, 0, 1);
+                const int np = a.variant == LCA_VARIANT_POOL_POSITION ? 5 : 4;
                 ok = mbar_wait(aready, 0, abort_flag, K_PREFILL_CONDENSE, 5);
                 if (ok) tc_fence_after();
 #pragma unroll 1
-                for (int idx = 0; idx < 4 * CP_G && ok; ++idx) {
-                    const int jj = idx >> 2, cc = idx & 3;
+                for (int idx = 0; idx < np * CP_G && ok; ++idx) {
+                    const int jj = idx / np, cc = idx - jj * np;
                     if (!(ok = mbar_wait(pempty, (idx & 1) ^ 1, abort_flag, K_PREFILL_CONDENSE, 6))) break;
                     tc_fence_after();
-                    mma_ss(tmem + CP_TM_P, sdesc_sw128(abase + 32 * jj, 16, 1024),
-                           sdesc_sw128(rbase + 2 * cc * CP_BOX + 2048 * jj, CP_BOX, 1024), IDESC_P, 0u);
+                    if (cc < 4)
+                        mma_ss(tmem + CP_TM_P, sdesc_sw128(abase + 32 * jj, 16, 1024),
+                               sdesc_sw128(rbase + 2 * cc * CP_BOX + 2048 * jj, CP_BOX, 1024), IDESC_P, 0u);
+                    else
+                        mma_ss(tmem + CP_TM_P, sdesc_sw128(abase + 32 * jj, 16, 1024),
+                               sdesc_sw128(rbase + 8 * CP_BOX + 2048 * jj, CP_BOX, 1024), IDESC_PK, 0u);
                     tc_commit(pfull);
                 }
             }
@@ -252,13 +260,18 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
                     den += ex[e];
                 }
                 const float inv = 1.f / den;
+                // sparse ablation: weight 1 on the anchor (the pooling MMA then
+                // reproduces the anchor's latent exactly), 0 elsewhere
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    ex[e] = a.variant == LCA_VARIANT_SPARSE ? (e == gi ? 1.f : 0.f) : ex[e] * inv;
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
                     uint4 pk;
-                    pk.x = pack_bf16(ex[8 * c2 + 0] * inv, ex[8 * c2 + 1] * inv);
-                    pk.y = pack_bf16(ex[8 * c2 + 2] * inv, ex[8 * c2 + 3] * inv);
-                    pk.z = pack_bf16(ex[8 * c2 + 4] * inv, ex[8 * c2 + 5] * inv);
-                    pk.w = pack_bf16(ex[8 * c2 + 6] * inv, ex[8 * c2 + 7] * inv);
+                    pk.x = pack_bf16(ex[8 * c2 + 0], ex[8 * c2 + 1]);
+                    pk.y = pack_bf16(ex[8 * c2 + 2], ex[8 * c2 + 3]);
+                    pk.z = pack_bf16(ex[8 * c2 + 4], ex[8 * c2 + 5]);
+                    pk.w = pack_bf16(ex[8 * c2 + 6], ex[8 * c2 + 7]);
                     const int c = 2 * jj + c2;
                     *reinterpret_cast<uint4 *>(arow + ((c ^ (row & 7)) << 4)) = pk;
                 }
@@ -280,11 +293,18 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
         // representative (group j, chunk block kk) lives in row j nbc + kk
         auto rep_row = [&](int64_t j, int64_t kk) -> size_t { return size_t(j * a.nbc + kk); };
 
-        // anchor keys (bit copies from the tile) and anchor positions
+        // anchor keys (bit copies from the tile) and anchor positions; the
+        // pooled-key ablation writes its pooled keys with the latents below
+        const bool pool_key = a.variant == LCA_VARIANT_POOL_POSITION;
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(rfull, 0, abort_flag, K_PREFILL_CONDENSE, 9));
 #pragma unroll 1
         for (int jj = 0; jj < CP_G && ok; ++jj) {
             const int64_t j = int64_t(CP_G) * gt + jj;
+            if (pool_key) {
+                if (a.anchor && vblk && j < mk)
+                    a.anchor[size_t(k - a.k0) * size_t(a.m_ld) + size_t(j)] = int32_t(16 * j + anc[jj]);
+                continue;
+            }
             {
                 const int rr = 16 * jj + anc[jj];
                 const uint8_t *src = smem + 8 * CP_BOX + rr * 128;
@@ -309,12 +329,42 @@ __global__ void __launch_bounds__(CP_THREADS, 2)
         }
 
         // drain the pooled latents: group jj, d-chunk cc, one TMEM buffer
+        // (cc = 4: the pooled RoPE key of the pooled-key ablation)
+        const int np = pool_key ? 5 : 4;
 #pragma unroll 1
-        for (int idx = 0; idx < 4 * CP_G && ok; ++idx) {
-            const int jj = idx >> 2, cc = idx & 3;
+        for (int idx = 0; idx < np * CP_G && ok; ++idx) {
+            const int jj = idx / np, cc = idx - jj * np;
             ok = __all_sync(0xffffffffu, mbar_wait(pfull, idx & 1, abort_flag, K_PREFILL_CONDENSE, 10));
             if (!ok) break;
             tc_fence_after();
+            if (cc == 4) {
+#pragma unroll 1
+                for (int q2 = 0; q2 < 2; ++q2) {   // columns 32 q2 .. 32 q2 + 31
+                    float v[32];
+                    tmem_ld32(tmem + lane_base + CP_TM_P + 32 * q2, v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int c = 4 * q2 + e;   // 16-byte chunk of the 128-byte row
+                        *reinterpret_cast<uint4 *>(stg_rope + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_uint4(pack_bf16(v[8 * e], v[8 * e + 1]), pack_bf16(v[8 * e + 2], v[8 * e + 3]),
+                                       pack_bf16(v[8 * e + 4], v[8 * e + 5]), pack_bf16(v[8 * e + 6], v[8 * e + 7]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(pempty);
+                const int64_t j = int64_t(CP_G) * gt + jj;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const int rr = 4 * x + (lane >> 3), c = lane & 7;
+                    if (kk_warp + rr < a.nbc) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(stg_rope + rr * 128 + ((c ^ (rr & 7)) << 4));
+                        *reinterpret_cast<uint4 *>(a.rep + rep_row(j, kk_warp + rr) * LCA_D + LCA_DC + 8 * c) = v;
+                    }
+                }
+                __syncwarp();
+                continue;
+            }
 #pragma unroll 1
             for (int q4 = 0; q4 < 4; ++q4) {   // columns 32 q4 .. 32 q4 + 31
                 float v[32];

@@ -101,10 +101,12 @@ def test_other_entry_points_reject_bad_arguments(lcalib):
     assert lcalib.lca_condense_append(A, A, 1, 4096, p, 0, A, 100, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
     assert lcalib.lca_condense_append(A, A, 1, 4096, p, 193, A, 192, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
     assert lcalib.lca_decode_stored(A, A, 100, A, A, 1, 4096, p, A, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
-    # ablation variants: prefill and the no-alloc decode condense, so they refuse them
+    # ablation variants: the no-alloc decode condenses on the fly, so it
+    # refuses them (prefill accepts them); an unknown variant is refused
     pv = LcaParams(16, 1024, 0.07, _lib.VARIANT_SPARSE)
-    assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 0, 4096, pv, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
     assert lcalib.lca_decode_noalloc(A, A, A, A, 1, 4096, pv, A, None, None, None) == _lib.LCA_ERR_UNSUPPORTED
+    bad = LcaParams(16, 1024, 0.07, 3)
+    assert lcalib.lca_prefill_block(A, A, A, 1, 4096, 0, 4096, bad, A, None, None, A, big, None) == _lib.LCA_ERR_INVALID_ARG
     # prefill size limits: L beyond 2^27, and 2^31 blocks over the batch
     assert lcalib.lca_prefill_block(A, A, A, 1, (1 << 27) + 16, 0, 16, p, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED
     assert lcalib.lca_prefill_block(A, A, A, 1 << 8, 1 << 27, 0, 1 << 27, p, A, None, None, A, big, None) == _lib.LCA_ERR_UNSUPPORTED

@@ -32,28 +32,29 @@ def _device():
     assert rc == 0, f"device status {rc} detail {detail:#x}"
 
 
-def run_gpu(inp, q_start, q_len, w):
+def run_gpu(inp, q_start, q_len, w, variant=oracle.LCA):
     cache, q, w_uv = inp.cache.cuda(), inp.q.cuda(), inp.w_uv.cuda()
     B = inp.B
     m_last = oracle.num_groups(q_start + q_len - G, G, w)
     anchor = torch.full((B, q_len // G, max(m_last, 1)), -1, dtype=torch.int32, device="cuda")
     o_lat = torch.empty(B, q_len, 16, 512, dtype=torch.float32, device="cuda")
-    out = api.lca_prefill_block(cache, q, w_uv, q_start, q_len, w=w, o_lat=o_lat, anchor=anchor)
+    out = api.lca_prefill_block(cache, q, w_uv, q_start, q_len, w=w, o_lat=o_lat, anchor=anchor,
+                                variant=variant)
     torch.cuda.synchronize()
     return out, o_lat, anchor
 
 
-def check_prefill(inp, q_start, q_len, w, blocks=None, gpu=None):
+def check_prefill(inp, q_start, q_len, w, blocks=None, gpu=None, variant=oracle.LCA):
     """Compare the GPU prefill of [q_start, q_start+q_len) with the oracle on
     `blocks` (absolute block indices; None = all)."""
-    out, o_lat, anchor = gpu if gpu is not None else run_gpu(inp, q_start, q_len, w)
+    out, o_lat, anchor = gpu if gpu is not None else run_gpu(inp, q_start, q_len, w, variant)
     k0 = q_start // G
     if blocks is None:
         blocks = list(range(k0, k0 + q_len // G))
     blocks = sorted(set(int(k) for k in blocks))
     cache_b, q_b = bf16_bits(inp.cache), bf16_bits(inp.q)
     ol_ref, out_ref, anc_ref = oracle.lca_prefill(cache_b, q_b, bf16_bits(inp.w_uv), q_start, q_len, G, w,
-                                                  inp.scale, blocks=blocks, want_anchor=True)
+                                                  inp.scale, blocks=blocks, want_anchor=True, variant=variant)
     rows = np.concatenate([np.arange((k - k0) * G, (k - k0 + 1) * G) for k in blocks])
     rows_t = torch.as_tensor(rows, device="cuda")
     compare(out.index_select(1, rows_t).cpu().numpy(), out_ref[:, rows], "prefill out")
@@ -111,6 +112,17 @@ def test_prefill_peaked_anchors():
     B, L, w = 2, 16 * 160, 512
     inp = make_prefill_inputs(B, L, w=w, seed=43, peak=30.0)
     check_prefill(inp, 0, L, w, blocks=[31, 32, 33, 64, 100, 127, 128, 158, 159])
+
+
+@pytest.mark.parametrize("variant", [oracle.POOL_POSITION, oracle.SPARSE])
+def test_prefill_ablations(variant):
+    """The two ablations of the page's ablation table: the RoPE key pooled
+    with the latent's weights, or the anchor token's whole row.  Peaked
+    queries make the weights far from uniform; the blocks span two condense
+    block tiles, several representative tiles and the window edge."""
+    B, L, w = 2, 16 * 300, 256
+    inp = make_prefill_inputs(B, L, w=w, seed=44, peak=30.0)
+    check_prefill(inp, 0, L, w, blocks=[0, 15, 16, 17, 60, 127, 128, 129, 255, 256, 299], variant=variant)
 
 
 def test_prefill_range_split_consistency():
