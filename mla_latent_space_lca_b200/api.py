@@ -204,7 +204,7 @@ def lca_decode_varlen(cache, lens, q_recent, q, w_uv, g=16, w=1024, scale=None, 
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
     ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_varlen(_ptr(cache), _ptr(lens), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
-                                      _params(g, w, scale, variant, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
+                                      _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
                                       _ptr(ws), ws.numel(), _stream(stream))
     check(rc, "lca_decode_varlen")
     return out

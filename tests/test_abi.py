@@ -188,3 +188,33 @@ def test_valid_call_without_gpu_reports_no_device(lcalib):
     if torch.cuda.is_available():
         pytest.skip("a GPU is present")
     assert call_decode(lcalib) == _lib.LCA_ERR_NO_DEVICE
+
+
+def test_binding_functions_reference_only_defined_globals():
+    """Every global name the Python binding's functions load exists (the
+    binding cannot reach a GPU here, so a misspelt or missing name would
+    otherwise only show on a device)."""
+    import builtins
+    import dis
+    import types
+
+    from mla_latent_space_lca_b200 import api, split_blocks, split_l
+
+    def code_objects(co):
+        yield co
+        for c in co.co_consts:
+            if isinstance(c, types.CodeType):
+                yield from code_objects(c)
+
+    missing = []
+    for mod in (api, _lib, split_l, split_blocks):
+        for name, fn in vars(mod).items():
+            if not isinstance(fn, types.FunctionType) or fn.__module__ != mod.__name__:
+                continue
+            for co in code_objects(fn.__code__):
+                for ins in dis.get_instructions(co):
+                    if ins.opname == "LOAD_GLOBAL":
+                        g = ins.argval
+                        if g not in vars(mod) and not hasattr(builtins, g):
+                            missing.append(f"{mod.__name__}.{name}: {g}")
+    assert not missing, missing
