@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stored", action="store_true",
                     help="decode: stored-representative mode (groups condensed once and kept)")
-    ap.add_argument("--unfused-compare", type=int, default=0,
+    ap.add_argument("--unfused-compare", type=int, default=100,
                     help="decode: also time N steps of the unfused path (condense, then attend stored reps)")
     ap.add_argument("--varlen", action="store_true",
                     help="decode: a ragged batch, lengths drawn uniformly from [L/8, 15L/8] (mean L)")
@@ -400,15 +400,27 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(3):
             unfused_step()
         torch.cuda.synchronize()
-        u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        u0.record(stream)
-        for _ in range(args.unfused_compare):
-            unfused_step()
-        u1.record(stream)
+        # timed like the main loop: back to back, or one by one after an L2
+        # flush when the cache would otherwise stay in L2
+        uev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.unfused_compare if flush is not None else 1)]
+        if flush is None:
+            uev[0][0].record(stream)
+            for _ in range(args.unfused_compare):
+                unfused_step()
+            uev[0][1].record(stream)
+        else:
+            for a_, b_ in uev:
+                flush.zero_()
+                a_.record(stream)
+                unfused_step()
+                b_.record(stream)
         torch.cuda.synchronize()
-        unfused_ms = max_over_ranks(u0.elapsed_time(u1) / args.unfused_compare, world, dev)
+        unfused_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in uev) / args.unfused_compare, world, dev)
         lca.profile_enable(True)
         for _ in range(min(args.unfused_compare, 200)):
+            if flush is not None:
+                flush.zero_()
             unfused_step()
         torch.cuda.synchronize()
         uprof = lca.profile_collect()
