@@ -42,6 +42,8 @@ ROW_BYTES = 576 * 2
 METRIC = "LCA decode tokens/s and cache-read GB/s (fraction of B200 HBM roofline)"
 PREFILL_METRIC = "LCA blockwise prefill tokens/s (fraction of B200 bf16 tensor roofline)"
 PROFILE_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+# lca_params.variant: the method and the two ablations of the page's ablation table
+VARIANTS = {"lca": 0, "pool_position": 1, "sparse": 2}
 
 
 def parse():
@@ -66,6 +68,9 @@ def parse():
                     help="decode: every sequence's cache split along L over the ranks (strong scaling)")
     ap.add_argument("--split-blocks", action="store_true",
                     help="prefill: one prompt's query blocks split over the ranks by work (strong scaling)")
+    ap.add_argument("--variant", choices=list(VARIANTS), default="lca",
+                    help="the method, or one of the page's two ablations: decode runs lca_condense "
+                         "+ lca_decode_attn (the fused kernel has only the method), prefill passes it on")
     ap.add_argument("--mla-compare", type=int, default=0,
                     help="decode: also time N plain MLA decode steps (g = 1, every row attended) on the "
                          "same inputs; prefill: N full causal MLA prefills (w = L)")
@@ -100,7 +105,7 @@ def prefill_flops(L: int, w: int, k0: int = 0, k1: int | None = None, g: int = 1
     return {"attention": att, "condense": cond, "wuv": wuv}
 
 
-def prefill_cpu_baseline(inp, n_blocks: int, steps: int = 1, warmup: int = 0):
+def prefill_cpu_baseline(inp, n_blocks: int, steps: int = 1, warmup: int = 0, variant: int = 0):
     """The oracle on `n_blocks` evenly spaced blocks of the prefill (their
     average cost matches the whole range's); tokens/s extrapolated."""
     import oracle
@@ -111,11 +116,13 @@ def prefill_cpu_baseline(inp, n_blocks: int, steps: int = 1, warmup: int = 0):
                         [i * (nb - 1) / max(1, n_blocks - 1) for i in range(n_blocks)]))
     c, q, w = bf16_bits(inp.cache), bf16_bits(inp.q), bf16_bits(inp.w_uv)
     for _ in range(warmup):
-        oracle.lca_prefill(c, q, w, 0, inp.L, 16, inp.w, inp.scale, blocks=blocks, want_olat=False)
+        oracle.lca_prefill(c, q, w, 0, inp.L, 16, inp.w, inp.scale, blocks=blocks, want_olat=False,
+                           variant=variant)
     times = []
     for _ in range(max(1, steps)):
         t0 = time.perf_counter()
-        oracle.lca_prefill(c, q, w, 0, inp.L, 16, inp.w, inp.scale, blocks=blocks, want_olat=False)
+        oracle.lca_prefill(c, q, w, 0, inp.L, 16, inp.w, inp.scale, blocks=blocks, want_olat=False,
+                           variant=variant)
         times.append(time.perf_counter() - t0)
     tok_s = 16 * len(blocks) * inp.B / statistics.mean(times)
     sample = (f"{len(blocks)} evenly spaced blocks of {nb} (16 queries each) per oracle call, "
@@ -223,12 +230,23 @@ def ncu_traffic(workload):
 REF_BUDGET_S = 150.0   # whole reference-arm run (all K + W steps), seconds
 
 
-def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0, seqs: int = 0):
+def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0, seqs: int = 0, variant: int = 0):
     """The oracle as it stands, on host cores, over a bounded sample of the
-    workload (whole sequences; `seqs` per call, else ~2 s worth).  Returns
-    (tokens/s, cores, sample text, per-step seconds)."""
+    workload (whole sequences; `seqs` per call, else ~2 s worth).  An
+    ablation runs the oracle's condensation with it, rounds the
+    representatives to bf16 as the GPU stores them, and attends them.
+    Returns (tokens/s, cores, sample text, per-step seconds)."""
+    import numpy as np
+
     import oracle
     from mla_latent_space_lca_b200.inputs import bf16_bits
+
+    def decode(c, qr, q, w):
+        if not variant:
+            return oracle.lca_decode(c, qr, q, w, inp.g, inp.w, inp.scale)
+        r = oracle.lca_condense(c, qr, inp.g, inp.w, inp.scale, variant=variant)
+        rep = bf16_bits(torch.from_numpy(np.concatenate([r["rep_c"], r["rep_k"]], axis=2)).to(torch.bfloat16))
+        return oracle.lca_attend_reps(c, rep, q, w, inp.g, inp.w, inp.scale)
 
     B = inp.cache.shape[0]
     # sample size: sequences whose oracle decode takes ~1-3 s
@@ -241,13 +259,13 @@ def cpu_baseline(inp, budget_s: float, steps: int = 0, warmup: int = 0, seqs: in
     q = bf16_bits(inp.q[:S])
     w = bf16_bits(inp.w_uv)
     for _ in range(warmup):
-        oracle.lca_decode(c, qr, q, w, inp.g, inp.w, inp.scale)
+        decode(c, qr, q, w)
     times = []
     t_start = time.time()
     n = 0
     while True:
         t0 = time.perf_counter()
-        oracle.lca_decode(c, qr, q, w, inp.g, inp.w, inp.scale)
+        decode(c, qr, q, w)
         times.append(time.perf_counter() - t0)
         n += 1
         if (steps and n >= steps) or (not steps and time.time() - t_start >= budget_s):
@@ -283,17 +301,20 @@ def run_reference(args, rank, world):
         inp = make_prefill_inputs(wl["B"], wl["L"], seed=0)
         # blocks per step so that all K + W steps fit REF_BUDGET_S
         n0 = oracle.num_threads()
-        _, _, _, t0 = prefill_cpu_baseline(inp, n0, steps=1)
+        v = VARIANTS[args.variant]
+        _, _, _, t0 = prefill_cpu_baseline(inp, n0, steps=1, variant=v)
         per_step = REF_BUDGET_S / max(1, args.steps + args.warmup)
         n = max(1, min(2 * n0, int(n0 * per_step / max(t0[0], 1e-6))))
-        tok_s, cores, sample, times = prefill_cpu_baseline(inp, n, steps=args.steps, warmup=args.warmup)
+        tok_s, cores, sample, times = prefill_cpu_baseline(inp, n, steps=args.steps, warmup=args.warmup,
+                                                           variant=v)
         ms = 1e3 * statistics.mean(times)
         line = {
             "impl": "reference", "metric": PREFILL_METRIC, "value": tok_s, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": args.workload, "B": wl["B"], "L": wl["L"], "g": 16, "w": 1024},
+            "config": {"workload": args.workload, "B": wl["B"], "L": wl["L"], "g": 16, "w": 1024,
+                       "variant": args.variant},
             "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -304,17 +325,20 @@ def run_reference(args, rank, world):
     inp = make_decode_inputs(wl["B"], wl["L"], seed=0)
     # size each step's sample so that all K + W steps fit REF_BUDGET_S: time
     # one single-sequence call first
-    _, _, _, t1 = cpu_baseline(inp, 0, steps=1, warmup=0, seqs=1)
+    v = VARIANTS[args.variant]
+    _, _, _, t1 = cpu_baseline(inp, 0, steps=1, warmup=0, seqs=1, variant=v)
     per_step = REF_BUDGET_S / max(1, args.steps + args.warmup)
     seqs = max(1, min(wl["B"], int(per_step / max(t1[0], 1e-6))))
-    tok_s, cores, sample, times = cpu_baseline(inp, 0, steps=args.steps, warmup=args.warmup, seqs=seqs)
+    tok_s, cores, sample, times = cpu_baseline(inp, 0, steps=args.steps, warmup=args.warmup, seqs=seqs,
+                                               variant=v)
     ms = 1e3 * statistics.mean(times)
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": args.workload, "B": wl["B"], "L": wl["L"], "g": 16, "w": 1024},
+        "config": {"workload": args.workload, "B": wl["B"], "L": wl["L"], "g": 16, "w": 1024,
+                   "variant": args.variant},
         "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -339,9 +363,20 @@ def run_ours(args, rank, world, local_rank):
     ws = lca.workspace(3, B, L, device=dev)
     out = torch.empty(B, 16, 128, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    variant = VARIANTS[args.variant]
+    rep_v = (torch.empty(B, max(1, lca.num_groups(L)), 576, dtype=torch.bfloat16, device=dev)
+             if variant else None)
+
+    def decode(q_rec, q_now):
+        if variant:
+            # an ablation: condense with it, then attend the representatives
+            lca.lca_condense(cache, q_rec, scale=inp.scale, rep=rep_v, ws=ws, stream=stream, variant=variant)
+            lca.lca_decode_attn(cache, rep_v, q_now, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+        else:
+            lca.lca_decode(cache, q_rec, q_now, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
 
     def step():
-        lca.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+        decode(q_recent, q)
 
     def barrier():
         if world > 1:
@@ -390,7 +425,7 @@ def run_ours(args, rank, world, local_rank):
     # in-run comparison: the unfused path (condense to stored representatives,
     # then attention over them), which writes and re-reads the representatives
     unfused_ms = condense_ms = None
-    if args.unfused_compare and lca.num_groups(L) > 0:
+    if args.unfused_compare and lca.num_groups(L) > 0 and not variant:
         rep_u = torch.empty(B, lca.num_groups(L), 576, dtype=torch.bfloat16, device=dev)
 
         def unfused_step():
@@ -432,7 +467,7 @@ def run_ours(args, rank, world, local_rank):
     # in-run comparison: plain MLA decode (g = 1) over the whole cache, the
     # same inputs, timed the same way
     mla = None
-    if args.mla_compare:
+    if args.mla_compare and not variant:
         def mla_step():
             lca.mla_decode_attn(cache, q, w_uv, inp.scale, out=out, ws=ws, stream=stream)
 
@@ -492,7 +527,7 @@ def run_ours(args, rank, world, local_rank):
         dq.copy_(pin_q, non_blocking=True)
         ring[:, slot[0]].copy_(dq)
         slot[0] = (slot[0] + 1) % ring.shape[1]
-        lca.lca_decode(cache, ring, dq, w_uv, scale=inp.scale, out=out, ws=ws)
+        decode(ring, dq)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -514,7 +549,7 @@ def run_ours(args, rank, world, local_rank):
     # for reference: the same step with the whole cache and all recent
     # queries copied in from the host
     full_ms = None
-    if args.e2e_full_copy:
+    if args.e2e_full_copy and not variant:
         pin_cache = inp.cache.pin_memory()
         pin = [t.pin_memory() for t in (inp.q_recent, inp.q)]
         dbuf = [torch.empty_like(t, device=dev) for t in pin]
@@ -541,11 +576,20 @@ def run_ours(args, rank, world, local_rank):
     value = tokens / (ms / 1e3)
     gbs = B * L * ROW_BYTES * world / (ms / 1e3) / 1e9
     peak, peak_kind = measured_hbm_peak()
-    attn = prof.get("attn_decode")
+    if variant:
+        # the ablation's step is dominated by the condensation: 16 m history
+        # rows read and m representatives written per sequence
+        attn = prof.get("condense")
+        algo_bytes = B * 17 * lca.num_groups(L) * ROW_BYTES
+        traffic = None
+        rl_kernel = f"condense ({args.variant})"
+    else:
+        attn = prof.get("attn_decode")
+        algo_bytes = B * L * ROW_BYTES
+        traffic = ncu_traffic(args.workload)
+        rl_kernel = "attn_decode (fused LCA)"
     attn_ms = attn[1] / attn[0] if attn else None
-    algo_bytes = B * L * ROW_BYTES
     achieved = algo_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
-    traffic = ncu_traffic(args.workload)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -553,11 +597,12 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": args.workload, "B_per_gpu": B, "L": L, "g": 16, "w": 1024,
                    "heads": 16, "d_c": 512, "d_r": 64, "parallelism": f"replicas x{world}",
+                   "variant": args.variant,
                    "l2": ("inputs (B*L*1152 B) larger than the 126 MB L2; no flush" if flush is None else
                           "flushed (256 MB write) before every step; steps timed one by one")},
         "cache_gbps": gbs, "cache_frac_of_hbm": gbs / world / peak,
         "cache_frac_of_nominal_8tbs": gbs / world / 8000.0,
-        "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA)",
+        "roofline": {"bound": "hbm", "kernel": rl_kernel,
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak if achieved else None, "traffic": traffic,
                      "algorithmic_bytes_per_launch": algo_bytes,
@@ -567,7 +612,8 @@ def run_ours(args, rank, world, local_rank):
         "clocks": sampler.summary() if sampler else None,
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "note": "lca_decode in a decode loop: cache and recent-query ring resident on the device; "
+                "note": ("lca_decode" if not variant else "lca_condense + lca_decode_attn") +
+                        " in a decode loop: cache and recent-query ring resident on the device; "
                         "per step the new token's row and query in from pinned host memory, out back"},
     }
     if full_ms is not None:
@@ -600,7 +646,7 @@ def run_ours(args, rank, world, local_rank):
                 "achieved_gbs": cbytes / (condense_ms / 1e3) / 1e9,
                 "frac_of_measured_hbm": cbytes / (condense_ms / 1e3) / 1e9 / peak}
     if world == 1 and not args.no_cpu_baseline:
-        tok_s, cores, sample, _ = cpu_baseline(inp, args.cpu_seconds)
+        tok_s, cores, sample, _ = cpu_baseline(inp, args.cpu_seconds, variant=variant)
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample}
     print(json.dumps(line), flush=True)
@@ -1069,8 +1115,11 @@ def run_ours_prefill(args, rank, world, local_rank):
     out = torch.empty(B, ql, 16, 128, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    variant = VARIANTS[args.variant]
+
     def step():
-        lca.lca_prefill_block(cache, q, w_uv, qs, ql, scale=inp.scale, out=out, ws=ws, stream=stream)
+        lca.lca_prefill_block(cache, q, w_uv, qs, ql, scale=inp.scale, out=out, ws=ws, stream=stream,
+                              variant=variant)
 
     def barrier():
         if world > 1:
@@ -1120,7 +1169,7 @@ def run_ours_prefill(args, rank, world, local_rank):
     def e2e_step():
         dcache[:, :qs + ql].copy_(pin[0], non_blocking=True)
         dq[:, qs:qs + ql].copy_(pin[1], non_blocking=True)
-        lca.lca_prefill_block(dcache, dq, w_uv, qs, ql, scale=inp.scale, out=out, ws=ws)
+        lca.lca_prefill_block(dcache, dq, w_uv, qs, ql, scale=inp.scale, out=out, ws=ws, variant=variant)
         h_out.copy_(out, non_blocking=True)
 
     e2e_step()
@@ -1174,7 +1223,8 @@ def run_ours_prefill(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "strong" if split else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": args.workload, "B_per_gpu": B, "L": L, "q_len": L, "g": 16, "w": 1024,
+        "config": {"workload": args.workload, "variant": args.variant, "B_per_gpu": B, "L": L, "q_len": L,
+                   "g": 16, "w": 1024,
                    "heads": 16, "d_c": 512, "d_r": 64,
                    "parallelism": f"split-blocks x{world}" if split else f"replicas x{world}",
                    "rank0_queries": [qs, qs + ql],
@@ -1197,7 +1247,7 @@ def run_ours_prefill(args, rank, world, local_rank):
                                "step_tflops": B * sum(mla_fl.values()) / (mla_ms / 1e3) / 1e12}
     if world == 1 and not args.no_cpu_baseline:
         import oracle
-        tok_s, cores, sample, _ = prefill_cpu_baseline(inp, 2 * oracle.num_threads())
+        tok_s, cores, sample, _ = prefill_cpu_baseline(inp, 2 * oracle.num_threads(), variant=variant)
         line["cpu_baseline"] = {"value": tok_s, "unit": "tokens/s", "cores": cores,
                                 "kind": "oracle", "sample": sample}
     print(json.dumps(line), flush=True)
@@ -1213,6 +1263,8 @@ def main():
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.variant != "lca" and (args.stored or args.varlen or args.split_l):
+        raise SystemExit("--variant applies to the plain decode and prefill workloads only")
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
