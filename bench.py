@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--e2e-full-copy", type=int, default=2,
                     help="decode: also time N steps that copy the whole cache in from the host")
+    ap.add_argument("--no-e2e-graph", action="store_true",
+                    help="decode: skip the end-to-end loop replayed from CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--stored", action="store_true",
@@ -367,13 +369,13 @@ def run_ours(args, rank, world, local_rank):
     rep_v = (torch.empty(B, max(1, lca.num_groups(L)), 576, dtype=torch.bfloat16, device=dev)
              if variant else None)
 
-    def decode(q_rec, q_now):
+    def decode(q_rec, q_now, st=stream):   # st None: the current stream (a graph capture's)
         if variant:
             # an ablation: condense with it, then attend the representatives
-            lca.lca_condense(cache, q_rec, scale=inp.scale, rep=rep_v, ws=ws, stream=stream, variant=variant)
-            lca.lca_decode_attn(cache, rep_v, q_now, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+            lca.lca_condense(cache, q_rec, scale=inp.scale, rep=rep_v, ws=ws, stream=st, variant=variant)
+            lca.lca_decode_attn(cache, rep_v, q_now, w_uv, scale=inp.scale, out=out, ws=ws, stream=st)
         else:
-            lca.lca_decode(cache, q_rec, q_now, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
+            lca.lca_decode(cache, q_rec, q_now, w_uv, scale=inp.scale, out=out, ws=ws, stream=st)
 
     def step():
         decode(q_recent, q)
@@ -546,6 +548,40 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in xev) / n_e2e, world, dev)
     assert torch.equal(h_out, out.cpu())
 
+    # the same loop with each step captured once in a CUDA graph (one graph
+    # per ring slot: the slot a step writes is part of the step) and replayed:
+    # the copies and launches of a step go to the GPU in one call
+    graph_ms = None
+    if not args.no_e2e_graph:
+        def graph_step(sl):
+            cache[:, L - 1].copy_(pin_row, non_blocking=True)
+            dq.copy_(pin_q, non_blocking=True)
+            ring[:, sl].copy_(dq)
+            decode(ring, dq, st=None)
+            h_out.copy_(out, non_blocking=True)
+
+        graphs = []
+        for sl in range(ring.shape[1]):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                graph_step(sl)
+            graphs.append(gph)
+        for i in range(3):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+        barrier()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+        for i, (a_, b_) in enumerate(gev):
+            if flush is not None:
+                flush.zero_()
+            a_.record(stream)
+            graphs[i % len(graphs)].replay()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in gev) / n_e2e, world, dev)
+        assert torch.equal(h_out, out.cpu())
+        del graphs
+
     # for reference: the same step with the whole cache and all recent
     # queries copied in from the host
     full_ms = None
@@ -616,6 +652,12 @@ def run_ours(args, rank, world, local_rank):
                         " in a decode loop: cache and recent-query ring resident on the device; "
                         "per step the new token's row and query in from pinned host memory, out back"},
     }
+    if graph_ms is not None:
+        line["e2e_graph"] = {
+            "value": tokens / (graph_ms / 1e3), "unit": "tokens/s", "ms_per_step": graph_ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "the e2e loop with each step (copies in, decode, copy out) captured once as a CUDA "
+                    "graph through the same public calls and replayed"}
     if full_ms is not None:
         line["e2e_full_cache_copy"] = {
             "value": tokens / (full_ms / 1e3), "unit": "tokens/s", "ms_per_step": full_ms,
