@@ -2,12 +2,13 @@
 // representatives to memory in cache-row format.
 //
 // One warp condenses one group of 16 tokens at a time.  The group is one
-// contiguous 18 KB span of the cache ([16 rows x 1152 B]); each warp keeps a
-// 3-slot ring of such spans in shared memory, filled by cp.async.bulk with an
-// L2 evict-first hint, so the cache streams through once with ~54 KB per warp
-// in flight.  Per group, from shared memory:
-//   s_i   = u . row_i           (u = folded summary query, fp32 FMA; lanes
-//                                own 16-byte column slices, a halving
+// contiguous 18 KB span of the cache ([16 rows x 1152 B]), copied into the
+// warp's own shared-memory slot by cp.async.bulk with an L2 evict-first hint;
+// twelve warps per CTA (three per scheduler) keep ~216 KB per SM in flight
+// while the cache streams through once.  Per group, from shared memory:
+//   s_i   = u . row_i           (u = folded summary query, fp32 FMA, held in
+//                                registers; lanes own 16-byte column slices,
+//                                36 of the 16 x 72 per lane, and a halving
 //                                shuffle transpose sums the 16 dots so that
 //                                lanes 2t, 2t+1 end up with token t)
 //   alpha = softmax(s)          (shuffle max / sum over the 16 tokens)
