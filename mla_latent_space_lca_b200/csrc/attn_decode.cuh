@@ -96,6 +96,10 @@ struct AttnArgs {
     const int32_t *tile_start;
     int B;
     int w;
+    // 1: launched right after prep_summary_kernel, which lets this grid
+    // launch only once everything before it in the stream has completed, so
+    // the cache may be read without waiting for the summary query
+    int after_prep;
 };
 
 // Geometry of one sequence of L rows: its groups m, first window row and
@@ -323,8 +327,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             prefetch_tensormap(&map_cache);
             if (MODE == MODE_REPS && a.m > 0) prefetch_tensormap(&map_rep);
             // rows may come from a kernel earlier in the stream: read them only
-            // once the preceding grid (and so everything before it) is complete
-            griddep_wait();
+            // once the preceding grid (and so everything before it) is
+            // complete -- already the case when that grid is the summary-query
+            // fold, which triggers this launch after its own wait
+            if (!a.after_prep) griddep_wait();
             const uint64_t pol = policy_evict_first();
             int last[3] = {-1, -1, -1};
             int i = 0;

@@ -98,8 +98,10 @@ __global__ void __launch_bounds__(W * 32, 1) condense_kernel(const CondenseArgs 
         bulk_load(smem_u32(ring + s * CD_GROUP_BYTES), src, CD_GROUP_BYTES, bar, pol);
     };
 
-    // the cache rows and u may come from the previous kernel in the stream
-    griddep_wait();
+    // The library launches this kernel right after the summary-query fold,
+    // which lets it launch only once everything before that fold in the
+    // stream has completed: the cache rows are final, so the first copies go
+    // out at once; u (the fold's output) is read only after the wait below.
     if (lane == 0) {
 #pragma unroll
         for (int s = 0; s < S; ++s) {
@@ -107,6 +109,7 @@ __global__ void __launch_bounds__(W * 32, 1) condense_kernel(const CondenseArgs 
             if (gi < a.total) issue(gi, s);
         }
     }
+    griddep_wait();
 
     // this lane's 16-byte column slices of u: lane, lane + 32 (for all 16
     // rows) and 64 + lane % 8 (for rows 4 (lane / 8) .. + 3), so that the

@@ -319,6 +319,7 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     a.tile_start = VARLEN ? w.tile_start : nullptr;
     a.B = B;
     a.w = window;
+    a.after_prep = (!VARLEN && MODE == MODE_LCA && m > 0) ? 1 : 0;
 
     CUtensorMap map_cache, map_rep;
     rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,

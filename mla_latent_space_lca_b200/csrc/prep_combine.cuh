@@ -20,13 +20,14 @@ namespace lca {
 // g = 16), reduced by shuffles within a warp and through 2 KB of shared
 // memory across the 8 warps.
 //
-// Ordering: the kernel lets its dependent (the attention kernel) launch at
-// once, then waits for its own predecessor in the stream (whose output may
-// be q_recent) before reading.  The attention kernel reads nothing before
-// it has waited for this grid to complete, which covers that predecessor
-// too; meanwhile its launch and prologue overlap the predecessor's tail.
-// Every CTA of this grid is resident before the dependent can launch (each
-// triggers first thing), so the dependent never starves it of an SM.
+// Ordering: every CTA first waits for its predecessor in the stream (whose
+// output may be q_recent, or the cache row of the current token) and only
+// then lets its dependent (the attention or condense kernel) launch.  So the
+// dependent launches only once everything earlier in the stream has
+// completed: it may stream the cache at once, overlapping this kernel, and
+// waits for this grid to complete only before it reads u.  The dependent
+// cannot launch before every CTA of this grid has triggered, so it never
+// starves this grid of an SM.
 constexpr int PREP_THREADS = 256;
 
 __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16_t *__restrict__ q_recent,
@@ -35,8 +36,8 @@ __global__ void __launch_bounds__(PREP_THREADS) prep_summary_kernel(const uint16
                                                                     uint16_t *__restrict__ uhl)
 {
     __shared__ float part[8][64];
-    griddep_launch_dependents();
     griddep_wait();
+    griddep_launch_dependents();
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cg = threadIdx.x & 7, sl = threadIdx.x >> 3;   // 32 slices
