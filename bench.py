@@ -563,7 +563,9 @@ def run_ours(args, rank, world, local_rank):
         graphs = []
         for sl in range(ring.shape[1]):
             gph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gph):
+            # thread-local capture: other host threads (a process group's
+            # watchdog) may keep making CUDA calls meanwhile
+            with torch.cuda.graph(gph, capture_error_mode="thread_local"):
                 graph_step(sl)
             graphs.append(gph)
         for i in range(3):
