@@ -30,7 +30,11 @@
  *    `const void*` holding IEEE bfloat16 values, row-major and contiguous.
  *  - Every bf16 / fp32 tensor pointer must be 16-byte aligned.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
- *    asynchronous on it and never synchronise the host.
+ *    asynchronous on it and never synchronise the host.  The kernels of a
+ *    call are chained with programmatic dependent launch, but none reads an
+ *    input before all earlier work in the stream has completed: writes
+ *    issued on the stream before the call (copies, or the caller's kernels,
+ *    programmatic-launch ones included) are seen by it.
  *  - Return 0 (LCA_OK) or a negative lca_status.  Invalid arguments are
  *    rejected before anything is launched.  A launch failure returns
  *    LCA_ERR_CUDA with nothing further enqueued.
