@@ -125,6 +125,15 @@ def test_prefill_ablations(variant):
     check_prefill(inp, 0, L, w, blocks=[0, 15, 16, 17, 60, 127, 128, 129, 255, 256, 299], variant=variant)
 
 
+@pytest.mark.parametrize("variant", [oracle.POOL_POSITION, oracle.SPARSE])
+def test_prefill_ablations_ragged_window_mid_range(variant):
+    """The ablations with a window that is not a multiple of 16, a range
+    that starts mid-sequence and a cache longer than the range."""
+    B, L, w = 1, 16 * 90 + 5, 100
+    inp = make_prefill_inputs(B, L, w=w, seed=45, peak=30.0)
+    check_prefill(inp, 16 * 20, 16 * 70, w, variant=variant)
+
+
 def test_prefill_range_split_consistency():
     """Two calls over adjacent ranges give the rows of one call over both."""
     B, L, w = 1, 16 * 96, 256
