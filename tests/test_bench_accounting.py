@@ -79,3 +79,16 @@ def test_decode_workloads(bench):
         assert wl["B"] * wl["L"] * bench.ROW_BYTES == 1207959552
     assert bench.ROW_BYTES == 1152
     assert set(bench.VARIANTS) == {"lca", "pool_position", "sparse"}
+
+
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_cpu_baseline_runs_each_variant(bench, variant):
+    """The oracle baselines the benchmark times (its reference arm too) run
+    for the method and both ablations, on a tiny decode and prefill."""
+    from mla_latent_space_lca_b200.inputs import make_decode_inputs, make_prefill_inputs
+    inp = make_decode_inputs(2, 1100, seed=3)
+    tok_s, cores, sample, times = bench.cpu_baseline(inp, 0, steps=1, seqs=2, variant=variant)
+    assert tok_s > 0 and cores >= 1 and len(times) == 1 and "2 of 2 sequences" in sample
+    pre = make_prefill_inputs(1, 1024, w=128, seed=4)
+    tok_s, _, sample, times = bench.prefill_cpu_baseline(pre, 4, steps=1, variant=variant)
+    assert tok_s > 0 and len(times) == 1
