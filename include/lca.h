@@ -250,11 +250,11 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
                       int32_t *anchor, void *ws, size_t ws_bytes, void *stream);
 
 /* lca_decode without any device allocation, for callers that cannot call
- * cudaMalloc or hand the library a workspace: code running inside a stream
- * capture or under an allocator that forbids new device memory, plugins that
- * only receive pre-allocated input and output buffers, and embedded runtimes
- * with a fixed memory plan.  (The page has no counterpart: this is an
- * interface convenience, not part of the method.)
+ * cudaMalloc or hand the library a workspace: plugins and operators that
+ * only receive their pre-allocated input and output buffers, runtimes whose
+ * device memory plan is fixed before they start, and allocators that forbid
+ * new device memory while they run.  (The page has no counterpart: this is
+ * an interface convenience, not part of the method.)
  *
  * Same arguments and results as lca_decode, minus ws / ws_bytes: the scratch
  * (summary query, split-L partials) lives in a file-scope device array of
@@ -263,14 +263,16 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
  * otherwise LCA_ERR_SCRATCH_LIMIT and nothing is launched; g must be 16
  * (or 1, which is MLA decode as for lca_decode).
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before capturing a stream.  All calls on a device share the one array:
- * every byte a call reads is written earlier in the same call (nothing needs
- * to start at zero), but two calls whose work overlaps on the GPU (different
- * streams, or host threads racing) corrupt each other's results.  With
- * kernel timing switched on (lca_profile_enable) the library creates CUDA
- * event objects; leave it off where that is not allowed. */
+ * The first call on a device does its set-up, with that device current: it
+ * looks up the array's device address (cudaGetSymbolAddress) and runs the
+ * library's one-time per-device set-up (kernel attributes, the tensor-map
+ * encoder).  Make that first call before any stream capture.  All calls on
+ * a device share the one array: every byte a call reads is written earlier
+ * in the same call (nothing needs to start at zero), but two calls whose
+ * work overlaps on the GPU (different streams, or host threads racing)
+ * corrupt each other's results.  With kernel timing switched on
+ * (lca_profile_enable) the library creates CUDA event objects; leave it off
+ * where that is not allowed. */
 #define LCA_NOALLOC_MAX_BATCH 8
 int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, const void *w_uv,
                        int B, int64_t L, lca_params p, float *out, float *o_lat, int32_t *anchor,

@@ -47,21 +47,22 @@ def _load():
         lib.ora_num_threads.restype = I
         lib.ora_num_groups.restype = Lg
         lib.ora_num_groups.argtypes = [Lg, I, I]
-        lib.ora_lca_condense_v.restype = I
-        lib.ora_lca_condense_v.argtypes = [P, P, I, Lg, I, I, I, I, I, Dd, I, P, P, P, P, P]
+        lib.ora_lca_condense_fv.restype = I
+        lib.ora_lca_condense_fv.argtypes = [P, P, I, Lg, I, I, I, I, I, Dd, I, P, P, P, P, P, P]
         lib.ora_mla_decode.restype = I
         lib.ora_mla_decode.argtypes = [P, P, P, I, Lg, I, I, I, I, Dd, P, P]
-        lib.ora_lca_decode.restype = I
-        lib.ora_lca_decode.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
+        lib.ora_lca_decode_f.restype = I
+        lib.ora_lca_decode_f.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P, P]
         lib.ora_lca_attend_reps.restype = I
         lib.ora_lca_attend_reps.argtypes = [P, P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P]
-        lib.ora_lca_decode_stored.restype = I
-        lib.ora_lca_decode_stored.argtypes = [P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P]
-        lib.ora_lca_decode_shard.restype = I
-        lib.ora_lca_decode_shard.argtypes = [P, P, P, I, Lg, I, I, I, I, I, Dd, Lg, Lg, P, P, P]
-        lib.ora_lca_prefill_v.restype = I
-        lib.ora_lca_prefill_v.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, I, P, Lg,
-                                          P, P, P]
+        lib.ora_lca_decode_stored_f.restype = I
+        lib.ora_lca_decode_stored_f.argtypes = [P, P, P, I, Lg, I, I, I, I, I, I, Dd, P, P, P, P]
+        lib.ora_lca_decode_shard_f.restype = I
+        lib.ora_lca_decode_shard_f.argtypes = [P, P, P, I, Lg, I, I, I, I, I, Dd, Lg, Lg, P, P, P,
+                                               P]
+        lib.ora_lca_prefill_fv.restype = I
+        lib.ora_lca_prefill_fv.argtypes = [P, P, P, I, Lg, Lg, Lg, I, I, I, I, I, I, Dd, I, P, Lg,
+                                           P, P, P, P]
         _lib = lib
     return _lib
 
@@ -81,6 +82,24 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _forced(anchor_in, shape):
+    """Forced anchors (absolute positions) as a contiguous int32 array of
+    `shape`, or None."""
+    if anchor_in is None:
+        return None
+    a = np.ascontiguousarray(np.asarray(anchor_in, dtype=np.int32))
+    if a.shape != tuple(shape):
+        raise ValueError(f"anchor_in has shape {a.shape}, expected {tuple(shape)}")
+    return a
+
+
+def _check_forced(rc):
+    if rc == -2:
+        raise ValueError("a forced anchor lies outside its group")
+    if rc != 0:
+        raise ValueError(f"oracle call failed ({rc})")
+
+
 def num_threads() -> int:
     return _load().ora_num_threads()
 
@@ -95,10 +114,14 @@ def num_groups(L: int, g: int, w: int) -> int:
 LCA, POOL_POSITION, SPARSE = 0, 1, 2
 
 
-def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64, variant: int = LCA):
+def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64, variant: int = LCA,
+                 anchor_in=None):
     """cache [B,L,dc+dr] u16, q_recent [B,g,H,dc+dr] u16 ->
     dict(rep_c [B,m,dc], rep_k [B,m,dr], anchor [B,m] int32 (position in the
-    sequence), alpha [B,m,g], score [B,m,g])."""
+    sequence), alpha [B,m,g], score [B,m,g]).  anchor_in [B,m] (absolute
+    positions) forces the anchors instead of the argmax ("forced-anchor"
+    mode, for checking a result computed with another valid anchor where the
+    group maximum is a near-tie); nothing else changes."""
     cache, q_recent = _u16(cache), _u16(q_recent)
     B, L, D = cache.shape
     H = q_recent.shape[2]
@@ -107,9 +130,11 @@ def lca_condense(cache, q_recent, g: int, w: int, scale: float, dr: int = 64, va
     out = dict(rep_c=np.zeros((B, m, dc)), rep_k=np.zeros((B, m, dr)),
                anchor=np.zeros((B, m), np.int32), alpha=np.zeros((B, m, g)),
                score=np.zeros((B, m, g)))
-    _load().ora_lca_condense_v(_ptr(cache), _ptr(q_recent), B, L, H, dc, dr, g, w, scale, int(variant),
-                             _ptr(out["rep_c"]), _ptr(out["rep_k"]), _ptr(out["anchor"]),
-                             _ptr(out["alpha"]), _ptr(out["score"]))
+    forced = _forced(anchor_in, (B, m))
+    _check_forced(_load().ora_lca_condense_fv(
+        _ptr(cache), _ptr(q_recent), B, L, H, dc, dr, g, w, scale, int(variant), _ptr(forced),
+        _ptr(out["rep_c"]), _ptr(out["rep_k"]), _ptr(out["anchor"]), _ptr(out["alpha"]),
+        _ptr(out["score"])))
     return out
 
 
@@ -127,8 +152,10 @@ def mla_decode(cache, q, w_uv, scale: float, dr: int = 64):
     return o_lat, out
 
 
-def lca_decode(cache, q_recent, q, w_uv, g: int, w: int, scale: float, dr: int = 64):
-    """-> (o_lat [B,H,dc], out [B,H,dv], anchor [B,m])."""
+def lca_decode(cache, q_recent, q, w_uv, g: int, w: int, scale: float, dr: int = 64,
+               anchor_in=None):
+    """-> (o_lat [B,H,dc], out [B,H,dv], anchor [B,m]).  anchor_in [B,m]:
+    forced anchors (see lca_condense)."""
     cache, q_recent, q, w_uv = _u16(cache), _u16(q_recent), _u16(q), _u16(w_uv)
     B, L, D = cache.shape
     H = q.shape[1]
@@ -138,16 +165,19 @@ def lca_decode(cache, q_recent, q, w_uv, g: int, w: int, scale: float, dr: int =
     o_lat = np.zeros((B, H, dc))
     out = np.zeros((B, H, dv))
     anchor = np.zeros((B, max(m, 1)), np.int32)
-    _load().ora_lca_decode(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L, H, dc, dr,
-                           dv, g, w, scale, _ptr(o_lat), _ptr(out), _ptr(anchor))
+    forced = _forced(anchor_in, (B, m))
+    _check_forced(_load().ora_lca_decode_f(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
+                                           H, dc, dr, dv, g, w, scale, _ptr(forced), _ptr(o_lat),
+                                           _ptr(out), _ptr(anchor)))
     return o_lat, out, anchor[:, :m]
 
 
 def lca_decode_shard(cache, q_recent, q, g: int, w: int, scale: float, row0: int, row1: int,
-                     dr: int = 64):
+                     dr: int = 64, anchor_in=None):
     """One shard (rows row0 .. row1-1) of the LCA decode attention.
     -> (o [B,H,dc] normalised over the shard's rows, lse [B,H] = natural
-    log-sum-exp of the shard's logits, anchor [B,m_shard] absolute)."""
+    log-sum-exp of the shard's logits, anchor [B,m_shard] absolute).
+    anchor_in [B,m] (every group of the sequence, absolute): forced anchors."""
     cache, q_recent, q = _u16(cache), _u16(q_recent), _u16(q)
     B, L, D = cache.shape
     H = q.shape[1]
@@ -157,10 +187,13 @@ def lca_decode_shard(cache, q_recent, q, g: int, w: int, scale: float, row0: int
     o = np.zeros((B, H, dc))
     lse = np.zeros((B, H))
     anchor = np.zeros((B, max(m_shard, 1)), np.int32)
-    rc = _load().ora_lca_decode_shard(_ptr(cache), _ptr(q_recent), _ptr(q), B, L, H, dc, dr, g, w,
-                                      scale, row0, row1, _ptr(o), _ptr(lse), _ptr(anchor))
-    if rc != 0:
+    forced = _forced(anchor_in, (B, m))
+    rc = _load().ora_lca_decode_shard_f(_ptr(cache), _ptr(q_recent), _ptr(q), B, L, H, dc, dr, g,
+                                        w, scale, row0, row1, _ptr(forced), _ptr(o), _ptr(lse),
+                                        _ptr(anchor))
+    if rc == -1:
         raise ValueError("shard rows must start at a group boundary and be non-empty")
+    _check_forced(rc)
     return o, lse, anchor[:, :m_shard]
 
 
@@ -193,11 +226,13 @@ def lca_attend_reps(cache, rep, q, w_uv, g: int, w: int, scale: float, dr: int =
     return o_lat, out
 
 
-def lca_decode_stored(cache, q_all, w_uv, g: int, w: int, scale: float, dr: int = 64):
+def lca_decode_stored(cache, q_all, w_uv, g: int, w: int, scale: float, dr: int = 64,
+                      anchor_in=None):
     """Stored-representative decode at cache length L: group j condensed with
     the summary query of the step where it left the window (queries at
     positions w + g j .. w + g j + g - 1), query at L-1 attends [reps || window].
-    q_all [B,L,H,D] u16.  -> (o_lat [B,H,dc], out [B,H,dv], anchor [B,m])."""
+    q_all [B,L,H,D] u16.  -> (o_lat [B,H,dc], out [B,H,dv], anchor [B,m]).
+    anchor_in [B,m]: forced anchors (see lca_condense)."""
     cache, q_all, w_uv = _u16(cache), _u16(q_all), _u16(w_uv)
     B, L, D = cache.shape
     H = q_all.shape[2]
@@ -207,17 +242,22 @@ def lca_decode_stored(cache, q_all, w_uv, g: int, w: int, scale: float, dr: int 
     o_lat = np.zeros((B, H, dc))
     out = np.zeros((B, H, dv))
     anchor = np.zeros((B, max(m, 1)), np.int32)
-    _load().ora_lca_decode_stored(_ptr(cache), _ptr(q_all), _ptr(w_uv), B, L, H, dc, dr, dv, g, w,
-                                  scale, _ptr(o_lat), _ptr(out), _ptr(anchor))
+    forced = _forced(anchor_in, (B, m))
+    _check_forced(_load().ora_lca_decode_stored_f(_ptr(cache), _ptr(q_all), _ptr(w_uv), B, L, H,
+                                                  dc, dr, dv, g, w, scale, _ptr(forced),
+                                                  _ptr(o_lat), _ptr(out), _ptr(anchor)))
     return o_lat, out, anchor[:, :m]
 
 
 def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, scale: float,
                 blocks=None, dr: int = 64, want_anchor: bool = False, want_olat: bool = True,
-                variant: int = LCA):
+                variant: int = LCA, anchor_in=None):
     """Blockwise LCA prefill.  -> (o_lat [B,q_len,H,dc] | None, out [B,q_len,H,dv], anchor|None).
     `blocks` = absolute block indices to evaluate (others left as NaN).
-    `variant`: the method (LCA) or an ablation (POOL_POSITION, SPARSE)."""
+    `variant`: the method (LCA) or an ablation (POOL_POSITION, SPARSE).
+    anchor_in [B, q_len/g, max(1, m_last)] (laid out like the anchor output;
+    entries of groups a block does not have are ignored): forced anchors of
+    the evaluated blocks (see lca_condense)."""
     cache, qpre, w_uv = _u16(cache), _u16(qpre), _u16(w_uv)
     B, L, D = cache.shape
     H = qpre.shape[2]
@@ -232,9 +272,11 @@ def lca_prefill(cache, qpre, w_uv, q_start: int, q_len: int, g: int, w: int, sca
         nbl = len(bl)
     m_max = num_groups(q_start + q_len - g, g, w)
     anchor = np.full((B, q_len // g, max(m_max, 1)), -1, np.int32) if want_anchor else None
-    rc = _load().ora_lca_prefill_v(_ptr(cache), _ptr(qpre), _ptr(w_uv), B, L, q_start, q_len, H,
-                                   dc, dr, dv, g, w, scale, int(variant), _ptr(bl), nbl, _ptr(o_lat),
-                                   _ptr(out), _ptr(anchor))
-    if rc != 0:
+    forced = _forced(anchor_in, (B, q_len // g, max(m_max, 1)))
+    rc = _load().ora_lca_prefill_fv(_ptr(cache), _ptr(qpre), _ptr(w_uv), B, L, q_start, q_len, H,
+                                    dc, dr, dv, g, w, scale, int(variant), _ptr(bl), nbl,
+                                    _ptr(forced), _ptr(o_lat), _ptr(out), _ptr(anchor))
+    if rc == -1:
         raise ValueError("bad prefill range")
+    _check_forced(rc)
     return o_lat, out, anchor

@@ -95,12 +95,15 @@ enum { ORA_LCA = 0, ORA_POOL_POSITION = 1, ORA_SPARSE = 2 };
 /* 关键设计 1 + 2 for one group of g rows starting at `rows`:
  * alpha = softmax(s) over the group, rep_c = sum_i alpha_i c_i,
  * I = argmax_i s_i (first index on an exact tie), rep_k = k^R_I.
+ * forced >= 0 replaces the argmax by that offset ("forced-anchor" mode: the
+ * result for another valid choice of I where the maximum is a near-tie);
+ * nothing else changes.
  * Ablations (消融实验): ORA_POOL_POSITION pools the RoPE key with the same
  * weights, rep_k = sum_i alpha_i k^R_i ("纯池化（含位置）"); ORA_SPARSE keeps
  * only the most important token, rep_c = c_I, rep_k = k^R_I ("纯稀疏").
  * Returns I (offset inside the group). */
 static int condense_group_v(const double *qv, const uint16_t *rows, int g, int H, int dc, int dr,
-                            double scale, int variant, double *rep_c, double *rep_k,
+                            double scale, int variant, int forced, double *rep_c, double *rep_k,
                             double *alpha_out, double *score_out)
 {
     int D = dc + dr;
@@ -111,6 +114,7 @@ static int condense_group_v(const double *qv, const uint16_t *rows, int g, int H
     double mx = s[0];
     for (int i = 1; i < g; i++)
         if (s[i] > mx) { mx = s[i]; I = i; }
+    if (forced >= 0) I = forced;
     double den = 0.0;
     for (int i = 0; i < g; i++) { a[i] = exp(s[i] - mx); den += a[i]; }
     for (int i = 0; i < g; i++) a[i] /= den;
@@ -139,26 +143,35 @@ static int condense_group_v(const double *qv, const uint16_t *rows, int g, int H
     return I;
 }
 
-static int condense_group(const double *qv, const uint16_t *rows, int g, int H, int dc, int dr,
-                          double scale, double *rep_c, double *rep_k, double *alpha_out,
-                          double *score_out)
+/* Forced anchor of group j, or -1 for the argmax: anchor_in [B][m] holds
+ * absolute positions (NULL = no forcing).  Returns -2 for a position
+ * outside the group, which the callers report as an error. */
+static int forced_offset(const int32_t *anchor_in, size_t o, long j, int g)
 {
-    return condense_group_v(qv, rows, g, H, dc, dr, scale, ORA_LCA, rep_c, rep_k, alpha_out,
-                            score_out);
+    if (!anchor_in) return -1;
+    long off = (long)anchor_in[o] - j * g;
+    return (off >= 0 && off < g) ? (int)off : -2;
 }
 
 /* Condense every group of every sequence (decode: summary query from
  * q_recent).  Outputs (any may be NULL except none are required):
  * rep_c [B][m][dc], rep_k [B][m][dr], anchor [B][m] (absolute position
  * inside the sequence), alpha [B][m][g], score [B][m][g].  `variant`
- * selects the method or one of its ablations (condense_group_v). */
-int ora_lca_condense_v(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
-                       int dc, int dr, int g, int w, double scale, int variant, double *rep_c,
-                       double *rep_k, int32_t *anchor, double *alpha, double *score)
+ * selects the method or one of its ablations (condense_group_v).
+ * anchor_in [B][m] (absolute positions, or NULL) forces each group's anchor
+ * (forced-anchor mode); returns -2 if one lies outside its group. */
+int ora_lca_condense_fv(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
+                        int dc, int dr, int g, int w, double scale, int variant,
+                        const int32_t *anchor_in, double *rep_c, double *rep_k, int32_t *anchor,
+                        double *alpha, double *score)
 {
     int D = dc + dr;
     long m = ora_num_groups(L, g, w);
     if (m == 0) return 0;
+    if (anchor_in)
+        for (int b = 0; b < B; b++)
+            for (long j = 0; j < m; j++)
+                if (forced_offset(anchor_in, (size_t)b * m + j, j, g) < 0) return -2;
     double *qbar = (double *)malloc(sizeof(double) * (size_t)B * H * D);
     for (int b = 0; b < B; b++)
         summary_query(q_recent + (size_t)b * g * H * D, g, H, D, qbar + (size_t)b * H * D);
@@ -172,9 +185,10 @@ int ora_lca_condense_v(const uint16_t *cache, const uint16_t *q_recent, int B, l
         for (int b = 0; b < B; b++)
             for (long j = 0; j < m; j++) {
                 const uint16_t *rows = cache + ((size_t)b * L + (size_t)j * g) * D;
-                int I = condense_group_v(qbar + (size_t)b * H * D, rows, g, H, dc, dr, scale,
-                                         variant, rc, rk, al, sc);
                 size_t o = (size_t)b * m + j;
+                int I = condense_group_v(qbar + (size_t)b * H * D, rows, g, H, dc, dr, scale,
+                                         variant, forced_offset(anchor_in, o, j, g), rc, rk, al,
+                                         sc);
                 if (rep_c) memcpy(rep_c + o * dc, rc, sizeof(double) * dc);
                 if (rep_k) memcpy(rep_k + o * dr, rk, sizeof(double) * dr);
                 if (anchor) anchor[o] = (int32_t)(j * g + I);
@@ -188,6 +202,14 @@ int ora_lca_condense_v(const uint16_t *cache, const uint16_t *q_recent, int B, l
     }
     free(qbar);
     return 0;
+}
+
+int ora_lca_condense_v(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
+                       int dc, int dr, int g, int w, double scale, int variant, double *rep_c,
+                       double *rep_k, int32_t *anchor, double *alpha, double *score)
+{
+    return ora_lca_condense_fv(cache, q_recent, B, L, H, dc, dr, g, w, scale, variant, NULL,
+                               rep_c, rep_k, anchor, alpha, score);
 }
 
 int ora_lca_condense(const uint16_t *cache, const uint16_t *q_recent, int B, long L, int H,
@@ -290,17 +312,20 @@ int ora_mla_decode(const uint16_t *cache, const uint16_t *q, const uint16_t *w_u
 
 /* LCA decode: condense the m groups with the summary query of q_recent,
  * then the current query q attends [m representatives || window rows
- * m*g .. L-1].  anchor_out [B][m] may be NULL. */
-int ora_lca_decode(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q,
-                   const uint16_t *w_uv, int B, long L, int H, int dc, int dr, int dv, int g,
-                   int w, double scale, double *o_lat, double *out, int32_t *anchor_out)
+ * m*g .. L-1].  anchor_out [B][m] may be NULL.  anchor_in [B][m] (absolute
+ * positions) or NULL: forced anchors (ora_lca_condense_fv). */
+int ora_lca_decode_f(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q,
+                     const uint16_t *w_uv, int B, long L, int H, int dc, int dr, int dv, int g,
+                     int w, double scale, const int32_t *anchor_in, double *o_lat, double *out,
+                     int32_t *anchor_out)
 {
     int D = dc + dr;
     long m = ora_num_groups(L, g, w);
     double *rc = (double *)malloc(sizeof(double) * (size_t)B * (m > 0 ? m : 1) * dc);
     double *rk = (double *)malloc(sizeof(double) * (size_t)B * (m > 0 ? m : 1) * dr);
-    ora_lca_condense(cache, q_recent, B, L, H, dc, dr, g, w, scale, rc, rk, anchor_out, NULL,
-                     NULL);
+    int rcode = ora_lca_condense_fv(cache, q_recent, B, L, H, dc, dr, g, w, scale, ORA_LCA,
+                                    anchor_in, rc, rk, anchor_out, NULL, NULL);
+    if (rcode) { free(rc); free(rk); return rcode; }
     double *ol = (double *)malloc(sizeof(double) * (size_t)B * H * dc);
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < B; b++)
@@ -317,16 +342,26 @@ int ora_lca_decode(const uint16_t *cache, const uint16_t *q_recent, const uint16
     return 0;
 }
 
+int ora_lca_decode(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q,
+                   const uint16_t *w_uv, int B, long L, int H, int dc, int dr, int dv, int g,
+                   int w, double scale, double *o_lat, double *out, int32_t *anchor_out)
+{
+    return ora_lca_decode_f(cache, q_recent, q, w_uv, B, L, H, dc, dr, dv, g, w, scale, NULL,
+                            o_lat, out, anchor_out);
+}
+
 /* One shard of the LCA decode attention: the rows row0 .. row1-1 of each
  * sequence (row0 a multiple of g).  The groups among them (those below
  * m*g) are condensed exactly as in ora_lca_decode, and the current query
  * attends [those representatives || the shard's window rows] alone:
  * o_part [B][H][dc] is normalised over the shard's rows and
  * lse [B][H] = log sum exp(z) over them.  anchor_out [B][m_shard] (or NULL)
- * receives absolute positions. */
-int ora_lca_decode_shard(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q, int B,
-                         long L, int H, int dc, int dr, int g, int w, double scale, long row0,
-                         long row1, double *o_part, double *lse, int32_t *anchor_out)
+ * receives absolute positions.  anchor_in [B][m] (absolute positions of
+ * every group of the sequence) or NULL: forced anchors. */
+int ora_lca_decode_shard_f(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q,
+                           int B, long L, int H, int dc, int dr, int g, int w, double scale,
+                           long row0, long row1, const int32_t *anchor_in, double *o_part,
+                           double *lse, int32_t *anchor_out)
 {
     int D = dc + dr;
     long m = ora_num_groups(L, g, w);
@@ -339,7 +374,9 @@ int ora_lca_decode_shard(const uint16_t *cache, const uint16_t *q_recent, const 
     double *rc = (double *)malloc(sizeof(double) * (size_t)B * (m > 0 ? m : 1) * dc);
     double *rk = (double *)malloc(sizeof(double) * (size_t)B * (m > 0 ? m : 1) * dr);
     int32_t *an = (int32_t *)malloc(sizeof(int32_t) * (size_t)B * (m > 0 ? m : 1));
-    ora_lca_condense(cache, q_recent, B, L, H, dc, dr, g, w, scale, rc, rk, an, NULL, NULL);
+    int rcode = ora_lca_condense_fv(cache, q_recent, B, L, H, dc, dr, g, w, scale, ORA_LCA,
+                                    anchor_in, rc, rk, an, NULL, NULL);
+    if (rcode) { free(an); free(rc); free(rk); return rcode; }
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < B; b++)
         for (int h = 0; h < H; h++)
@@ -355,6 +392,14 @@ int ora_lca_decode_shard(const uint16_t *cache, const uint16_t *q_recent, const 
     free(rc);
     free(rk);
     return 0;
+}
+
+int ora_lca_decode_shard(const uint16_t *cache, const uint16_t *q_recent, const uint16_t *q, int B,
+                         long L, int H, int dc, int dr, int g, int w, double scale, long row0,
+                         long row1, double *o_part, double *lse, int32_t *anchor_out)
+{
+    return ora_lca_decode_shard_f(cache, q_recent, q, B, L, H, dc, dr, g, w, scale, row0, row1,
+                                  NULL, o_part, lse, anchor_out);
 }
 
 /* LCA decode attention over representatives supplied as bf16 rows
@@ -393,17 +438,30 @@ int ora_lca_attend_reps(const uint16_t *cache, const uint16_t *rep, const uint16
  * not processed are left untouched.  anchor_out, if not NULL, receives
  * [B][q_len/g][m_max] absolute anchor positions (m_max = max m_k over the
  * range, unused slots untouched).  `variant` selects the representative as
- * in condense_group_v: the method or one of the two ablations. */
-int ora_lca_prefill_v(const uint16_t *cache, const uint16_t *qpre, const uint16_t *w_uv, int B,
-                      long L, long q_start, long q_len, int H, int dc, int dr, int dv, int g, int w,
-                      double scale, int variant, const int64_t *blocks, long n_blocks, double *o_lat,
-                      double *out, int32_t *anchor_out)
+ * in condense_group_v: the method or one of the two ablations.  anchor_in
+ * (NULL, or laid out like anchor_out) forces the anchors of the processed
+ * blocks (forced-anchor mode); returns -2 if one lies outside its group. */
+int ora_lca_prefill_fv(const uint16_t *cache, const uint16_t *qpre, const uint16_t *w_uv, int B,
+                       long L, long q_start, long q_len, int H, int dc, int dr, int dv, int g,
+                       int w, double scale, int variant, const int64_t *blocks, long n_blocks,
+                       const int32_t *anchor_in, double *o_lat, double *out, int32_t *anchor_out)
 {
     int D = dc + dr;
     if (q_start % g || q_len % g || q_start < 0 || q_start + q_len > L) return -1;
     long nb_range = q_len / g;
     long nb = blocks ? n_blocks : nb_range;
     long m_max = ora_num_groups(q_start + q_len - g, g, w);
+    size_t m_row = (size_t)(m_max > 0 ? m_max : 1);
+    if (anchor_in)
+        for (int b = 0; b < B; b++)
+            for (long bi = 0; bi < nb; bi++) {
+                long k = blocks ? blocks[bi] : q_start / g + bi;
+                if (k * g < q_start || k * g + g > q_start + q_len) continue;
+                long m = ora_num_groups(k * g, g, w);
+                size_t base = ((size_t)b * nb_range + (size_t)(k - q_start / g)) * m_row;
+                for (long j = 0; j < m; j++)
+                    if (forced_offset(anchor_in, base + (size_t)j, j, g) < 0) return -2;
+            }
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < B; b++)
         for (long bi = 0; bi < nb; bi++) {
@@ -417,12 +475,12 @@ int ora_lca_prefill_v(const uint16_t *cache, const uint16_t *qpre, const uint16_
             summary_query(qb, g, H, D, qbar);
             double *rc = (double *)malloc(sizeof(double) * (m > 0 ? m : 1) * dc);
             double *rk = (double *)malloc(sizeof(double) * (m > 0 ? m : 1) * dr);
+            size_t abase = ((size_t)b * nb_range + (size_t)(k - q_start / g)) * m_row;
             for (long j = 0; j < m; j++) {
                 int I = condense_group_v(qbar, seq + (size_t)j * g * D, g, H, dc, dr, scale, variant,
+                                         forced_offset(anchor_in, abase + (size_t)j, j, g),
                                          rc + (size_t)j * dc, rk + (size_t)j * dr, NULL, NULL);
-                if (anchor_out)
-                    anchor_out[((size_t)b * nb_range + (k - q_start / g)) * (m_max > 0 ? m_max : 1) + j] =
-                        (int32_t)(j * g + I);
+                if (anchor_out) anchor_out[abase + (size_t)j] = (int32_t)(j * g + I);
             }
             double *ol = (double *)malloc(sizeof(double) * H * dc);
             for (int tt = 0; tt < g; tt++) {
@@ -441,6 +499,15 @@ int ora_lca_prefill_v(const uint16_t *cache, const uint16_t *qpre, const uint16_
             free(qbar);
         }
     return 0;
+}
+
+int ora_lca_prefill_v(const uint16_t *cache, const uint16_t *qpre, const uint16_t *w_uv, int B,
+                      long L, long q_start, long q_len, int H, int dc, int dr, int dv, int g, int w,
+                      double scale, int variant, const int64_t *blocks, long n_blocks, double *o_lat,
+                      double *out, int32_t *anchor_out)
+{
+    return ora_lca_prefill_fv(cache, qpre, w_uv, B, L, q_start, q_len, H, dc, dr, dv, g, w, scale,
+                              variant, blocks, n_blocks, NULL, o_lat, out, anchor_out);
 }
 
 /* The method's prefill (variant ORA_LCA). */
@@ -462,13 +529,19 @@ int ora_lca_prefill(const uint16_t *cache, const uint16_t *qpre, const uint16_t 
  * attends [the m(L) kept representatives || rows m g .. L-1] with the query
  * at position L - 1 (整体框架).
  *   q_all [B][L][H][D] holds the query of every position.
- *   anchor_out [B][m] (absolute positions) may be NULL. */
-int ora_lca_decode_stored(const uint16_t *cache, const uint16_t *q_all, const uint16_t *w_uv,
-                          int B, long L, int H, int dc, int dr, int dv, int g, int w,
-                          double scale, double *o_lat, double *out, int32_t *anchor_out)
+ *   anchor_out [B][m] (absolute positions) may be NULL.
+ *   anchor_in [B][m] (absolute positions) or NULL: forced anchors. */
+int ora_lca_decode_stored_f(const uint16_t *cache, const uint16_t *q_all, const uint16_t *w_uv,
+                            int B, long L, int H, int dc, int dr, int dv, int g, int w,
+                            double scale, const int32_t *anchor_in, double *o_lat, double *out,
+                            int32_t *anchor_out)
 {
     int D = dc + dr;
     long m = ora_num_groups(L, g, w);
+    if (anchor_in)
+        for (int b = 0; b < B; b++)
+            for (long j = 0; j < m; j++)
+                if (forced_offset(anchor_in, (size_t)b * m + j, j, g) < 0) return -2;
     size_t mm = (size_t)(m > 0 ? m : 1);
     double *rc = (double *)malloc(sizeof(double) * (size_t)B * mm * dc);
     double *rk = (double *)malloc(sizeof(double) * (size_t)B * mm * dr);
@@ -478,9 +551,11 @@ int ora_lca_decode_stored(const uint16_t *cache, const uint16_t *q_all, const ui
             long Lj = (long)w + (long)g * (j + 1);
             double *qbar = (double *)malloc(sizeof(double) * H * D);
             summary_query(q_all + ((size_t)b * L + (size_t)(Lj - g)) * H * D, g, H, D, qbar);
-            int I = condense_group(qbar, cache + ((size_t)b * L + (size_t)j * g) * D, g, H, dc,
-                                   dr, scale, rc + ((size_t)b * mm + j) * dc,
-                                   rk + ((size_t)b * mm + j) * dr, NULL, NULL);
+            int I = condense_group_v(qbar, cache + ((size_t)b * L + (size_t)j * g) * D, g, H, dc,
+                                     dr, scale, ORA_LCA,
+                                     forced_offset(anchor_in, (size_t)b * m + j, j, g),
+                                     rc + ((size_t)b * mm + j) * dc,
+                                     rk + ((size_t)b * mm + j) * dr, NULL, NULL);
             if (anchor_out) anchor_out[(size_t)b * m + j] = (int32_t)(j * g + I);
             free(qbar);
         }
@@ -499,4 +574,12 @@ int ora_lca_decode_stored(const uint16_t *cache, const uint16_t *q_all, const ui
     free(rc);
     free(rk);
     return 0;
+}
+
+int ora_lca_decode_stored(const uint16_t *cache, const uint16_t *q_all, const uint16_t *w_uv,
+                          int B, long L, int H, int dc, int dr, int dv, int g, int w,
+                          double scale, double *o_lat, double *out, int32_t *anchor_out)
+{
+    return ora_lca_decode_stored_f(cache, q_all, w_uv, B, L, H, dc, dr, dv, g, w, scale, NULL,
+                                   o_lat, out, anchor_out);
 }

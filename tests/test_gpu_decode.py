@@ -1,15 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on
-the same seeded inputs.
-
-Acceptance (the stated bar for bf16 inputs with fp32 accumulation):
-  * anchors (group argmax) bit-exact, except where the oracle's own scores
-    put the GPU's pick within 1e-4 * max|s| of the group maximum;
-  * outputs max-abs <= 2e-2 and mean-abs <= 2e-3 against fp64.
-Because decode outputs are small (|o| ~ 1e-2 for these input distributions),
-the absolute bar alone would accept almost anything, so every comparison also
-bounds the relative L2 error at 1e-2: the path rounds attention weights and
-o_lat to bf16 (relative 2^-9 ~ 2e-3 each), so 1e-2 leaves a 5x margin while
-still catching any wrong term, sign or index.
+the same seeded inputs, at the bar stated in tests/parity.py (anchors
+bit-exact except near-ties, which are re-checked against the oracle run with
+the GPU's anchors; outputs within max-abs 2e-2, mean-abs 2e-3 and relative
+L2 1e-2).  Output buffers carry guard regions that must stay untouched.
 """
 import numpy as np
 import pytest
@@ -18,42 +11,10 @@ import torch
 import oracle
 from mla_latent_space_lca_b200 import api
 from mla_latent_space_lca_b200.inputs import bf16_bits, make_decode_inputs
+from parity import (MAX_ABS, MEAN_ABS, NEAR_TIE, REL_L2, Canaries, check_anchors, compare,  # noqa: F401
+                    lca_decode_reference)
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS, MEAN_ABS, REL_L2 = 2e-2, 2e-3, 1e-2
-NEAR_TIE = 1e-4
-
-
-def compare(got, ref, what, rel=REL_L2):
-    got = np.asarray(got, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    assert got.shape == ref.shape, (what, got.shape, ref.shape)
-    assert np.isfinite(got).all(), f"{what}: non-finite values"
-    err = np.abs(got - ref)
-    rl2 = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    msg = f"{what}: max_abs={err.max():.3e} mean_abs={err.mean():.3e} rel_l2={rl2:.3e}"
-    assert err.max() <= MAX_ABS, msg
-    assert err.mean() <= MEAN_ABS, msg
-    assert rl2 <= rel, msg
-    return rl2
-
-
-def check_anchors(gpu_anchor, ora_anchor, ora_score, g=16):
-    """Bit-exact anchors except near-ties judged on the oracle's fp64 scores.
-    Returns (number of near-tie mismatches, number of groups)."""
-    gpu_anchor = np.asarray(gpu_anchor)
-    ora_anchor = np.asarray(ora_anchor)
-    assert gpu_anchor.shape == ora_anchor.shape
-    bad = np.argwhere(gpu_anchor != ora_anchor)
-    for idx in bad:
-        b, j = idx
-        s = ora_score[b, j]
-        gi = int(gpu_anchor[b, j]) - j * g
-        assert 0 <= gi < g, f"anchor outside its group at {tuple(idx)}"
-        gap = s[int(ora_anchor[b, j]) - j * g] - s[gi]
-        assert gap <= NEAR_TIE * np.abs(s).max(), f"anchor mismatch at {tuple(idx)}: gap {gap}"
-    return len(bad), gpu_anchor.size
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -78,9 +39,12 @@ def bits(inp):
 def test_mla_decode_parity(B, L):
     inp = make_decode_inputs(B, L, seed=100 + L)
     cache, _, q, w_uv = dev(inp)
-    o_lat = torch.empty(B, 16, 512, device="cuda")
-    out = api.mla_decode_attn(cache, q, w_uv, inp.scale, o_lat=o_lat)
+    cn = Canaries()
+    o_lat = cn.empty((B, 16, 512), torch.float32)
+    out = cn.empty((B, 16, 128), torch.float32)
+    api.mla_decode_attn(cache, q, w_uv, inp.scale, out=out, o_lat=o_lat)
     torch.cuda.synchronize()
+    cn.check("mla_decode_attn")
     c, _, qb, wb = bits(inp)
     ol_ref, out_ref = oracle.mla_decode(c, qb, wb, inp.scale)
     compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
@@ -105,21 +69,23 @@ def test_condense_parity(B, L, peak):
     inp = make_decode_inputs(B, L, seed=200 + L, peak=peak)
     cache, q_recent, _, _ = dev(inp)
     m = api.num_groups(L)
-    anchor = torch.full((B, max(m, 1)), -1, dtype=torch.int32, device="cuda")
-    alpha = torch.empty(B, max(m, 1), 16, device="cuda")
-    rep = api.lca_condense(cache, q_recent, scale=inp.scale, anchor=anchor, alpha=alpha)
+    cn = Canaries()
+    anchor = cn.empty((B, m), torch.int32)
+    alpha = cn.empty((B, m, 16), torch.float32)
+    rep = cn.empty((B, m, 576), torch.bfloat16)
+    api.lca_condense(cache, q_recent, scale=inp.scale, rep=rep, anchor=anchor, alpha=alpha)
     torch.cuda.synchronize()
+    cn.check("lca_condense")
     c, qr, _, _ = bits(inp)
     r = oracle.lca_condense(c, qr, 16, 1024, inp.scale)
     if m == 0:
-        assert rep.shape == (B, 0, 576)
         return
-    ga = anchor.cpu().numpy()[:, :m]
+    ga = anchor.cpu().numpy()
     check_anchors(ga, r["anchor"], r["score"])
     same = ga == r["anchor"]
     rep_f = rep.float().cpu().numpy()
     compare(rep_f[:, :, :512], r["rep_c"], "rep_c")
-    compare(alpha.cpu().numpy()[:, :m], r["alpha"], "alpha")
+    compare(alpha.cpu().numpy(), r["alpha"], "alpha")
     # the anchor's RoPE key is copied bit for bit
     kr_bits = c[:, :, 512:]
     rep_bits = rep.view(torch.int16).cpu().numpy().view(np.uint16)
@@ -146,15 +112,16 @@ def test_condense_ablation_variants(variant):
     r = oracle.lca_condense(c, qr, 16, 1024, inp.scale, variant=variant)
     ga = anchor.cpu().numpy()
     check_anchors(ga, r["anchor"], r["score"])
-    same = ga == r["anchor"]
+    if not np.array_equal(ga, r["anchor"]):      # near-ties: the GPU's anchors, forced
+        r = oracle.lca_condense(c, qr, 16, 1024, inp.scale, variant=variant, anchor_in=ga)
     rep_bits = rep.view(torch.int16).cpu().numpy().view(np.uint16)
     rows = c[np.arange(B)[:, None], ga]                 # the GPU's anchor rows
     if variant == 2:
         assert np.array_equal(rep_bits, rows)           # whole row, bit for bit
     else:
         rep_f = rep.float().cpu().numpy()
-        compare(rep_f[:, :, :512][same], r["rep_c"][same], "rep_c (pool position)")
-        compare(rep_f[:, :, 512:][same], r["rep_k"][same], "rep_k (pooled)")
+        compare(rep_f[:, :, :512], r["rep_c"], "rep_c (pool position)")
+        compare(rep_f[:, :, 512:], r["rep_k"], "rep_k (pooled)")
     ol_ref, out_ref = oracle.lca_attend_reps(c, rep_bits, qb, wb, 16, 1024, inp.scale)
     compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
     compare(out.cpu().numpy(), out_ref, "out")
@@ -199,17 +166,17 @@ def test_lca_decode_fused_parity(B, L, peak):
     inp = make_decode_inputs(B, L, seed=400 + L, peak=peak)
     cache, q_recent, q, w_uv = dev(inp)
     m = api.num_groups(L)
-    anchor = torch.full((B, max(m, 1)), -1, dtype=torch.int32, device="cuda")
-    o_lat = torch.empty(B, 16, 512, device="cuda")
-    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=o_lat, anchor=anchor)
+    cn = Canaries()
+    anchor = cn.empty((B, m), torch.int32)
+    o_lat = cn.empty((B, 16, 512), torch.float32)
+    out = cn.empty((B, 16, 128), torch.float32)
+    api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, out=out, o_lat=o_lat, anchor=anchor)
     torch.cuda.synchronize()
+    cn.check("lca_decode")
     c, qr, qb, wb = bits(inp)
-    ol_ref, out_ref, a_ref = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    ol_ref, out_ref, _, _ = lca_decode_reference(c, qr, qb, wb, anchor.cpu().numpy(), inp.scale)
     compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
     compare(out.cpu().numpy(), out_ref, "out")
-    if m > 0:
-        r = oracle.lca_condense(c, qr, 16, 1024, inp.scale)
-        check_anchors(anchor.cpu().numpy()[:, :m], a_ref, r["score"])
 
 
 @pytest.mark.parametrize("where", ["window", "history"])
@@ -228,11 +195,12 @@ def test_reference_max_rescale(where):
         inp.cache[b, pos] = row
     cache, q_recent, q, w_uv = dev(inp)
     o_lat = torch.empty(B, 16, 512, device="cuda")
-    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=o_lat)
+    anchor = torch.empty(B, api.num_groups(L), dtype=torch.int32, device="cuda")
+    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=o_lat, anchor=anchor)
     mla = api.mla_decode_attn(cache, q, w_uv, inp.scale)
     torch.cuda.synchronize()
     c, qr, qb, wb = bits(inp)
-    ol_ref, out_ref, _ = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    ol_ref, out_ref, _, _ = lca_decode_reference(c, qr, qb, wb, anchor.cpu().numpy(), inp.scale)
     compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
     compare(out.cpu().numpy(), out_ref, "out")
     _, mla_ref = oracle.mla_decode(c, qb, wb, inp.scale)
@@ -256,11 +224,12 @@ def test_reference_max_rescale_on_consecutive_tiles():
             inp.cache[b, 16 * j: 16 * (j + 1), 512:] = key
     cache, q_recent, q, w_uv = dev(inp)
     o_lat = torch.empty(B, 16, 512, device="cuda")
-    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=o_lat)
+    anchor = torch.empty(B, api.num_groups(L), dtype=torch.int32, device="cuda")
+    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=o_lat, anchor=anchor)
     mla = api.mla_decode_attn(cache, q, w_uv, inp.scale)
     torch.cuda.synchronize()
     c, qr, qb, wb = bits(inp)
-    ol_ref, out_ref, _ = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    ol_ref, out_ref, _, _ = lca_decode_reference(c, qr, qb, wb, anchor.cpu().numpy(), inp.scale)
     compare(o_lat.cpu().numpy(), ol_ref, "o_lat")
     compare(out.cpu().numpy(), out_ref, "out")
     _, mla_ref = oracle.mla_decode(c, qb, wb, inp.scale)
@@ -330,20 +299,21 @@ def full_size_check(B, L, sample, with_mla=False):
     inp = make_decode_inputs(B, L, seed=0)
     cache, q_recent, q, w_uv = dev(inp)
     m = api.num_groups(L)
-    anchor = torch.empty(B, m, dtype=torch.int32, device="cuda")
-    out = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, anchor=anchor)
+    cn = Canaries()
+    anchor = cn.empty((B, m), torch.int32)
+    out = cn.empty((B, 16, 128), torch.float32)
+    api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, out=out, anchor=anchor)
     mla = api.mla_decode_attn(cache, q, w_uv, inp.scale) if with_mla else None
     torch.cuda.synchronize()
+    cn.check("lca_decode")
     sl = list(sample)
     c = bf16_bits(inp.cache[sl])
     qr = bf16_bits(inp.q_recent[sl])
     qb = bf16_bits(inp.q[sl])
     wb = bf16_bits(inp.w_uv)
-    _, out_ref, a_ref = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    _, out_ref, _, nt = lca_decode_reference(c, qr, qb, wb, anchor.cpu().numpy()[sl], inp.scale)
     compare(out.cpu().numpy()[sl], out_ref, "out")
-    r = oracle.lca_condense(c, qr, 16, 1024, inp.scale)
-    nt, n = check_anchors(anchor.cpu().numpy()[sl], a_ref, r["score"])
-    assert nt <= max(3, n // 1000)
+    assert nt <= max(3, len(sl) * m // 1000)
     if with_mla:
         _, mla_ref = oracle.mla_decode(c, qb, wb, inp.scale)
         compare(mla.cpu().numpy()[sl], mla_ref, "mla out")

@@ -8,6 +8,9 @@ group maximum.  The oracle evaluates a subset of blocks where the full range
 would take it too long (blocks are independent given the cache); the subsets
 always include the first and last blocks, the blocks around the window edge,
 the 128-block condense tiles and the 256-block chunks of the GPU path.
+Where a near-tie anchor went the other way on the GPU, the outputs are
+compared with the oracle re-run on the GPU's anchors (forced-anchor mode).
+Output buffers carry guard regions that must stay untouched.
 """
 import numpy as np
 import pytest
@@ -17,7 +20,7 @@ import oracle
 from mla_latent_space_lca_b200 import api
 from mla_latent_space_lca_b200.inputs import bf16_bits, make_prefill_inputs
 
-from test_gpu_decode import NEAR_TIE, compare
+from parity import Canaries, FORCED_RERUNS, compare, prefill_anchor_check
 
 pytestmark = pytest.mark.gpu
 G = 16
@@ -32,21 +35,29 @@ def _device():
     assert rc == 0, f"device status {rc} detail {detail:#x}"
 
 
-def run_gpu(inp, q_start, q_len, w, variant=oracle.LCA):
+def run_gpu(inp, q_start, q_len, w, variant=oracle.LCA, canaries=True):
     cache, q, w_uv = inp.cache.cuda(), inp.q.cuda(), inp.w_uv.cuda()
     B = inp.B
     m_last = oracle.num_groups(q_start + q_len - G, G, w)
-    anchor = torch.full((B, q_len // G, max(m_last, 1)), -1, dtype=torch.int32, device="cuda")
-    o_lat = torch.empty(B, q_len, 16, 512, dtype=torch.float32, device="cuda")
-    out = api.lca_prefill_block(cache, q, w_uv, q_start, q_len, w=w, o_lat=o_lat, anchor=anchor,
-                                variant=variant)
+    cn = Canaries() if canaries else None
+    alloc = cn.empty if cn else (lambda shape, dt: torch.empty(shape, dtype=dt, device="cuda"))
+    anchor = alloc((B, q_len // G, max(m_last, 1)), torch.int32)
+    anchor.fill_(-1)
+    o_lat = alloc((B, q_len, 16, 512), torch.float32)
+    out = alloc((B, q_len, 16, 128), torch.float32)
+    api.lca_prefill_block(cache, q, w_uv, q_start, q_len, w=w, out=out, o_lat=o_lat, anchor=anchor,
+                          variant=variant)
     torch.cuda.synchronize()
+    if cn:
+        cn.check("lca_prefill_block")
     return out, o_lat, anchor
 
 
-def check_prefill(inp, q_start, q_len, w, blocks=None, gpu=None, variant=oracle.LCA):
+def check_prefill(inp, q_start, q_len, w, blocks=None, gpu=None, variant=oracle.LCA, max_flip_frac=0.01):
     """Compare the GPU prefill of [q_start, q_start+q_len) with the oracle on
-    `blocks` (absolute block indices; None = all)."""
+    `blocks` (absolute block indices; None = all).  At most max_flip_frac of
+    the groups may be near-tie anchor flips (None: no bound, for inputs with
+    planted ties).  Returns the number of flips."""
     out, o_lat, anchor = gpu if gpu is not None else run_gpu(inp, q_start, q_len, w, variant)
     k0 = q_start // G
     if blocks is None:
@@ -55,33 +66,22 @@ def check_prefill(inp, q_start, q_len, w, blocks=None, gpu=None, variant=oracle.
     cache_b, q_b = bf16_bits(inp.cache), bf16_bits(inp.q)
     ol_ref, out_ref, anc_ref = oracle.lca_prefill(cache_b, q_b, bf16_bits(inp.w_uv), q_start, q_len, G, w,
                                                   inp.scale, blocks=blocks, want_anchor=True, variant=variant)
+    anc = anchor.cpu().numpy()
+    n_bad, n_all = prefill_anchor_check(cache_b, q_b, w, inp.scale, k0, blocks, anc, anc_ref)
+    if max_flip_frac is not None:
+        assert n_bad <= max(1, int(n_all * max_flip_frac)), f"{n_bad} near-tie anchor flips of {n_all}"
+    if n_bad:
+        # two valid results: compare with the oracle run on the GPU's anchors
+        forced = np.where(anc < 0, 0, anc)
+        ol_ref, out_ref, _ = oracle.lca_prefill(cache_b, q_b, bf16_bits(inp.w_uv), q_start, q_len, G, w,
+                                                inp.scale, blocks=blocks, variant=variant, anchor_in=forced)
+        FORCED_RERUNS["calls"] += 1
+        FORCED_RERUNS["flips"] += n_bad
     rows = np.concatenate([np.arange((k - k0) * G, (k - k0 + 1) * G) for k in blocks])
     rows_t = torch.as_tensor(rows, device="cuda")
     compare(out.index_select(1, rows_t).cpu().numpy(), out_ref[:, rows], "prefill out")
     compare(o_lat.index_select(1, rows_t).cpu().numpy(), ol_ref[:, rows], "prefill o_lat")
-    # anchors of every evaluated block and group
-    anc = anchor.cpu().numpy()
-    n_bad = n_all = 0
-    for k in blocks:
-        m = oracle.num_groups(G * k, G, w)
-        if m == 0:
-            continue
-        a_gpu = anc[:, k - k0, :m]
-        a_ref = anc_ref[:, k - k0, :m]
-        n_all += a_gpu.size
-        bad = np.argwhere(a_gpu != a_ref)
-        if len(bad) == 0:
-            continue
-        sc = oracle.lca_condense(np.ascontiguousarray(cache_b[:, :G * k]),
-                                 np.ascontiguousarray(q_b[:, G * k:G * k + G]), G, w, inp.scale)["score"]
-        for b, j in bad:
-            s = sc[b, j]
-            gi = int(a_gpu[b, j]) - j * G
-            assert 0 <= gi < G, f"block {k}: anchor outside its group ({b}, {j})"
-            gap = s[int(a_ref[b, j]) - j * G] - s[gi]
-            assert gap <= NEAR_TIE * np.abs(s).max(), f"block {k}: anchor mismatch ({b}, {j}) gap {gap}"
-            n_bad += 1
-    assert n_bad <= max(1, n_all // 100), f"{n_bad} near-tie anchor flips of {n_all}"
+    return n_bad
 
 
 @pytest.mark.parametrize("B,L,w,q_start,q_len,peak", [
@@ -138,9 +138,9 @@ def test_prefill_range_split_consistency():
     """Two calls over adjacent ranges give the rows of one call over both."""
     B, L, w = 1, 16 * 96, 256
     inp = make_prefill_inputs(B, L, w=w, seed=47)
-    full, _, _ = run_gpu(inp, 0, L, w)
-    a, _, _ = run_gpu(inp, 0, 16 * 40, w)
-    b, _, _ = run_gpu(inp, 16 * 40, L - 16 * 40, w)
+    full, _, _ = run_gpu(inp, 0, L, w, canaries=False)
+    a, _, _ = run_gpu(inp, 0, 16 * 40, w, canaries=False)
+    b, _, _ = run_gpu(inp, 16 * 40, L - 16 * 40, w, canaries=False)
     torch.testing.assert_close(torch.cat([a, b], dim=1), full, rtol=0, atol=0)
 
 
@@ -150,8 +150,8 @@ def test_prefill_split_over_ranks_by_work():
     from mla_latent_space_lca_b200.split_blocks import prefill_block_ranges
     B, L, w = 2, 16 * 700, 512
     inp = make_prefill_inputs(B, L, w=w, seed=48)
-    full, _, _ = run_gpu(inp, 0, L, w)
-    parts = [run_gpu(inp, qs, ql, w)[0] for qs, ql in prefill_block_ranges(L, 3, w=w)]
+    full, _, _ = run_gpu(inp, 0, L, w, canaries=False)
+    parts = [run_gpu(inp, qs, ql, w, canaries=False)[0] for qs, ql in prefill_block_ranges(L, 3, w=w)]
     torch.testing.assert_close(torch.cat(parts, dim=1), full, rtol=0, atol=0)
 
 

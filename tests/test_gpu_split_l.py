@@ -23,7 +23,7 @@ from mla_latent_space_lca_b200 import api
 from mla_latent_space_lca_b200.inputs import bf16_bits, make_decode_inputs
 from mla_latent_space_lca_b200.split_l import shard_bounds
 
-from test_gpu_decode import check_anchors, compare
+from parity import FORCED_RERUNS, check_anchors, compare, lca_decode_reference
 
 pytestmark = pytest.mark.gpu
 
@@ -74,19 +74,26 @@ def test_shard_records_and_merge_match_oracle(peak):
     for cuts in (balanced, ragged):
         recs, anchors = run_shards(cache, q_recent, q, L, cuts)
         o, lse2 = unpack(recs, B)
-        for s, (r0, r1) in enumerate(zip(cuts[:-1], cuts[1:])):
-            o_ref, lse_ref, _ = oracle.lca_decode_shard(c, qr, qb, 16, 1024, inp.scale, r0, r1)
-            compare(o[s], o_ref, f"shard [{r0},{r1}) o")
-            d = np.abs(lse2[s] - lse_ref * LOG2E).max()
-            assert d <= LSE2_TOL, f"shard [{r0},{r1}) lse2 off by {d:.3e}"
         gpu_anchor = np.concatenate([a.cpu().numpy() + r0 for a, r0 in anchors], axis=1)
         nt, n = check_anchors(gpu_anchor, a_ref, score)
         assert nt <= max(2, n // 1000)
+        # near-tie flips: every reference is taken with the GPU's anchors
+        forced = gpu_anchor if nt else None
+        ol_r, out_r = ol_ref, out_ref
+        if nt:
+            ol_r, out_r, _ = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale, anchor_in=forced)
+            FORCED_RERUNS["calls"] += 1
+            FORCED_RERUNS["flips"] += nt
+        for s, (r0, r1) in enumerate(zip(cuts[:-1], cuts[1:])):
+            o_ref, lse_ref, _ = oracle.lca_decode_shard(c, qr, qb, 16, 1024, inp.scale, r0, r1, anchor_in=forced)
+            compare(o[s], o_ref, f"shard [{r0},{r1}) o")
+            d = np.abs(lse2[s] - lse_ref * LOG2E).max()
+            assert d <= LSE2_TOL, f"shard [{r0},{r1}) lse2 off by {d:.3e}"
         ol = torch.empty(B, 16, 512, device="cuda")
         out = api.lca_combine_shards(recs, w_uv, B, o_lat=ol)
         torch.cuda.synchronize()
-        compare(ol.cpu().numpy(), ol_ref, "merged o_lat")
-        compare(out.cpu().numpy(), out_ref, "merged out")
+        compare(ol.cpu().numpy(), ol_r, "merged o_lat")
+        compare(out.cpu().numpy(), out_r, "merged out")
 
 
 def test_one_shard_merge_is_bit_exact_with_decode():
@@ -128,7 +135,9 @@ def test_million_token_sequence_in_eight_shards():
     fused = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=ol_fused, anchor=fused_anchor)
     torch.cuda.synchronize()
     c, qr, qb, wb = bf16_bits(inp.cache), bf16_bits(inp.q_recent), bf16_bits(inp.q), bf16_bits(inp.w_uv)
-    _, out_ref, a_ref = oracle.lca_decode(c, qr, qb, wb, 16, 1024, inp.scale)
+    gpu_anchor = np.concatenate([a.cpu().numpy() + r0 for a, r0 in anchors], axis=1)
+    _, out_ref, _, nt = lca_decode_reference(c, qr, qb, wb, gpu_anchor, inp.scale)
+    assert nt <= max(3, gpu_anchor.size // 1000)
     compare(out.cpu().numpy(), out_ref, "8-shard out")
     # against the fused decode: other split points give other reference
     # maxima, so the bf16-rounded attention weights differ at the 2^-9 level
@@ -136,9 +145,5 @@ def test_million_token_sequence_in_eight_shards():
     a, b = ol.double().cpu().numpy(), ol_fused.double().cpu().numpy()
     assert np.linalg.norm(a - b) / np.linalg.norm(b) <= 2e-3
     compare(out.cpu().numpy(), fused.cpu().numpy(), "8-shard out vs fused")
-    gpu_anchor = np.concatenate([a.cpu().numpy() + r0 for a, r0 in anchors], axis=1)
     # the fused kernel and the shards condense every group the same way
     assert np.array_equal(gpu_anchor, fused_anchor.cpu().numpy())
-    score = oracle.lca_condense(c, qr, 16, 1024, inp.scale)["score"]
-    nt, n = check_anchors(gpu_anchor, a_ref, score)
-    assert nt <= max(3, n // 1000)

@@ -4,7 +4,9 @@ lca_decode_stored, through the C ABI) against the fp64 oracle.
 Each group is condensed once, at the decode step where it leaves the window
 (cache length w + 16 (j + 1)), with that step's summary query, and kept in a
 representative cache; every step then attends [kept representatives ||
-window].  Same bar as the other parity tests (see test_gpu_decode).
+window].  Same bar as the other parity tests (tests/parity.py), near-tie
+anchor flips included: the outputs are then compared with the oracle re-run
+on the GPU's anchors.
 """
 import numpy as np
 import pytest
@@ -15,7 +17,7 @@ from mla_latent_space_lca_b200 import api
 from mla_latent_space_lca_b200._lib import LCA_ERR_INVALID_ARG, LcaError
 from mla_latent_space_lca_b200.inputs import bf16_bits, make_decode_inputs, make_prefill_inputs
 
-from test_gpu_decode import NEAR_TIE, compare
+from parity import FORCED_RERUNS, NEAR_TIE, Canaries, compare
 
 pytestmark = pytest.mark.gpu
 G = 16
@@ -63,9 +65,13 @@ class Stream:
     def step(self, L):
         if api.num_groups(L, G, self.w) > self.m:
             self.append(L)
-        o_lat = torch.empty(self.inp.B, 16, 512, device="cuda")
-        out = api.lca_decode_stored(self.view(L), self.rep, self.q[:, L - 1].contiguous(), self.w_uv,
-                                    w=self.w, scale=self.inp.scale, o_lat=o_lat)
+        cn = Canaries()
+        o_lat = cn.empty((self.inp.B, 16, 512), torch.float32)
+        out = cn.empty((self.inp.B, 16, 128), torch.float32)
+        api.lca_decode_stored(self.view(L), self.rep, self.q[:, L - 1].contiguous(), self.w_uv,
+                              w=self.w, scale=self.inp.scale, out=out, o_lat=o_lat)
+        torch.cuda.synchronize()
+        cn.check(f"lca_decode_stored L={L}")
         return out, o_lat
 
 
@@ -75,11 +81,10 @@ def check_step(st, L, out, o_lat):
     qa = bf16_bits(inp.q[:, :L])
     ol_ref, out_ref, anc_ref = oracle.lca_decode_stored(c, qa, bf16_bits(inp.w_uv), G, st.w, inp.scale)
     torch.cuda.synchronize()
-    compare(out.cpu().numpy(), out_ref, f"stored out L={L}")
-    compare(o_lat.cpu().numpy(), ol_ref, f"stored o_lat L={L}")
     m = anc_ref.shape[1]
     got = st.anchor[:, :m].cpu().numpy()
-    for b, j in np.argwhere(got != anc_ref):
+    flips = np.argwhere(got != anc_ref)
+    for b, j in flips:
         Lj = st.w + G * (j + 1)
         sc = oracle.lca_condense(np.ascontiguousarray(c[:, :Lj]), np.ascontiguousarray(qa[:, Lj - G:Lj]),
                                  G, st.w, inp.scale)["score"][b, j]
@@ -87,6 +92,13 @@ def check_step(st, L, out, o_lat):
         assert 0 <= gi < G, f"anchor outside group ({b}, {j})"
         gap = sc[int(anc_ref[b, j]) - j * G] - sc[gi]
         assert gap <= NEAR_TIE * np.abs(sc).max(), f"anchor mismatch ({b}, {j}) gap {gap}"
+    if len(flips):
+        ol_ref, out_ref, _ = oracle.lca_decode_stored(c, qa, bf16_bits(inp.w_uv), G, st.w, inp.scale,
+                                                      anchor_in=got)
+        FORCED_RERUNS["calls"] += 1
+        FORCED_RERUNS["flips"] += len(flips)
+    compare(out.cpu().numpy(), out_ref, f"stored out L={L}")
+    compare(o_lat.cpu().numpy(), ol_ref, f"stored o_lat L={L}")
 
 
 @pytest.mark.parametrize("w,peak", [(64, 1.0), (100, 30.0)])

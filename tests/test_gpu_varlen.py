@@ -23,7 +23,7 @@ import oracle
 from mla_latent_space_lca_b200 import api
 from mla_latent_space_lca_b200.inputs import bf16_bits, make_decode_inputs
 
-from test_gpu_decode import check_anchors, compare
+from parity import Canaries, compare, lca_decode_reference
 
 pytestmark = pytest.mark.gpu
 
@@ -51,13 +51,17 @@ def run(inp, lens, g=16, w=1024):
     B, L = inp.B, inp.L
     cache = ragged(inp, lens)
     lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    m = api.num_groups(L, 16, w)
-    anchor = torch.full((B, max(m, 1)), -1, dtype=torch.int32, device="cuda")
-    o_lat = torch.empty(B, 16, 512, device="cuda")
-    out = api.lca_decode_varlen(cache, lens_d, inp.q_recent.cuda(), inp.q.cuda(), inp.w_uv.cuda(), g=g, w=w,
-                                scale=inp.scale, o_lat=o_lat, anchor=anchor)
+    m = api.num_groups(L, 16, w) if g != 1 else 0
+    cn = Canaries()
+    anchor = cn.empty((B, max(m, 1)), torch.int32)
+    anchor.fill_(-1)
+    o_lat = cn.empty((B, 16, 512), torch.float32)
+    out = cn.empty((B, 16, 128), torch.float32)
+    api.lca_decode_varlen(cache, lens_d, inp.q_recent.cuda(), inp.q.cuda(), inp.w_uv.cuda(), g=g, w=w,
+                          scale=inp.scale, out=out, o_lat=o_lat, anchor=anchor if g != 1 else None)
     torch.cuda.synchronize()
-    return out.cpu().numpy(), o_lat.cpu().numpy(), anchor.cpu().numpy()
+    cn.check("lca_decode_varlen")
+    return out.cpu().numpy(), o_lat.cpu().numpy(), anchor.cpu().numpy()[:, :m]
 
 
 @pytest.mark.parametrize("w", [1024, 64])
@@ -69,13 +73,10 @@ def test_ragged_batch_matches_oracle_per_sequence(w):
     for b, n in enumerate(lens):
         c = bf16_bits(inp.cache[b:b + 1, :n])
         qr, qb, wb = bf16_bits(inp.q_recent[b:b + 1]), bf16_bits(inp.q[b:b + 1]), bf16_bits(inp.w_uv)
-        ol_ref, out_ref, a_ref = oracle.lca_decode(c, qr, qb, wb, 16, w, inp.scale)
+        mb = oracle.num_groups(n, 16, w)
+        ol_ref, out_ref, _, _ = lca_decode_reference(c, qr, qb, wb, anchor[b:b + 1, :mb], inp.scale, w=w)
         compare(o_lat[b:b + 1], ol_ref, f"o_lat seq {b} (len {n})")
         compare(out[b:b + 1], out_ref, f"out seq {b} (len {n})")
-        mb = a_ref.shape[1]
-        if mb:
-            score = oracle.lca_condense(c, qr, 16, w, inp.scale)["score"]
-            check_anchors(anchor[b:b + 1, :mb], a_ref, score)
 
 
 def test_equal_lengths_reproduce_lca_decode():

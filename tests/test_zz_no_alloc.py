@@ -1,13 +1,15 @@
 """lca_decode_noalloc: the decode step for callers that cannot allocate device
-memory (no cudaMalloc, no caller workspace).  It must give the same results
-as lca_decode with a caller-provided workspace, call after call, although
-every call reuses the library's one built-in scratch array.
+memory (no cudaMalloc, no caller workspace).  It runs the same kernels with
+the same scratch layout as lca_decode, so its results must be bit-identical
+to lca_decode with a caller-provided workspace, call after call, although
+every call reuses the library's one built-in scratch array.  The largest
+batch runs first, so the later, smaller calls sit on top of stale non-zero
+scratch: a call that read a slot before writing it would differ.
 
 Kept in a file of its own that pytest collects last; it also passes when run
 alone in a fresh process."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
@@ -15,18 +17,6 @@ from mla_latent_space_lca_b200 import _lib, api
 from mla_latent_space_lca_b200.inputs import make_decode_inputs
 
 pytestmark = pytest.mark.gpu
-
-MAX_ABS, MEAN_ABS, REL_L2 = 2e-2, 2e-3, 1e-2   # the suite's output tolerance
-
-
-def _close(got, ref, what):
-    got = got.double().cpu().numpy()
-    ref = ref.double().cpu().numpy()
-    err = np.abs(got - ref)
-    rl2 = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    assert np.isfinite(got).all(), what
-    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS and rl2 <= REL_L2, \
-        f"{what}: max_abs={err.max():.3e} mean_abs={err.mean():.3e} rel_l2={rl2:.3e}"
 
 
 def _noalloc(lib, cache, q_recent, q, w_uv, scale, out, o_lat, anchor):
@@ -42,7 +32,8 @@ def _noalloc(lib, cache, q_recent, q, w_uv, scale, out, o_lat, anchor):
 def test_noalloc_matches_workspace_path_on_consecutive_calls(lcalib):
     assert torch.cuda.is_available()
     api.device_status(clear=True)
-    cases = [make_decode_inputs(4, 5000, seed=31), make_decode_inputs(8, 3000, seed=32, peak=8.0)]
+    big = make_decode_inputs(_lib.NOALLOC_MAX_BATCH, 3000, seed=32, peak=8.0)
+    cases = [big, make_decode_inputs(4, 5000, seed=31), make_decode_inputs(2, 1100, seed=30), big]
     for n, inp in enumerate(cases):
         cache, q_recent, q, w_uv = (t.cuda() for t in (inp.cache, inp.q_recent, inp.q, inp.w_uv))
         B, L = inp.B, inp.L
@@ -56,9 +47,10 @@ def test_noalloc_matches_workspace_path_on_consecutive_calls(lcalib):
         ref_anchor = torch.empty_like(anchor)
         ref = api.lca_decode(cache, q_recent, q, w_uv, scale=inp.scale, o_lat=ref_olat, anchor=ref_anchor)
         torch.cuda.synchronize()
-        _close(out, ref, f"out, call {n}")
-        _close(o_lat, ref_olat, f"o_lat, call {n}")
-        assert torch.equal(anchor, ref_anchor)
+        assert torch.isfinite(out).all() and torch.isfinite(o_lat).all()
+        assert torch.equal(out, ref), f"out, call {n}"
+        assert torch.equal(o_lat, ref_olat), f"o_lat, call {n}"
+        assert torch.equal(anchor, ref_anchor), f"anchor, call {n}"
     rc, detail = api.device_status(clear=True)
     assert rc == 0, f"device status {detail:#x}"
 
