@@ -9,28 +9,20 @@ are pinned here:
   definition: rep attention ~1.84e13 flops, window ~4.7e12, condensation
   ~1.15e12, W_UV ~2.7e11.
 """
-import importlib.util
-import os
-import sys
+import types
 
 import pytest
 
+from mla_latent_space_lca_b200.inputs import WORKLOADS
 from mla_latent_space_lca_b200.split_blocks import block_flops
-
-HERE = os.path.dirname(os.path.abspath(__file__))
 
 
 @pytest.fixture(scope="module")
 def bench():
-    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(HERE, "..", "bench.py"))
-    mod = importlib.util.module_from_spec(spec)
-    argv = sys.argv
-    try:
-        sys.argv = ["bench.py"]
-        spec.loader.exec_module(mod)
-    finally:
-        sys.argv = argv
-    return mod
+    from benchmarks import common
+    ns = types.SimpleNamespace(**{k: getattr(common, k) for k in dir(common) if not k.startswith("_")})
+    ns.WORKLOADS = WORKLOADS
+    return ns
 
 
 PER_KEY = 16 * (576 + 512) * 2        # 16 heads, q.k over 576 and p.v over 512
@@ -92,3 +84,29 @@ def test_cpu_baseline_runs_each_variant(bench, variant):
     pre = make_prefill_inputs(1, 1024, w=128, seed=4)
     tok_s, _, sample, times = bench.prefill_cpu_baseline(pre, 4, steps=1, variant=variant)
     assert tok_s > 0 and len(times) == 1
+
+
+def test_both_arms_print_the_same_config():
+    """The reference arm's config dict is built by the same function as the
+    GPU arm's, for every workload of the default suite."""
+    import bench as entry
+    from benchmarks import common
+    for wl in (entry.HEADLINE,) + entry.SUITE:
+        spec = WORKLOADS[wl]
+        if spec["kind"] == "decode":
+            flushed = spec["B"] * spec["L"] * common.ROW_BYTES < (256 << 20)
+            a = common.decode_config(wl, spec["B"], spec["L"], 1, "lca", flushed)
+            assert a["workload"] == wl and a["B_per_gpu"] == spec["B"] and a["L"] == spec["L"]
+            assert not flushed
+        else:
+            a = common.prefill_config(wl, spec["B"], spec["L"], 1, "lca", False, (0, spec["L"]))
+            assert a["rank0_queries"] == [0, spec["L"]]
+
+
+def test_default_run_arguments():
+    import bench as entry
+    a = entry.parse([])
+    assert a.workload is None and entry.defaults(a, entry.HEADLINE) == (2000, 20)
+    assert entry.defaults(a, "prefill_b1_l128k") == (10, 3)
+    a = entry.parse(["--steps", "7", "--warmup", "4"])
+    assert entry.defaults(a, entry.HEADLINE) == (7, 4)
