@@ -21,10 +21,10 @@ def _worker(rank, world, port, q):
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        import bench
+        from benchmarks import common
         from mla_latent_space_lca_b200.inputs import make_decode_inputs
-        t = bench.max_over_ranks(1.0 + 2.5 * rank, world)
-        inp = make_decode_inputs(1, 64, seed=bench.replica_seed(rank))
+        t = common.max_over_ranks(1.0 + 2.5 * rank, world)
+        inp = make_decode_inputs(1, 64, seed=common.replica_seed(rank))
         q.put((rank, t, float(inp.cache.float().sum())))
     finally:
         dist.destroy_process_group()
@@ -48,8 +48,8 @@ def test_max_over_ranks_and_replica_inputs():
 
 def test_single_rank_is_identity():
     sys.path.insert(0, ROOT)
-    import bench
-    assert bench.max_over_ranks(2.0, 1) == 2.0
+    from benchmarks import common
+    assert common.max_over_ranks(2.0, 1) == 2.0
 
 
 # ------------------------------------------------ decode split along the cache
