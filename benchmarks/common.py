@@ -182,6 +182,28 @@ def barrier(world: int):
         dist.barrier()
 
 
+class L2Flush:
+    """Evicts every input from the 126 MB L2 between timed steps: writes a
+    256 MB buffer, then reads another 256 MB buffer, so that the L2 is left
+    holding clean lines of that second buffer.  (After the write alone the
+    L2 is full of dirty lines, and the next step would pay for writing the
+    flush buffer back to HBM as its own reads evict them.)"""
+
+    BYTES = 256 << 20
+
+    def __init__(self, dev):
+        self.w = torch.empty(self.BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(self.BYTES // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def zero_(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.sink)
+
+    NOTE = ("flushed before every step (256 MB written, then another 256 MB read, so the L2 holds "
+            "none of the inputs and no dirty lines); steps timed one by one")
+
+
 def time_steps(step, n: int, stream, flush=None) -> float:
     """Milliseconds per step over n steps with CUDA events on `stream`:
     back to back, or (flush given) one by one after an L2 flush."""
@@ -218,9 +240,9 @@ def kernel_profile(lca, step, n: int, flush=None) -> dict:
 
 
 def flush_buffer(nbytes_inputs: int, dev):
-    """A 256 MB buffer to flush L2 between steps when the inputs would
-    otherwise stay in the 126 MB L2; None when they are larger."""
-    return torch.empty(256 << 20, dtype=torch.uint8, device=dev) if nbytes_inputs < (256 << 20) else None
+    """An L2 flush (L2Flush) between steps when the inputs would otherwise
+    stay in the 126 MB L2; None when they are larger."""
+    return L2Flush(dev) if nbytes_inputs < (256 << 20) else None
 
 
 def decode_config(workload: str, B: int, L: int, world: int, variant: str = "lca", flushed: bool = False):
@@ -228,8 +250,7 @@ def decode_config(workload: str, B: int, L: int, world: int, variant: str = "lca
     return {"workload": workload, "B_per_gpu": B, "L": L, "g": 16, "w": 1024,
             "heads": 16, "d_c": 512, "d_r": 64, "parallelism": f"replicas x{world}",
             "variant": variant,
-            "l2": ("flushed (256 MB write) before every step; steps timed one by one" if flushed else
-                   "inputs (B*L*1152 B) larger than the 126 MB L2; no flush")}
+            "l2": (L2Flush.NOTE if flushed else "inputs (B*L*1152 B) larger than the 126 MB L2; no flush")}
 
 
 def prefill_config(workload: str, B: int, L: int, world: int, variant: str = "lca", split: bool = False,

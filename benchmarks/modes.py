@@ -9,8 +9,8 @@ import torch
 
 from mla_latent_space_lca_b200.inputs import WORKLOADS, make_decode_inputs
 
-from .common import (METRIC, ROW_BYTES, ClockSampler, cpu_baseline, max_over_ranks, measured_hbm_peak, ncu_traffic,
-                     replica_seed)
+from .common import (METRIC, ROW_BYTES, ClockSampler, L2Flush, cpu_baseline, flush_buffer, max_over_ranks,
+                     measured_hbm_peak, ncu_traffic, replica_seed)
 
 
 def run_stored(args, rank, world, local_rank):
@@ -35,7 +35,7 @@ def run_stored(args, rank, world, local_rank):
     out = torch.empty(B, 16, 128, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     lca.lca_condense_append(cache, q_recent, rep, 0, scale=inp.scale, ws=ws, stream=stream)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def step(i):
         if i % 16 == 15 and m > 0:   # one group per sequence leaves the window every 16 steps
@@ -135,7 +135,7 @@ def run_stored(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": args.workload, "mode": "stored representatives", "B_per_gpu": B, "L": L,
                    "g": 16, "w": 1024, "kept_rows_per_seq": rows, "parallelism": f"replicas x{world}",
-                   "l2": "flushed (256 MB write) before every step; steps timed one by one"},
+                   "l2": L2Flush.NOTE},
         "read_gbps": read_bytes * world / (ms / 1e3) / 1e9,
         "kv_rows_read_fraction": rows / L,
         "roofline": {"bound": "hbm", "kernel": "attn_decode (stored representatives)", "achieved": achieved,
@@ -318,7 +318,7 @@ def run_split(args, rank, world, local_rank):
             dist.barrier()
 
     shard_bytes = B * (row1 - row0) * ROW_BYTES
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if shard_bytes < (256 << 20) else None
+    flush = flush_buffer(shard_bytes, dev)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -429,7 +429,7 @@ def run_split(args, rank, world, local_rank):
                    "d_c": 512, "d_r": 64, "parallelism": f"split-L x{world}",
                    "rank0_rows": [row0, row1],
                    "l2": ("shard larger than the 126 MB L2; no flush" if flush is None else
-                          "flushed (256 MB write) before every step")},
+                          L2Flush.NOTE)},
         "cache_gbps": B * L * ROW_BYTES / (ms / 1e3) / 1e9,
         "roofline": {"bound": "hbm", "kernel": "attn_decode (fused LCA, rank 0's shard)",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
