@@ -67,8 +67,11 @@ constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
 constexpr int AT_NBAR = 24;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
-constexpr int AT_OFF_ALB = AT_OFF_MISC + 256;           // per softmax warp: e [4 sub][16], anchors [4], 1/den [4]
-constexpr int AT_ALB = 72;                               // floats per softmax warp
+// per softmax warp: e [4 sub][16], anchors [4], 1/den [4], then the tile's
+// importance halves u_hi . row [64] and u_lo . row [64]
+constexpr int AT_OFF_ALB = AT_OFF_MISC + 256;
+constexpr int AT_ALB = 200;                              // floats per softmax warp
+constexpr int AT_ALB_SC = 72;                            // offset of the importance halves
 constexpr int AT_SMEM = AT_OFF_ALB + 4 * AT_ALB * 4;     // 226944
 constexpr int AT_SMEM_ALLOC = AT_SMEM + 1024;           // + alignment slack
 
@@ -496,55 +499,46 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 float w[16];        // P^T weights of this thread's head and tokens (g < 4)
                 float f = 1.f;      // reference-max rescale factor of this head
                 if (MODE == MODE_LCA && ti.hist) {
-                    // ---- fused condensation of 4 groups; threads g == 4 own u
+                    // ---- fused condensation of 4 groups.  Rows g = 4 and g = 5
+                    // hold u_hi . row and u_lo . row; they go through this warp's
+                    // shared-memory slot so that every lane takes 2 of the 64
+                    // tokens (group j = lanes 8j .. 8j+7): group max, first-index
+                    // argmax and denominator in 3 shuffle rounds, 2 exponentials
+                    // per lane.  al (exp(s - group max), unnormalised) comes back
+                    // in the layout each thread reads: [sub][x] for its tokens.
                     float al[16];       // exp(s - group max); alpha = al * rinv
                     float rinv[4];      // 1 / sum of the group's al
-                    int anc[4];
+                    int anc[4];         // the group's argmax (offset within the group)
+                    float *sch = alb + AT_ALB_SC;
+                    if (g == 4 || g == 5) {
+                        float *dst = sch + 64 * (g - 4);
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) al[x] = lo[x] + __shfl_down_sync(0xffffffffu, lo[x], 4);
+                        for (int j = 0; j < 8; ++j)
+                            *reinterpret_cast<float2 *>(dst + 8 * j + 2 * sub) = make_float2(lo[2 * j], lo[2 * j + 1]);
+                    }
+                    __syncwarp();
+                    {
+                        const float2 h2 = *reinterpret_cast<const float2 *>(sch + 2 * lane);
+                        const float2 l2 = *reinterpret_cast<const float2 *>(sch + 64 + 2 * lane);
+                        const float s0 = h2.x + l2.x, s1 = h2.y + l2.y;   // tokens 2 lane, 2 lane + 1
+                        float gm = s0;
+                        int gi = 2 * lane;
+                        if (s1 > gm) { gm = s1; gi = 2 * lane + 1; }
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        float sc[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) sc[e] = al[4 * k4 + e];
-                        // group max and first-index argmax (token order)
-                        float gm = sc[0];
-                        int gi = 2 * sub;
-#pragma unroll
-                        for (int e = 1; e < 4; ++e) {
-                            const int te = 8 * (e >> 1) + 2 * sub + (e & 1);
-                            if (sc[e] > gm) { gm = sc[e]; gi = te; }
-                        }
-#pragma unroll
-                        for (int off = 1; off <= 2; off <<= 1) {
+                        for (int off = 1; off <= 4; off <<= 1) {
                             const float og = __shfl_xor_sync(0xffffffffu, gm, off);
                             const int oi = __shfl_xor_sync(0xffffffffu, gi, off);
                             if (og > gm || (og == gm && oi < gi)) { gm = og; gi = oi; }
                         }
-                        float den = 0.f;
+                        const float e0 = fast_exp2((s0 - gm) * kLog2e), e1 = fast_exp2((s1 - gm) * kLog2e);
+                        float den = e0 + e1;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            sc[e] = fast_exp2((sc[e] - gm) * kLog2e);
-                            den += sc[e];
-                        }
-                        den += __shfl_xor_sync(0xffffffffu, den, 1);
-                        den += __shfl_xor_sync(0xffffffffu, den, 2);
-                        rinv[k4] = __fdividef(1.f, den);   // den >= 1 (the maximum's term)
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) al[4 * k4 + e] = sc[e];
-                        anc[k4] = gi;
-                    }
-                    // alpha of my tokens from thread (g=4, my sub), anchors from (g=4,
-                    // sub=0), through this warp's shared-memory slot
-                    __syncwarp();
-                    if (g == 4) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            *reinterpret_cast<float4 *>(alb + 16 * sub + 4 * v) =
-                                make_float4(al[4 * v], al[4 * v + 1], al[4 * v + 2], al[4 * v + 3]);
-                        if (sub == 0) {
-                            *reinterpret_cast<int4 *>(alb + 64) = make_int4(anc[0], anc[1], anc[2], anc[3]);
-                            *reinterpret_cast<float4 *>(alb + 68) = make_float4(rinv[0], rinv[1], rinv[2], rinv[3]);
+                        for (int off = 1; off <= 4; off <<= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+                        *reinterpret_cast<float2 *>(alb + 16 * (lane & 3) + 2 * (lane >> 2)) = make_float2(e0, e1);
+                        if ((lane & 7) == 0) {
+                            const int j = lane >> 3;
+                            reinterpret_cast<int *>(alb + 64)[j] = gi - 16 * j;
+                            alb[68 + j] = __fdividef(1.f, den);   // den >= 1 (the maximum's term)
                         }
                     }
                     __syncwarp();
