@@ -13,6 +13,31 @@ from .common import (METRIC, ROW_BYTES, ClockSampler, L2Flush, cpu_baseline, flu
                      measured_hbm_peak, ncu_traffic, replica_seed)
 
 
+def stored_cpu_baseline(inp, budget_s: float):
+    """The oracle's step over kept representatives (attention over [bf16
+    representatives || window], then W_UV) on one sequence, timed for about
+    budget_s on the host cores; the representatives come from the oracle's
+    own condensation, built before the timed loop."""
+    import numpy as np
+
+    import oracle
+    from mla_latent_space_lca_b200.inputs import bf16_bits
+
+    c = bf16_bits(inp.cache[:1])
+    qr, qb, w = bf16_bits(inp.q_recent[:1]), bf16_bits(inp.q[:1]), bf16_bits(inp.w_uv)
+    r = oracle.lca_condense(c, qr, inp.g, inp.w, inp.scale)
+    rep = bf16_bits(torch.from_numpy(np.concatenate([r["rep_c"], r["rep_k"]], axis=2)).to(torch.bfloat16))
+    n, total, t_start = 0, 0.0, time.time()
+    while n == 0 or time.time() - t_start < budget_s:
+        t0 = time.perf_counter()
+        oracle.lca_attend_reps(c, rep, qb, w, inp.g, inp.w, inp.scale)
+        total += time.perf_counter() - t0
+        n += 1
+    return {"value": n / total, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"1 of {inp.B} sequences (L={inp.L}) per oracle call, {n} calls, {total:.1f} s of CPU "
+                      "time: attention over the kept representatives and the window, then W_UV"}
+
+
 def run_stored(args, rank, world, local_rank):
     """Stored-representative decode: the representative cache is built once
     (untimed); a step is lca_decode_stored, plus every 16th step the append of
@@ -140,7 +165,8 @@ def run_stored(args, rank, world, local_rank):
         "kv_rows_read_fraction": rows / L,
         "roofline": {"bound": "hbm", "kernel": "attn_decode (stored representatives)", "achieved": achieved,
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak if achieved else None, "traffic": None,
+                     "frac": achieved / peak if achieved else None,
+                     "traffic": ncu_traffic(args.workload + "_stored"),
                      "algorithmic_bytes_per_launch": read_bytes, "launch_ms": attn_ms},
         "kernels_ms_per_step": {k: v[1] / prof_steps for k, v in prof.items()},
         "gpu_launches": launches,
@@ -151,6 +177,8 @@ def run_stored(args, rank, world, local_rank):
                         "device; per step the new token's row and query in from pinned host memory (every "
                         "16th step also the append of one group), out back"},
     }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = stored_cpu_baseline(inp, args.cpu_seconds / 2)
     return line
 
 
