@@ -73,7 +73,8 @@ def parse(argv=None):
                          "+ lca_decode_attn (the fused kernel has only the method), prefill passes it on")
     ap.add_argument("--mla-compare", type=int, default=None,
                     help="decode: also time N plain MLA decode steps (g = 1, every row attended) on the "
-                         "same inputs (default 200 on the headline workload, else 0); prefill: N full "
+                         "same inputs (default: the headline's step count on the headline workload, else "
+                         "0); prefill: N full "
                          "causal MLA prefills (w = L)")
     return ap.parse_args(argv)
 
@@ -112,7 +113,9 @@ def run_ours(args, rank, world, local_rank):
     if kind == "prefill":
         return run_prefill(args, workload, rank, world, local_rank, steps, warmup, split=args.split_blocks,
                            mla_compare=args.mla_compare or 0, with_cpu=with_cpu)
-    mla = args.mla_compare if args.mla_compare is not None else (0 if single else 200)
+    # the in-run MLA comparison runs as many steps as the headline, right
+    # after it, with its own clock record (the step is power-capped when long)
+    mla = args.mla_compare if args.mla_compare is not None else (0 if single else steps)
     line = run_decode(args, workload, rank, world, local_rank, steps, warmup, mla_compare=mla,
                       unfused_compare=args.unfused_compare, e2e_graph=not args.no_e2e_graph,
                       e2e_full_copy=args.e2e_full_copy, cpu_seconds=args.cpu_seconds, with_cpu=with_cpu)

@@ -102,10 +102,19 @@ def run_decode(args, workload, rank, world, local_rank, steps, warmup, *, mla_co
         for _ in range(3):
             mla_step()
         torch.cuda.synchronize()
-        mla_ms = max_over_ranks(time_steps(mla_step, mla_compare, stream, flush), world, dev)
+        msampler = ClockSampler(local_rank) if rank == 0 else None
+        time.sleep(0.25 if msampler else 0)
+        if msampler:
+            msampler.mark()
+        mla_ms_local = time_steps(mla_step, mla_compare, stream, flush)
+        if msampler:
+            msampler.mark()
+            msampler.stop()
+        mla_ms = max_over_ranks(mla_ms_local, world, dev)
         mprof = kernel_profile(lca, mla_step, min(mla_compare, 200), flush)
         mattn = mprof.get("attn_decode")
-        mla = {"ms_per_step": mla_ms, "attn_ms": mattn[1] / mattn[0] if mattn else None}
+        mla = {"ms_per_step": mla_ms, "attn_ms": mattn[1] / mattn[0] if mattn else None,
+               "clocks": msampler.summary() if msampler else None, "steps": mla_compare}
 
     # per-kernel durations (CUDA events around each launch, on its stream)
     prof = kernel_profile(lca, step, min(steps, 200), flush)
@@ -277,6 +286,7 @@ def run_decode(args, workload, rank, world, local_rank, steps, warmup, *, mla_co
             line["mla_path"] = {
                 "ms_per_step": mla["ms_per_step"], "tokens_per_s": tokens / (mla["ms_per_step"] / 1e3),
                 "lca_speedup": mla["ms_per_step"] / ms,
+                "steps": mla["steps"], "clocks": mla["clocks"],
                 "attn_ms": mla["attn_ms"],
                 "attn_frac_of_hbm": (algo_bytes / (mla["attn_ms"] / 1e3) / 1e9 / peak) if mla["attn_ms"] else None,
                 "note": "mla_decode_attn (g = 1): every cached row attended, same inputs and timing; "

@@ -233,25 +233,36 @@ __device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int qu
         }
     }
     const uint32_t base = tmem + (uint32_t(32 * quad) << 16) + AT_TM_Q;
+    // three 32-element chunks per round trip: their loads are all issued
+    // before the first TMEM store (which orders memory), so the 9 chunks take
+    // 3 global-memory latencies instead of 9
 #pragma unroll 1
-    for (int cc = 0; cc < 9; ++cc) {
-        uint32_t r[16];
-        const int e0 = off + 32 * cc;
-        if (src && !(e0 >= z0 && e0 < z1)) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(src + e0);
+    for (int c0 = 0; c0 < 9; c0 += 3) {
+        uint4 x[3][4];
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+            const int e0 = off + 32 * (c0 + u);
+            if (src && !(e0 >= z0 && e0 < z1)) {
+                const uint4 *p = reinterpret_cast<const uint4 *>(src + e0);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) x[u][v] = p[v];
+            } else {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) x[u][v] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 3; ++u) {
+            uint32_t r[16];
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-                const uint4 x = p[v];
-                r[4 * v + 0] = x.x;
-                r[4 * v + 1] = x.y;
-                r[4 * v + 2] = x.z;
-                r[4 * v + 3] = x.w;
+                r[4 * v + 0] = x[u][v].x;
+                r[4 * v + 1] = x[u][v].y;
+                r[4 * v + 2] = x[u][v].z;
+                r[4 * v + 3] = x[u][v].w;
             }
-        } else {
-#pragma unroll
-            for (int v = 0; v < 16; ++v) r[v] = 0u;
+            tmem_st16(base + 16 * (c0 + u), r);
         }
-        tmem_st16(base + 16 * cc, r);
     }
 }
 
