@@ -131,9 +131,9 @@ def run_decode(args, workload, rank, world, local_rank, steps, warmup, *, mla_co
         # one by one, with the L2 flush between them when the cache would
         # otherwise stay in L2.
         # the step's inputs travel in one pinned buffer [new rows | query]:
-        # one host-to-device copy, then the rows go into row L-1 of each
-        # sequence and the query into the ring on the device; the decode
-        # reads the query where it landed
+        # one host-to-device copy, then lca_append_token puts the rows into
+        # row L-1 of each sequence and the query into the ring in one launch;
+        # the decode reads the query where it landed
         pin_in = torch.cat([inp.cache[:, L - 1].reshape(-1), inp.q.reshape(-1)]).pin_memory()
         stage = torch.empty_like(pin_in, device=dev)
         d_row = stage[:B * 576].view(B, 576)
@@ -146,8 +146,7 @@ def run_decode(args, workload, rank, world, local_rank, steps, warmup, *, mla_co
 
         def e2e_step():
             stage.copy_(pin_in, non_blocking=True)
-            cache[:, L - 1].copy_(d_row)
-            ring[:, slot[0]].copy_(dq)
+            lca.lca_append_token(cache, L - 1, d_row, q=dq, ring=ring, slot=slot[0])
             slot[0] = (slot[0] + 1) % ring.shape[1]
             decode(ring, dq)
             h_out.copy_(out, non_blocking=True)
@@ -175,8 +174,7 @@ def run_decode(args, workload, rank, world, local_rank, steps, warmup, *, mla_co
         if e2e_graph:
             def graph_step(sl):
                 stage.copy_(pin_in, non_blocking=True)
-                cache[:, L - 1].copy_(d_row)
-                ring[:, sl].copy_(dq)
+                lca.lca_append_token(cache, L - 1, d_row, q=dq, ring=ring, slot=sl)
                 decode(ring, dq, st=None)
                 h_out.copy_(out, non_blocking=True)
 
@@ -275,7 +273,7 @@ def run_decode(args, workload, rank, world, local_rank, steps, warmup, *, mla_co
                 "note": ("lca_decode" if not variant else "lca_condense + lca_decode_attn") +
                         " in a decode loop: cache and recent-query ring resident on the device; "
                         "per step the new token's rows and query in from pinned host memory (one copy), "
-                        "placed into the cache and the ring, then out back"}
+                        "placed into the cache and the ring (lca_append_token), then out back"}
         if graph_ms is not None:
             line["e2e_graph"] = {
                 "value": tokens / (graph_ms / 1e3), "unit": "tokens/s", "ms_per_step": graph_ms,

@@ -315,6 +315,23 @@ int lca_decode_shard(const void *cache_shard, const void *q_recent, const void *
 int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv, float *out,
                        float *o_lat, void *stream);
 
+/* A decode loop's per-step bookkeeping in one launch (no counterpart on the
+ * page, whose method starts from a cache that already holds the current
+ * token): the current token's cache row of every sequence goes into row
+ * `pos` of its cache, and its absorbed query into slot `slot` of the
+ * recent-query ring that lca_decode and lca_condense take as q_recent (only
+ * the ring's mean is used, so the oldest slot is the one to overwrite).
+ *   rows  [B][576] bf16            the new rows
+ *   cache [B][pitch][576] bf16     written at row pos, 0 <= pos < pitch
+ *   q     [B][16][576] bf16        the new queries, or NULL (rows only)
+ *   ring  [B][g][16][576] bf16     written at slot, 0 <= slot < g; NULL with q
+ * All pointers are device pointers, 16-byte aligned; B * pitch < 2^40.  The
+ * kernel waits for all earlier work in the stream before it reads or
+ * writes, so an earlier kernel still reading the cache is never overtaken;
+ * the next call in the stream (lca_decode, ...) sees the writes. */
+int lca_append_token(const void *rows, void *cache, int B, int64_t pitch, int64_t pos, const void *q,
+                     void *ring, int g, int slot, void *stream);
+
 /* Self-test of the failure path (no counterpart on the page): launches one
  * kernel whose bounded wait can never be satisfied.  After ~2 s it records
  * LCA_ERR_DEVICE_TIMEOUT in the device status word (kernel id 8 in bits

@@ -32,7 +32,7 @@ EXPORTS = ("lca_num_groups", "lca_workspace_bytes", "mla_decode_attn", "lca_cond
            "lca_device_status", "lca_profile_enable", "lca_profile_collect", "lca_launch_count",
            "lca_decode_noalloc", "lca_condense_append", "lca_decode_stored",
            "lca_selftest_wait_timeout", "lca_decode_shard", "lca_combine_shards", "lca_decode_varlen",
-           "lca_decode_stored_varlen")
+           "lca_decode_stored_varlen", "lca_append_token")
 # floats per head in a shard record: o (512) and its base-2 log-sum-exp
 SHARD_RECORD_PER_HEAD = 513
 
@@ -83,6 +83,8 @@ def lib():
         L.lca_combine_shards.argtypes = [P, I, I, P, P, P, P]
         L.lca_selftest_wait_timeout.restype = I
         L.lca_selftest_wait_timeout.argtypes = [P]
+        L.lca_append_token.restype = I
+        L.lca_append_token.argtypes = [P, P, I, I64, I64, P, P, I, I, P]
         L.lca_condense_append.restype = I
         L.lca_condense_append.argtypes = [P, P, I, I64, LcaParams, I64, P, I64, P, P, P, SZ, P]
         L.lca_decode_stored.restype = I

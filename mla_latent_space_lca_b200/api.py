@@ -294,6 +294,35 @@ def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, 
     return out
 
 
+def lca_append_token(cache, pos, rows, q=None, ring=None, slot=0, stream=None):
+    """A decode loop's per-step bookkeeping in one launch: rows [B, 576] go
+    into row `pos` of each sequence of `cache` ([B, L, 576], packed or a view
+    of a larger [B, L_max, 576] buffer whose rows are contiguous), and, if
+    given, the queries q [B, 16, 576] into slot `slot` of `ring`
+    [B, g, 16, 576] (the q_recent of the next decode call)."""
+    if not isinstance(cache, torch.Tensor) or not cache.is_cuda or cache.dtype != torch.bfloat16:
+        raise TypeError("cache must be a CUDA bfloat16 tensor")
+    if cache.dim() != 3 or cache.shape[2] != D or cache.stride(2) != 1 or cache.stride(1) != D:
+        raise ValueError(f"cache must be [B, L, {D}] with contiguous rows")
+    B, L, _ = cache.shape
+    if cache.stride(0) % D or cache.stride(0) < L * D:
+        raise ValueError(f"cache must hold each sequence's rows contiguously (strides {cache.stride()})")
+    pitch = cache.stride(0) // D
+    if not 0 <= pos < L:
+        raise ValueError(f"pos {pos} outside the cache's {L} rows")
+    _need(rows, "rows", torch.bfloat16, (B, D))
+    g = 0
+    if q is not None or ring is not None:
+        _need(q, "q", torch.bfloat16, (B, H, D))
+        if not isinstance(ring, torch.Tensor) or ring.dim() != 4:
+            raise ValueError("ring must be [B, g, 16, 576]")
+        g = ring.shape[1]
+        _need(ring, "ring", torch.bfloat16, (B, g, H, D))
+    rc = _lib.lib().lca_append_token(_ptr(rows), _ptr(cache), B, pitch, int(pos), _ptr(q), _ptr(ring), g,
+                                     int(slot), _stream(stream))
+    check(rc, "lca_append_token")
+
+
 def device_status(clear: bool = True) -> tuple[int, int]:
     d = ctypes.c_int(0)
     rc = _lib.lib().lca_device_status(1 if clear else 0, ctypes.byref(d))

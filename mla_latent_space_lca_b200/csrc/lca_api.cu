@@ -22,6 +22,7 @@
 #include "prefill.cuh"
 #include "selftest.cuh"
 #include "varlen.cuh"
+#include "append.cuh"
 
 using namespace lca;
 
@@ -117,8 +118,8 @@ struct ProfRec {
     int kid;
 };
 const char *kKernelNames[] = {"",         "prep_summary", "condense",    "attn_decode",      "combine_wuv",
-                               "wuv_gemm", "attn_prefill", "condense_prefill", "selftest_wait"};
-constexpr int kNumKernelIds = 9;
+                               "wuv_gemm", "attn_prefill", "condense_prefill", "selftest_wait", "append_token"};
+constexpr int kNumKernelIds = 10;
 bool g_prof_on = false;
 std::vector<ProfRec> g_prof_used;
 std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
@@ -825,6 +826,27 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
         }
     }
     return LCA_OK;
+}
+
+int lca_append_token(const void *rows, void *cache, int B, int64_t pitch, int64_t pos, const void *q, void *ring,
+                     int g, int slot, void *stream)
+{
+    if (!rows || !cache || B < 1 || pitch < 1 || pos < 0 || pos >= pitch) return LCA_ERR_INVALID_ARG;
+    if (int64_t(B) * pitch >= (int64_t(1) << 40)) return LCA_ERR_INVALID_ARG;
+    if ((q == nullptr) != (ring == nullptr)) return LCA_ERR_INVALID_ARG;
+    if (q && (g < 1 || slot < 0 || slot >= g)) return LCA_ERR_INVALID_ARG;
+    if (!aligned16(rows) || !aligned16(cache) || (q && (!aligned16(q) || !aligned16(ring))))
+        return LCA_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Launch l(st, K_APPEND);
+    const cudaError_t e = launch_ex(append_token_kernel, dim3(B), dim3(APPEND_THREADS), 0, st, true,
+                                    static_cast<const uint4 *>(rows), static_cast<uint4 *>(cache), pitch, pos,
+                                    static_cast<const uint4 *>(q), static_cast<uint4 *>(ring), g, slot);
+    if (e != cudaSuccess) return LCA_ERR_CUDA;
+    return l.done();
 }
 
 int lca_selftest_wait_timeout(void *stream)

@@ -218,3 +218,26 @@ def test_binding_functions_reference_only_defined_globals():
                         if g not in vars(mod) and not hasattr(builtins, g):
                             missing.append(f"{mod.__name__}.{name}: {g}")
     assert not missing, missing
+
+
+def test_append_token_rejects_bad_arguments(lcalib):
+    f = lcalib.lca_append_token
+    ok = dict(rows=A, cache=A, B=2, pitch=100, pos=99, q=A, ring=A, g=16, slot=15)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["rows"], a["cache"], a["B"], a["pitch"], a["pos"], a["q"], a["ring"], a["g"], a["slot"], None)
+
+    inval = _lib.LCA_ERR_INVALID_ARG
+    assert call(rows=None) == inval
+    assert call(cache=None) == inval
+    assert call(B=0) == inval
+    assert call(pos=100) == inval and call(pos=-1) == inval
+    assert call(q=None) == inval                      # q and ring come together
+    assert call(slot=16) == inval and call(slot=-1) == inval and call(g=0) == inval
+    assert call(pitch=1 << 40, pos=0) == inval        # B * pitch must stay below 2^40
+    assert call(rows=A + 8) == _lib.LCA_ERR_MISALIGNED
+    assert call(ring=A + 4) == _lib.LCA_ERR_MISALIGNED
+    # rows only (no ring): valid arguments, then no device on this host
+    assert call(q=None, ring=None, g=0, slot=0) == _lib.LCA_ERR_NO_DEVICE
