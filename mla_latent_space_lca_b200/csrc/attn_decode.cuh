@@ -65,11 +65,16 @@ constexpr int AT_THREADS = 352;
 
 constexpr int AT_OFF_P = AT_STAGES * AT_STAGE;          // 221184
 constexpr int AT_OFF_BAR = AT_OFF_P + 2 * AT_PBUF;      // 225280
-constexpr int AT_NBAR = 24;
+constexpr int AT_NBAR = 26;
 constexpr int AT_OFF_MISC = AT_OFF_BAR + 8 * 32;        // 225536
 // per softmax warp: e [4 sub][16], anchors [4], 1/den [4], then the tile's
 // importance halves u_hi . row [64] and u_lo . row [64]
 constexpr int AT_OFF_ALB = AT_OFF_MISC + 256;
+// The first segment's query rows (and, fused, the folded summary query) are
+// staged in stage 2 by two bulk copies before its first tile load.
+constexpr int AT_OFF_QSTAGE = 2 * AT_STAGE;
+constexpr int AT_QBYTES = LCA_HEADS * LCA_D * 2;         // 18432: q of one sequence
+constexpr int AT_UBYTES = 2 * LCA_D * 2;                 // 2304: u_hi, u_lo of one sequence
 constexpr int AT_ALB = 200;                              // floats per softmax warp
 constexpr int AT_ALB_SC = 72;                            // offset of the importance halves
 constexpr int AT_SMEM = AT_OFF_ALB + 4 * AT_ALB * 4;     // 226944
@@ -208,9 +213,11 @@ __device__ __forceinline__ TileInfo tile_info(const SeqGeom &a, int k)
 }
 
 // Write this lane's 288-wide query half-row (or zeros) into TMEM columns
-// AT_TM_Q.. of its lane.  See the row map in the file header.
+// AT_TM_Q.. of its lane.  See the row map in the file header.  qb: the
+// sequence's 16 query rows, ub: its u_hi, u_lo rows (LCA), in global or
+// shared memory.
 template <int MODE>
-__device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int quad, int lane,
+__device__ __forceinline__ void load_q_rows(const uint16_t *qb, const uint16_t *ub, int quad, int lane,
                                             uint32_t tmem)
 {
     const int g = lane & 7, half = (lane >> 3) & 1;
@@ -219,14 +226,14 @@ __device__ __forceinline__ void load_q_rows(const AttnArgs &a, int64_t b, int qu
     int z0 = 0, z1 = 0;              // elements [z0, z1) are zeroed (32-aligned)
     if (lane < 16) {
         if (g < 4) {
-            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + g) * LCA_D;
+            src = qb + size_t(4 * quad + g) * LCA_D;
             if (MODE == MODE_LCA) { z0 = LCA_DC; z1 = LCA_D; }   // X: latent only
         } else if (MODE == MODE_LCA && (g == 4 || g == 5)) {
-            src = a.uhl + (size_t(b) * 2 + (g - 4)) * LCA_D;
+            src = ub + size_t(g - 4) * LCA_D;
         } else if (MODE == MODE_LCA) {
             // g = 6, 7: Y rows of heads 4q + (g-6) + 2*half, always the
             // second half [0 | q_rope] so that S_1 carries q_rope . k^R
-            src = a.q + (size_t(b) * LCA_HEADS + 4 * quad + (g - 6) + 2 * half) * LCA_D;
+            src = qb + size_t(4 * quad + (g - 6) + 2 * half) * LCA_D;
             off = 288;
             z0 = 288;
             z1 = LCA_DC;
@@ -288,6 +295,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     auto fex = [&](int s) { return BAR(17 + s); };
     const uint32_t drain2 = BAR(19), drain3 = BAR(20), drain4 = BAR(21), drain5 = BAR(22), drain6 = BAR(23);
     const uint32_t ofull = BAR(14), segready = BAR(15), drain = BAR(16);
+    const uint32_t qfull = BAR(24), qempty = BAR(25);   // the staged first query rows
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + AT_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + AT_OFF_MISC + 4);
     float *fsc = reinterpret_cast<float *>(smem + AT_OFF_MISC + 128);   // [2][16]
@@ -314,6 +322,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         mbar_init(drain6, 1);
         mbar_init(fex(0), 4);
         mbar_init(fex(1), 4);
+        mbar_init(qfull, MODE == MODE_LCA ? 2 : 1);   // producer (q); softmax warp 0 (u)
+        mbar_init(qempty, 4);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -346,12 +356,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             // fold, which triggers this launch after its own wait
             if (!a.after_prep) griddep_wait();
             const uint64_t pol = policy_evict_first();
+            // the first segment's query rows, in one copy ahead of the tiles;
+            // stage 2 takes its first tile once they have moved to TMEM
+            const bool staged = t_begin < t_end;
+            if (staged) {
+                SeqTiles s0{};
+                s0.b = -1;
+                s0 = seq_of<MODE, VARLEN>(a, t_begin, s0);
+                mbar_expect_tx(qfull, AT_QBYTES);
+                bulk_load(sbase + AT_OFF_QSTAGE, a.q + size_t(s0.b) * LCA_HEADS * LCA_D, AT_QBYTES, qfull,
+                          policy_evict_last());
+            }
             int last[3] = {-1, -1, -1};
             int i = 0;
             SeqTiles sq{};
             sq.b = -1;
             for (int64_t t = t_begin; t < t_end; ++t, ++i) {
                 const int s = i % 3;
+                if (i == 2 && !mbar_wait(qempty, 0, abort_flag, K_ATTN, 14)) break;
                 if (!mbar_wait(empty(s), ((i / 3) & 1) ^ 1, abort_flag, K_ATTN, 1)) break;
                 sq = seq_of<MODE, VARLEN>(a, t, sq);
                 const int64_t b = sq.b;
@@ -366,6 +388,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             }
             for (int s = 0; s < 3; ++s)
                 if (last[s] >= 0) mbar_wait(full(s), (last[s] / 3) & 1, nullptr, K_ATTN, 2);
+            if (staged) mbar_wait(qfull, 0, nullptr, K_ATTN, 15);   // no copy left in flight
         }
     } else if (warp == 4 || warp == 7) {
         // ------------------------------------------------------------ S issuers
@@ -442,13 +465,31 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         griddep_wait();   // the folded summary query comes from the previous kernel
         SeqTiles sq{};
         sq.b = -1;
+        if (MODE == MODE_LCA && warp == 0 && lane == 0 && t_begin < t_end) {
+            sq = seq_of<MODE, VARLEN>(a, t_begin, sq);
+            mbar_expect_tx(qfull, AT_UBYTES);
+            bulk_load(sbase + AT_OFF_QSTAGE + AT_QBYTES, a.uhl + size_t(sq.b) * 2 * LCA_D, AT_UBYTES, qfull,
+                      policy_evict_last());
+        }
         while (ok && t < t_end) {
             sq = seq_of<MODE, VARLEN>(a, t, sq);
             const int64_t b = sq.b;
             const int64_t seg_end = min64(t_end, sq.t1);
-            load_q_rows<MODE>(a, b, quad, lane, tmem);
-            tc_fence_before();
-            __syncwarp();
+            if (seg == 0) {
+                // staged by the producer (q) and by warp 0 (u) in stage 2
+                ok = mbar_wait(qfull, 0, abort_flag, K_ATTN, 16);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                const uint16_t *qs = reinterpret_cast<const uint16_t *>(smem + AT_OFF_QSTAGE);
+                load_q_rows<MODE>(qs, qs + LCA_HEADS * LCA_D, quad, lane, tmem);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(qempty);
+            } else {
+                load_q_rows<MODE>(a.q + size_t(b) * LCA_HEADS * LCA_D, a.uhl + size_t(b) * 2 * LCA_D, quad, lane,
+                                  tmem);
+                tc_fence_before();
+                __syncwarp();
+            }
             if (lane == 0) mbar_arrive(segready);
             m_use = NEG_INF;
             l_run = 0.f;

@@ -74,6 +74,23 @@ int current_device(DeviceInfo **out)
         good &= cudaFuncSetAttribute(tail_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TD_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(condense_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CP_SMEM_ALLOC) == cudaSuccess;
         good &= cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AP_SMEM_ALLOC) == cudaSuccess;
+        // One shared-memory carveout (the largest) for every kernel of the
+        // decode chain, so that an SM moving from one kernel to the next of
+        // a step need not change its L1 / shared-memory split.
+        const auto carve = [](const void *k) {
+            return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        int(cudaSharedmemCarveoutMaxShared)) == cudaSuccess;
+        };
+        good &= carve(reinterpret_cast<const void *>(attn_decode_kernel<MODE_MLA>));
+        good &= carve(reinterpret_cast<const void *>(attn_decode_kernel<MODE_REPS>));
+        good &= carve(reinterpret_cast<const void *>(attn_decode_kernel<MODE_LCA>));
+        good &= carve(reinterpret_cast<const void *>(attn_decode_kernel<MODE_MLA, true>));
+        good &= carve(reinterpret_cast<const void *>(attn_decode_kernel<MODE_LCA, true>));
+        good &= carve(reinterpret_cast<const void *>(attn_decode_kernel<MODE_REPS, true>));
+        good &= carve(reinterpret_cast<const void *>(tail_decode_kernel));
+        good &= carve(reinterpret_cast<const void *>(prep_summary_kernel));
+        good &= carve(reinterpret_cast<const void *>(append_token_kernel));
+        good &= carve(reinterpret_cast<const void *>(condense_kernel<CdShape::kWarps, CdShape::kSlots>));
         if (!good) return LCA_ERR_CUDA;
         d.attrs_set = true;
     }
@@ -337,10 +354,12 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     }
     {
         Launch l(st, K_ATTN);
-        // after the summary-query kernel (LCA) the attention prologue and its
-        // first cache loads overlap it
+        // the attention prologue overlaps the kernel before it: the
+        // summary-query kernel (LCA; then the first cache loads too) or the
+        // previous step's tail (the kernel waits for it before it reads any
+        // input or writes a partial)
         const cudaError_t e = launch_ex(attn_decode_kernel<MODE, VARLEN>, dim3(a.G), dim3(AT_THREADS), AT_SMEM_ALLOC,
-                                        st, VARLEN || (MODE == MODE_LCA && m > 0), map_cache, map_rep, a);
+                                        st, true, map_cache, map_rep, a);
         if (e != cudaSuccess || (rc = l.done())) return LCA_ERR_CUDA;
     }
     CUtensorMap map_w = map_cache;   // unused when out is NULL (a shard's partial)

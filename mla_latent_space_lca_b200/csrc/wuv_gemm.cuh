@@ -228,6 +228,24 @@ __global__ void __launch_bounds__(256, 1)
             const int c0 = n_shards ? 0 : split_owner(s0, TT, G);
             const int ns = n_shards ? n_shards : split_owner(s1 - 1, TT, G) - c0 + 1;
             const int mine = (ns - sub + wpr - 1) / wpr;   // slots sub, sub+wpr, ...
+            auto slot_vec = [&](int k) {   // this lane's 16 floats of the warp's k-th slot
+                const int s = sub + wpr * k;
+                const float *rec = n_shards ? part_o + size_t(s) * shard_stride + (size_t(b) * LCA_HEADS + h) * LCA_DC
+                                            : part_o + (size_t(c0 + s + b) * LCA_HEADS + h) * LCA_DC;
+                return reinterpret_cast<const float4 *>(rec + 16 * lane);
+            };
+            // the first NPRE slot vectors are requested together with the
+            // (m, l) pairs: one memory round trip before the first FMAs
+            constexpr int NPRE = 4;
+            const int npre = min(NPRE, mine);
+            float4 pre[NPRE][4];
+#pragma unroll
+            for (int k = 0; k < NPRE; ++k)
+                if (k < npre) {
+                    const float4 *po = slot_vec(k);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) pre[k][v] = po[v];
+                }
             for (int base = 0; base < mine; base += 32) {
                 const int cnt = min(32, mine - base);
                 float m = -INFINITY, l = 0.f;
@@ -260,15 +278,8 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
                 for (int off = 16; off; off >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, off);
                 den += dl;
-#pragma unroll 4
-                for (int k = 0; k < cnt; ++k) {
-                    const float wk = __shfl_sync(0xffffffffu, wl, k);
-                    if (wk == 0.f) continue;   // warp-uniform: skipped slots contribute nothing
-                    const int s = sub + wpr * (base + k);
-                    const float *rec = n_shards ? part_o + size_t(s) * shard_stride + (size_t(b) * LCA_HEADS + h) * LCA_DC
-                                                : part_o + (size_t(c0 + s + b) * LCA_HEADS + h) * LCA_DC;
-                    const float4 *po = reinterpret_cast<const float4 *>(rec + 16 * lane);
-                    const float4 x0 = po[0], x1 = po[1], x2 = po[2], x3 = po[3];
+                auto accumulate = [&](float wk, const float4 &x0, const float4 &x1, const float4 &x2,
+                                      const float4 &x3) {
                     acc[0] = fmaf(wk, x0.x, acc[0]); acc[1] = fmaf(wk, x0.y, acc[1]);
                     acc[2] = fmaf(wk, x0.z, acc[2]); acc[3] = fmaf(wk, x0.w, acc[3]);
                     acc[4] = fmaf(wk, x1.x, acc[4]); acc[5] = fmaf(wk, x1.y, acc[5]);
@@ -277,6 +288,23 @@ __global__ void __launch_bounds__(256, 1)
                     acc[10] = fmaf(wk, x2.z, acc[10]); acc[11] = fmaf(wk, x2.w, acc[11]);
                     acc[12] = fmaf(wk, x3.x, acc[12]); acc[13] = fmaf(wk, x3.y, acc[13]);
                     acc[14] = fmaf(wk, x3.z, acc[14]); acc[15] = fmaf(wk, x3.w, acc[15]);
+                };
+                int k0 = 0;
+                if (base == 0) {
+#pragma unroll
+                    for (int k = 0; k < NPRE; ++k) {
+                        if (k >= npre) break;
+                        const float wk = __shfl_sync(0xffffffffu, wl, k);
+                        if (wk != 0.f) accumulate(wk, pre[k][0], pre[k][1], pre[k][2], pre[k][3]);
+                    }
+                    k0 = npre;
+                }
+#pragma unroll 4
+                for (int k = k0; k < cnt; ++k) {
+                    const float wk = __shfl_sync(0xffffffffu, wl, k);
+                    if (wk == 0.f) continue;   // warp-uniform: skipped slots contribute nothing
+                    const float4 *po = slot_vec(base + k);
+                    accumulate(wk, po[0], po[1], po[2], po[3]);
                 }
             }
         }
