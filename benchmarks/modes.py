@@ -106,11 +106,12 @@ def run_stored(args, rank, world, local_rank):
     lca.profile_enable(False)
 
     # end to end, as a decode loop runs: cache, kept representatives and the
-    # recent-query ring resident on the device; per step the new token's row
-    # (into row L-1) and its query from pinned memory, the query into the
-    # ring's oldest slot, every 16th step the append of the group that left
-    # the window, the decode, out back; steps timed one by one with the L2
-    # flush between them
+    # recent-query ring resident on the device; per step lca_append_token
+    # reads the new token's row (into row L-1) and its query (into the ring's
+    # oldest slot, and a device copy for the decode) in place from pinned
+    # host memory, every 16th step the append of the group that left the
+    # window, the decode writing out straight into pinned host memory; steps
+    # timed one by one with the L2 flush between them
     pin_row = inp.cache[:, L - 1].contiguous().pin_memory()
     pin_q = inp.q.pin_memory()
     ring = q_recent.clone()
@@ -122,13 +123,11 @@ def run_stored(args, rank, world, local_rank):
     def e2e_step():
         i = n_step[0]
         n_step[0] += 1
-        cache[:, L - 1].copy_(pin_row, non_blocking=True)
-        dq.copy_(pin_q, non_blocking=True)
-        ring[:, i % ring.shape[1]].copy_(dq)
+        lca.lca_append_token(cache, L - 1, pin_row, q=pin_q, ring=ring, slot=i % ring.shape[1], q_out=dq,
+                             stream=stream)
         if i % 16 == 15 and m > 0:
             lca.lca_condense_append(cache, ring, rep, m - 1, scale=inp.scale, ws=ws, stream=stream)
-        lca.lca_decode_stored(cache, rep, dq, w_uv, scale=inp.scale, out=out, ws=ws, stream=stream)
-        h_out.copy_(out, non_blocking=True)
+        lca.lca_decode_stored(cache, rep, dq, w_uv, scale=inp.scale, out=h_out, ws=ws, stream=stream)
 
     for _ in range(3):
         e2e_step()
@@ -174,8 +173,9 @@ def run_stored(args, rank, world, local_rank):
         "e2e": {"value": B * world / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * 4,
                 "note": "decode loop: cache, kept representatives and recent-query ring resident on the "
-                        "device; per step the new token's row and query in from pinned host memory (every "
-                        "16th step also the append of one group), out back"},
+                        "device; per step lca_append_token reads the new token's row and query in place from "
+                        "pinned host memory (every 16th step also the append of one group), and the decode "
+                        "writes out straight into pinned host memory"},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = stored_cpu_baseline(inp, args.cpu_seconds / 2)

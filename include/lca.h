@@ -26,8 +26,15 @@
  *
  * Conventions for every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the
- *    library allocates no device memory.  bf16 tensors are passed as
- *    `const void*` holding IEEE bfloat16 values, row-major and contiguous.
+ *    library allocates no device memory.  Two exceptions read or write host
+ *    memory in place over the host link (no copy engine involved): `out` of
+ *    every decode and prefill entry point and of lca_combine_shards, and the
+ *    inputs of lca_append_token, may be pinned host memory mapped at the
+ *    same address (cudaHostAlloc / cudaMallocHost / cudaHostRegister); such
+ *    a pointer is checked with cudaPointerGetAttributes, and pageable or
+ *    unknown memory is refused with LCA_ERR_INVALID_ARG.  bf16 tensors are
+ *    passed as `const void*` holding IEEE bfloat16 values, row-major and
+ *    contiguous.
  *  - Every bf16 / fp32 tensor pointer must be 16-byte aligned.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
  *    asynchronous on it and never synchronise the host.  The kernels of a
@@ -325,12 +332,20 @@ int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv
  *   cache [B][pitch][576] bf16     written at row pos, 0 <= pos < pitch
  *   q     [B][16][576] bf16        the new queries, or NULL (rows only)
  *   ring  [B][g][16][576] bf16     written at slot, 0 <= slot < g; NULL with q
- * All pointers are device pointers, 16-byte aligned; B * pitch < 2^40.  The
- * kernel waits for all earlier work in the stream before it reads or
- * writes, so an earlier kernel still reading the cache is never overtaken;
- * the next call in the stream (lca_decode, ...) sees the writes. */
+ *   q_dst [B][16][576] bf16        NULL, or a second copy of q (the q that
+ *                                  lca_decode takes), written alongside
+ * 16-byte aligned; B * pitch < 2^40.  rows and q may be pinned host memory
+ * (cudaHostAlloc / cudaMallocHost / cudaHostRegister, mapped at the same
+ * address): the kernel then reads them over the host link, in place of a
+ * host-to-device copy; the host must not change them until the call has
+ * completed.  Every pointer is checked first (cudaPointerGetAttributes):
+ * pageable host memory or an unknown address gives LCA_ERR_INVALID_ARG and
+ * launches nothing.  The kernel waits for all earlier work in the stream
+ * before it reads or writes, so an earlier kernel still reading the cache is
+ * never overtaken; the next call in the stream (lca_decode, ...) sees the
+ * writes. */
 int lca_append_token(const void *rows, void *cache, int B, int64_t pitch, int64_t pos, const void *q,
-                     void *ring, int g, int slot, void *stream);
+                     void *ring, int g, int slot, void *q_dst, void *stream);
 
 /* Self-test of the failure path (no counterpart on the page): launches one
  * kernel whose bounded wait can never be satisfied.  After ~2 s it records

@@ -84,7 +84,7 @@ def lib():
         L.lca_selftest_wait_timeout.restype = I
         L.lca_selftest_wait_timeout.argtypes = [P]
         L.lca_append_token.restype = I
-        L.lca_append_token.argtypes = [P, P, I, I64, I64, P, P, I, I, P]
+        L.lca_append_token.argtypes = [P, P, I, I64, I64, P, P, I, I, P, P]
         L.lca_condense_append.restype = I
         L.lca_condense_append.argtypes = [P, P, I, I64, LcaParams, I64, P, I64, P, P, P, SZ, P]
         L.lca_decode_stored.restype = I

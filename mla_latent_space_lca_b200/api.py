@@ -37,9 +37,14 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _need(t, name, dtype, shape=None):
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
+def _need(t, name, dtype, shape=None, host=False):
+    """A contiguous tensor of this dtype (and shape) on the GPU, or, with
+    host=True, in pinned host memory (read or written in place by the
+    kernels over the host link)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if not t.is_cuda and not (host and t.is_pinned()):
+        raise TypeError(f"{name} must be a CUDA tensor" + (" or pinned host memory" if host else ""))
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -88,6 +93,9 @@ def mla_decode_attn(cache, q, w_uv, scale=None, out=None, o_lat=None, ws=None, s
     _need(q, "q", torch.bfloat16, (B, H, D))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     ws = workspace(_lib.OP_MLA_DECODE, B, L, device=cache.device) if ws is None else ws
     if pitch:   # a strided cache: MLA decode through lca_decode with g = 1
         rc = _lib.lib().lca_decode(_ptr(cache), None, _ptr(q), _ptr(w_uv), B, L, _params(1, 0, scale, 0, pitch),
@@ -127,6 +135,9 @@ def lca_decode_attn(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     if m > 0:
         _need(rep, "rep", torch.bfloat16, (B, m, D))
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_attn(_ptr(cache), _ptr(rep) if m > 0 else None, _ptr(q), _ptr(w_uv),
                                     B, L, _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(ws),
@@ -164,6 +175,9 @@ def lca_decode_stored(cache, rep, q, w_uv, g=16, w=1024, scale=None, out=None, o
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     _need(rep, "rep", torch.bfloat16)
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_stored(_ptr(cache), _ptr(rep), rep.shape[1], _ptr(q), _ptr(w_uv), B, L,
                                       _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(ws), ws.numel(),
@@ -181,6 +195,9 @@ def lca_decode(cache, q_recent, q, w_uv, g=16, w=1024, scale=None, out=None, o_l
     if g != 1:
         _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode(_ptr(cache), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
                                _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor), _ptr(ws),
@@ -202,6 +219,9 @@ def lca_decode_varlen(cache, lens, q_recent, q, w_uv, g=16, w=1024, scale=None, 
     if g != 1:
         _need(q_recent, "q_recent", torch.bfloat16, (B, g, H, D))
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     ws = workspace(_lib.OP_DECODE, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_varlen(_ptr(cache), _ptr(lens), _ptr(q_recent), _ptr(q), _ptr(w_uv), B, L,
                                       _params(g, w, scale, 0, pitch), _ptr(out), _ptr(o_lat), _ptr(anchor),
@@ -222,6 +242,9 @@ def lca_decode_stored_varlen(cache, rep, lens, q, w_uv, g=16, w=1024, scale=None
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     _need(rep, "rep", torch.bfloat16)
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=cache.device) if out is None else out
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
+    if o_lat is not None:
+        _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     ws = workspace(_lib.OP_DECODE_ATTN, B, L, g=g, w=w, device=cache.device) if ws is None else ws
     rc = _lib.lib().lca_decode_stored_varlen(_ptr(cache), _ptr(rep), rep.shape[1], _ptr(lens), _ptr(q),
                                              _ptr(w_uv), B, L, _params(g, w, scale, 0, pitch), _ptr(out),
@@ -264,7 +287,7 @@ def lca_combine_shards(parts, w_uv, B, out=None, o_lat=None, stream=None):
     _need(parts, "parts", torch.float32, (n, shard_record_floats(B)))
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     out = torch.empty(B, H, D_V, dtype=torch.float32, device=parts.device) if out is None else out
-    _need(out, "out", torch.float32, (B, H, D_V))
+    _need(out, "out", torch.float32, (B, H, D_V), host=True)
     if o_lat is not None:
         _need(o_lat, "o_lat", torch.float32, (B, H, D_C))
     rc = _lib.lib().lca_combine_shards(_ptr(parts), n, B, _ptr(w_uv), _ptr(out), _ptr(o_lat),
@@ -281,7 +304,7 @@ def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, 
     _need(w_uv, "w_uv", torch.bfloat16, (H, D_C, D_V))
     out = (torch.empty(B, q_len, H, D_V, dtype=torch.float32, device=cache.device)
            if out is None else out)
-    _need(out, "out", torch.float32, (B, q_len, H, D_V))
+    _need(out, "out", torch.float32, (B, q_len, H, D_V), host=True)
     if o_lat is not None:
         _need(o_lat, "o_lat", torch.float32, (B, q_len, H, D_C))
     if anchor is not None:
@@ -294,12 +317,14 @@ def lca_prefill_block(cache, q, w_uv, q_start, q_len, g=16, w=1024, scale=None, 
     return out
 
 
-def lca_append_token(cache, pos, rows, q=None, ring=None, slot=0, stream=None):
+def lca_append_token(cache, pos, rows, q=None, ring=None, slot=0, q_out=None, stream=None):
     """A decode loop's per-step bookkeeping in one launch: rows [B, 576] go
     into row `pos` of each sequence of `cache` ([B, L, 576], packed or a view
     of a larger [B, L_max, 576] buffer whose rows are contiguous), and, if
     given, the queries q [B, 16, 576] into slot `slot` of `ring`
-    [B, g, 16, 576] (the q_recent of the next decode call)."""
+    [B, g, 16, 576] (the q_recent of the next decode call) and into q_out
+    [B, 16, 576] (the q of the next decode call).  rows and q may be pinned
+    host tensors: the kernel reads them in place, in lieu of a copy."""
     if not isinstance(cache, torch.Tensor) or not cache.is_cuda or cache.dtype != torch.bfloat16:
         raise TypeError("cache must be a CUDA bfloat16 tensor")
     if cache.dim() != 3 or cache.shape[2] != D or cache.stride(2) != 1 or cache.stride(1) != D:
@@ -310,16 +335,18 @@ def lca_append_token(cache, pos, rows, q=None, ring=None, slot=0, stream=None):
     pitch = cache.stride(0) // D
     if not 0 <= pos < L:
         raise ValueError(f"pos {pos} outside the cache's {L} rows")
-    _need(rows, "rows", torch.bfloat16, (B, D))
+    _need(rows, "rows", torch.bfloat16, (B, D), host=True)
     g = 0
-    if q is not None or ring is not None:
-        _need(q, "q", torch.bfloat16, (B, H, D))
+    if q is not None or ring is not None or q_out is not None:
+        _need(q, "q", torch.bfloat16, (B, H, D), host=True)
         if not isinstance(ring, torch.Tensor) or ring.dim() != 4:
             raise ValueError("ring must be [B, g, 16, 576]")
         g = ring.shape[1]
         _need(ring, "ring", torch.bfloat16, (B, g, H, D))
+        if q_out is not None:
+            _need(q_out, "q_out", torch.bfloat16, (B, H, D))
     rc = _lib.lib().lca_append_token(_ptr(rows), _ptr(cache), B, pitch, int(pos), _ptr(q), _ptr(ring), g,
-                                     int(slot), _stream(stream))
+                                     int(slot), _ptr(q_out), _stream(stream))
     check(rc, "lca_append_token")
 
 

@@ -286,6 +286,23 @@ int64_t num_groups(int64_t L, const lca_params &p)
     return (L - p.w) / p.g;
 }
 
+// A pointer the kernels may dereference: device or managed memory, or pinned
+// host memory mapped at the same address (cudaHostAlloc / cudaMallocHost /
+// cudaHostRegister under unified addressing).  Pageable host memory and
+// unknown addresses are refused before anything is launched.
+int check_reachable(const void *p)
+{
+    cudaPointerAttributes at{};
+    const cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return (e == cudaErrorInvalidValue) ? LCA_ERR_INVALID_ARG : LCA_ERR_NO_DEVICE;
+    }
+    if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return LCA_OK;
+    if (at.type == cudaMemoryTypeHost && at.devicePointer == p) return LCA_OK;
+    return LCA_ERR_INVALID_ARG;
+}
+
 int check_common(const void *cache, const void *q, const void *w_uv, int B, int64_t L, float *out)
 {
     if (!cache || !q || !w_uv || !out) return LCA_ERR_INVALID_ARG;
@@ -462,7 +479,7 @@ int mla_decode_attn(const void *cache, const void *q, const void *w_uv, int B, i
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     return run_attention<MODE_MLA>(dev, cache, nullptr, q, w_uv, B, L, L, 0, 0, scale, out, o_lat, nullptr, w,
                                    static_cast<cudaStream_t>(stream));
 }
@@ -530,7 +547,7 @@ int lca_decode_stored(const void *cache, const void *rep, int64_t rep_cap, const
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, cache_pitch(p, L), m, m * p.g, p.scale, out,
                                     o_lat, nullptr, w, static_cast<cudaStream_t>(stream), rep_cap);
 }
@@ -548,7 +565,7 @@ int lca_decode_attn(const void *cache, const void *rep, const void *q, const voi
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     return run_attention<MODE_REPS>(dev, cache, rep, q, w_uv, B, L, cache_pitch(p, L), m, m * p.g, p.scale, out,
                                     o_lat, nullptr, w, static_cast<cudaStream_t>(stream));
 }
@@ -568,7 +585,7 @@ int lca_decode(const void *cache, const void *q_recent, const void *q, const voi
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t pitch = cache_pitch(p, L);
     if (p.g == 1)   // every token its own representative: MLA decode
@@ -598,7 +615,7 @@ int lca_decode_varlen(const void *cache, const int32_t *lens, const void *q_rece
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t pitch = cache_pitch(p, L);
     {
@@ -634,7 +651,7 @@ int lca_decode_stored_varlen(const void *cache, const void *rep, int64_t rep_cap
     const DecodeWs w = decode_ws_layout(ws, B);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     {
         Launch l(st, K_PREP);
@@ -663,7 +680,7 @@ int lca_decode_noalloc(const void *cache, const void *q_recent, const void *q, c
     const DecodeWs w = decode_ws_layout(scratch, B);
     if (w.bytes > kNoAllocBytes) return LCA_ERR_SCRATCH_LIMIT;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t pitch = cache_pitch(p, L);
     if (p.g == 1)
@@ -717,7 +734,7 @@ int lca_combine_shards(const float *parts, int n_shards, int B, const void *w_uv
     int rc = get_encode();
     if (rc) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     CUtensorMap map_w;
     rc = make_map3(&map_w, w_uv, LCA_DV, LCA_DC, LCA_HEADS, LCA_DV * 2, LCA_DC * LCA_DV * 2, 64, 64, 1);
@@ -753,7 +770,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
     const PrefillWs w = prefill_ws_layout(ws, B, nb, m_ld);
     if ((rc = check_ws(ws, ws_bytes, w.bytes))) return rc;
     DeviceInfo *dev = nullptr;
-    if ((rc = current_device(&dev))) return rc;
+    if ((rc = current_device(&dev)) || (rc = check_reachable(out))) return rc;   // out: device or pinned host
     if ((rc = get_encode())) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint16_t *qv = static_cast<const uint16_t *>(q);
@@ -848,22 +865,27 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
 }
 
 int lca_append_token(const void *rows, void *cache, int B, int64_t pitch, int64_t pos, const void *q, void *ring,
-                     int g, int slot, void *stream)
+                     int g, int slot, void *q_dst, void *stream)
 {
     if (!rows || !cache || B < 1 || pitch < 1 || pos < 0 || pos >= pitch) return LCA_ERR_INVALID_ARG;
     if (int64_t(B) * pitch >= (int64_t(1) << 40)) return LCA_ERR_INVALID_ARG;
-    if ((q == nullptr) != (ring == nullptr)) return LCA_ERR_INVALID_ARG;
+    if ((q == nullptr) != (ring == nullptr) || (q_dst && !q)) return LCA_ERR_INVALID_ARG;
     if (q && (g < 1 || slot < 0 || slot >= g)) return LCA_ERR_INVALID_ARG;
-    if (!aligned16(rows) || !aligned16(cache) || (q && (!aligned16(q) || !aligned16(ring))))
+    if (!aligned16(rows) || !aligned16(cache) || (q && (!aligned16(q) || !aligned16(ring))) ||
+        (q_dst && !aligned16(q_dst)))
         return LCA_ERR_MISALIGNED;
     DeviceInfo *dev = nullptr;
     int rc = current_device(&dev);
     if (rc) return rc;
+    for (const void *p : {rows, static_cast<const void *>(cache), q, static_cast<const void *>(ring),
+                          static_cast<const void *>(q_dst)})
+        if (p && (rc = check_reachable(p))) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Launch l(st, K_APPEND);
-    const cudaError_t e = launch_ex(append_token_kernel, dim3(B), dim3(APPEND_THREADS), 0, st, true,
+    const cudaError_t e = launch_ex(append_token_kernel, dim3(B, APPEND_SPLIT), dim3(APPEND_THREADS), 0, st, true,
                                     static_cast<const uint4 *>(rows), static_cast<uint4 *>(cache), pitch, pos,
-                                    static_cast<const uint4 *>(q), static_cast<uint4 *>(ring), g, slot);
+                                    static_cast<const uint4 *>(q), static_cast<uint4 *>(ring), g, slot,
+                                    static_cast<uint4 *>(q_dst));
     if (e != cudaSuccess) return LCA_ERR_CUDA;
     return l.done();
 }

@@ -222,14 +222,18 @@ def test_binding_functions_reference_only_defined_globals():
 
 def test_append_token_rejects_bad_arguments(lcalib):
     f = lcalib.lca_append_token
-    ok = dict(rows=A, cache=A, B=2, pitch=100, pos=99, q=A, ring=A, g=16, slot=15)
+    ok = dict(rows=A, cache=A, B=2, pitch=100, pos=99, q=A, ring=A, g=16, slot=15, q_dst=None)
 
     def call(**kw):
         a = dict(ok)
         a.update(kw)
-        return f(a["rows"], a["cache"], a["B"], a["pitch"], a["pos"], a["q"], a["ring"], a["g"], a["slot"], None)
+        return f(a["rows"], a["cache"], a["B"], a["pitch"], a["pos"], a["q"], a["ring"], a["g"], a["slot"],
+                 a["q_dst"], None)
 
     inval = _lib.LCA_ERR_INVALID_ARG
+    # valid arguments on the fake address: no device on a host without a GPU;
+    # with one, the address is refused by the pointer check before any launch
+    nodev = inval if __import__("torch").cuda.is_available() else _lib.LCA_ERR_NO_DEVICE
     assert call(rows=None) == inval
     assert call(cache=None) == inval
     assert call(B=0) == inval
@@ -239,5 +243,9 @@ def test_append_token_rejects_bad_arguments(lcalib):
     assert call(pitch=1 << 40, pos=0) == inval        # B * pitch must stay below 2^40
     assert call(rows=A + 8) == _lib.LCA_ERR_MISALIGNED
     assert call(ring=A + 4) == _lib.LCA_ERR_MISALIGNED
-    # rows only (no ring): valid arguments, then no device on this host
-    assert call(q=None, ring=None, g=0, slot=0) == _lib.LCA_ERR_NO_DEVICE
+    assert call(q_dst=A + 4) == _lib.LCA_ERR_MISALIGNED
+    assert call(q=None, ring=None, g=0, slot=0, q_dst=A) == inval   # a second copy of no query
+    # the second copy of q: valid arguments
+    assert call(q_dst=A) == nodev
+    # rows only (no ring): valid arguments
+    assert call(q=None, ring=None, g=0, slot=0) == nodev
