@@ -149,6 +149,15 @@ __device__ __forceinline__ SeqTiles seq_of(const AttnArgs &a, int64_t t, const S
 {
     SeqTiles s;
     if constexpr (!VARLEN) {
+        // the same sequence, or the next one (a 64-bit division otherwise)
+        if (cur.b >= 0 && t >= cur.t0 && t < cur.t1) return cur;
+        if (cur.b >= 0 && t == cur.t1) {
+            s = cur;
+            s.b = cur.b + 1;
+            s.t0 = cur.t1;
+            s.t1 = cur.t1 + a.n_tiles;
+            return s;
+        }
         s.b = t / a.n_tiles;
         s.t0 = s.b * a.n_tiles;
         s.t1 = s.t0 + a.n_tiles;

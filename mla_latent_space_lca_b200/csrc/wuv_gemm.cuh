@@ -203,6 +203,17 @@ __global__ void __launch_bounds__(256, 1)
             for (int nh = 0; nh < 2; ++nh)
                 tma_load_3d(sbase + kc * 16384 + nh * 8192, &map_w, wbar, 64 * nh, 64 * kc, h, pol);
     }
+    // The slots of this warp's row: known from the arguments alone for an
+    // even split (worked out while the attention kernel finishes); a ragged
+    // batch's tile list comes from a kernel earlier in the stream and is
+    // read after the wait.
+    const int r = warp / wpr, sub = warp % wpr;
+    int c0 = 0, ns = n_shards;
+    int64_t TT = T;
+    if (r < nb && !n_shards && !tile_start) {
+        c0 = split_owner(int64_t(b0 + r) * n_tiles, T, G);
+        ns = split_owner(int64_t(b0 + r + 1) * n_tiles - 1, T, G) - c0 + 1;
+    }
     griddep_wait();   // the split-L partials come from the attention kernel
     // Only now may the next kernel (the next step's summary-query fold)
     // start: the attention kernel that read its output buffer has finished.
@@ -213,20 +224,16 @@ __global__ void __launch_bounds__(256, 1)
     // and sum, and then the slot vectors are accumulated with independent
     // loads (no serial rescaling chain).
     {
-        const int r = warp / wpr, sub = warp % wpr;
         float M = -INFINITY, den = 0.f, acc[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) acc[e] = 0.f;
         if (r < nb) {
             const int b = b0 + r;
-            int64_t s0 = int64_t(b) * n_tiles, s1 = int64_t(b + 1) * n_tiles, TT = T;
-            if (tile_start) {
-                s0 = tile_start[b];
-                s1 = tile_start[b + 1];
+            if (tile_start && !n_shards) {
                 TT = tile_start[B];
+                c0 = split_owner(int64_t(tile_start[b]), TT, G);
+                ns = split_owner(int64_t(tile_start[b + 1]) - 1, TT, G) - c0 + 1;
             }
-            const int c0 = n_shards ? 0 : split_owner(s0, TT, G);
-            const int ns = n_shards ? n_shards : split_owner(s1 - 1, TT, G) - c0 + 1;
             const int mine = (ns - sub + wpr - 1) / wpr;   // slots sub, sub+wpr, ...
             auto slot_vec = [&](int k) {   // this lane's 16 floats of the warp's k-th slot
                 const int s = sub + wpr * k;
@@ -254,9 +261,10 @@ __global__ void __launch_bounds__(256, 1)
                     if (n_shards) {
                         m = part_o[size_t(s) * shard_stride + lse_off + size_t(b) * LCA_HEADS + h];
                         l = 1.f;
-                    } else if (split_begin(c0 + s + 1, TT, G) > split_begin(c0 + s, TT, G)) {
+                    } else if (!tile_start || split_begin(c0 + s + 1, TT, G) > split_begin(c0 + s, TT, G)) {
                         // (a ragged batch can have fewer tiles than CTAs: a CTA
-                        // owning none wrote no slot, and its slot is skipped)
+                        // owning none wrote no slot, and its slot is skipped;
+                        // an even split gives every CTA a tile)
                         const size_t sl = size_t(c0 + s + b) * LCA_HEADS + h;
                         const float2 ml = *reinterpret_cast<const float2 *>(part_ml + sl * 2);
                         m = ml.x;
@@ -320,34 +328,39 @@ __global__ void __launch_bounds__(256, 1)
     }
     __syncthreads();
     // ---- per row: the warps' common max, the denominator and each warp's
-    // weight, once (thread r handles row r)
+    // weight (warp r handles row r, lane i the state of warp i of the row)
     float *coef = reinterpret_cast<float *>(smem + TD_OFF_COEF);
-    if (threadIdx.x < nb) {
-        const int r = threadIdx.x;
-        float Mt = -INFINITY;
-        for (int i = 0; i < wpr; ++i) Mt = fmaxf(Mt, scr[(r * wpr + i) * TD_SCR_STRIDE + LCA_DC]);
-        float dt = 0.f;
-        for (int i = 0; i < wpr; ++i) {
-            const float *wp = scr + (r * wpr + i) * TD_SCR_STRIDE;
-            const float f = (wp[LCA_DC] == -INFINITY) ? 0.f : fast_exp2(wp[LCA_DC] - Mt);
-            coef[r * 8 + i] = f;
-            dt = fmaf(f, wp[LCA_DC + 1], dt);
-        }
-        const float inv = 1.f / dt;
-        for (int i = 0; i < wpr; ++i) coef[r * 8 + i] *= inv;
-        if (lse_out) lse_out[size_t(b0 + r) * LCA_HEADS + h] = Mt + log2f(dt);
+    if (warp < nb) {
+        const int rr = warp;
+        const float *wp = scr + (rr * wpr + (lane & 7)) * TD_SCR_STRIDE;
+        const float mi = (lane < wpr) ? wp[LCA_DC] : -INFINITY;
+        const float di = (lane < wpr) ? wp[LCA_DC + 1] : 0.f;
+        float Mt = mi;
+#pragma unroll
+        for (int off = 4; off; off >>= 1) Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, off));
+        const float f = (mi == -INFINITY) ? 0.f : fast_exp2(mi - Mt);
+        float dt = f * di;
+#pragma unroll
+        for (int off = 4; off; off >>= 1) dt += __shfl_xor_sync(0xffffffffu, dt, off);
+        if (lane < wpr) coef[rr * 8 + lane] = f * (1.f / dt);
+        if (lse_out && lane == 0) lse_out[size_t(b0 + rr) * LCA_HEADS + h] = Mt + log2f(dt);
     }
     __syncthreads();
     // ---- merge the warps of each row; o -> o_lat (fp32) and the B operand (bf16)
-    for (int r = 0; r < TD_N; ++r) {
+    // (rows nb .. TD_N-1 of the B operand are left as they are: they only
+    // feed output columns that are never stored)
+    for (int r = 0; r < nb; ++r) {
         const int k = 2 * threadIdx.x;   // 256 threads x 2 columns
         float o0 = 0.f, o1 = 0.f;
-        if (r < nb) {
-            for (int i = 0; i < wpr; ++i) {
-                const float c = coef[r * 8 + i];
-                const float2 x = *reinterpret_cast<const float2 *>(scr + (r * wpr + i) * TD_SCR_STRIDE + k);
-                o0 = fmaf(c, x.x, o0);
-                o1 = fmaf(c, x.y, o1);
+        {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (i < wpr) {
+                    const float c = coef[r * 8 + i];
+                    const float2 x = *reinterpret_cast<const float2 *>(scr + (r * wpr + i) * TD_SCR_STRIDE + k);
+                    o0 = fmaf(c, x.x, o0);
+                    o1 = fmaf(c, x.y, o1);
+                }
             }
             if (o_lat)
                 *reinterpret_cast<float2 *>(o_lat + (size_t(b0 + r) * LCA_HEADS + h) * LCA_DC + k) =
