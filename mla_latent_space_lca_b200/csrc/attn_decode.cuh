@@ -1,8 +1,9 @@
 // attn_decode.cuh -- split-L flash-decode attention on tcgen05 tensor cores,
 // read straight from the MLA latent cache, with the LCA condensation fused in.
 //
-// Row sources ("tiles" of 64 rows, 1152 B each, TMA-loaded as 9 boxes of
-// [64 rows x 64 columns] with 128-byte swizzle, 72 KB per stage, 3 stages):
+// Row sources ("tiles" of 64 rows, 1152 B each, brought in by one 4-D TMA
+// copy as 9 blocks of [64 rows x 64 columns] with 128-byte swizzle, 72 KB
+// per stage, 3 stages):
 //   MODE_MLA : cache rows 0..L-1 (MLA decode, every token attends).
 //   MODE_REPS: stored representatives rep[b][0..m) then window rows m*g..L-1.
 //   MODE_LCA : raw history rows 0..m*16-1 (4 groups of 16 per tile), condensed
@@ -389,10 +390,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                 const TileInfo ti = tile_info<MODE>(sq.g, int(t - sq.t0));
                 mbar_expect_tx(full(s), AT_STAGE);
                 const CUtensorMap *mp = ti.from_rep ? &map_rep : &map_cache;
-                const uint32_t dst = sbase + s * AT_STAGE;
-#pragma unroll 1
-                for (int ch = 0; ch < 9; ++ch)
-                    tma_load_3d(dst + ch * AT_CHUNK, mp, full(s), 64 * ch, int(ti.row), int(b), pol);
+                // the whole tile, all nine 64-column blocks, in one copy
+                tma_load_4d(sbase + s * AT_STAGE, mp, full(s), 0, int(ti.row), 0, int(b), pol);
                 last[s] = i;
             }
             for (int s = 0; s < 3; ++s)

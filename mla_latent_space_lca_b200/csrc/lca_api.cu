@@ -129,6 +129,24 @@ int make_map3(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64
     return r == CUDA_SUCCESS ? LCA_OK : LCA_ERR_CUDA;
 }
 
+// Rows of 576 bf16 ([B][pitch][576]) as a 4-D tensor of 64-column chunks:
+// (column within the chunk, row, chunk, sequence), so that one TMA box of
+// [9 chunks][box_rows rows][64 columns] brings box_rows whole rows into
+// shared memory in the layout of nine [rows x 64 columns] 128B-swizzled
+// blocks, one per chunk.
+int make_map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint64_t B, uint64_t pitch_rows,
+                  uint32_t box_rows)
+{
+    cuuint64_t dims[4] = {64, rows, LCA_D / 64, B};
+    cuuint64_t strides[3] = {uint64_t(LCA_D) * 2, 128, pitch_rows * LCA_D * 2};
+    cuuint32_t box[4] = {64, box_rows, LCA_D / 64, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LCA_OK : LCA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ timing / counting
 struct ProfRec {
     cudaEvent_t a, b;
@@ -357,14 +375,12 @@ int run_attention(DeviceInfo *dev, const void *cache, const void *rep, const voi
     a.after_prep = (!VARLEN && MODE == MODE_LCA && m > 0) ? 1 : 0;
 
     CUtensorMap map_cache, map_rep;
-    rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2,
-                   uint64_t(pitch) * LCA_D * 2, 64, AT_TILE, 1);
+    rc = make_map_rows(&map_cache, cache, uint64_t(L), uint64_t(B), uint64_t(pitch), AT_TILE);
     if (rc) return rc;
     if (MODE == MODE_REPS && m > 0) {
         // rows per sequence: m, or the capacity of a representative cache
         const uint64_t stride_rows = uint64_t(rep_stride > 0 ? rep_stride : m);
-        rc = make_map3(&map_rep, rep, LCA_D, uint64_t(m), uint64_t(B), uint64_t(LCA_D) * 2,
-                       stride_rows * LCA_D * 2, 64, AT_TILE, 1);
+        rc = make_map_rows(&map_rep, rep, uint64_t(m), uint64_t(B), stride_rows, AT_TILE);
         if (rc) return rc;
     } else {
         map_rep = map_cache;
