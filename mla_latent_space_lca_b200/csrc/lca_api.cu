@@ -147,6 +147,21 @@ int make_map_rows(CUtensorMap *m, const void *base, uint64_t rows, uint64_t B, u
     return r == CUDA_SUCCESS ? LCA_OK : LCA_ERR_CUDA;
 }
 
+// The prefill's group-major representatives [groups][nbc blocks][576] as a
+// 4-D tensor (column within the chunk, block, group, chunk): a box of 64
+// groups of one block lands as nine [64 groups x 64 columns] blocks.
+int make_map_reps(CUtensorMap *m, const void *base, uint64_t nbc, uint64_t groups)
+{
+    cuuint64_t dims[4] = {64, nbc, groups, LCA_D / 64};
+    cuuint64_t strides[3] = {uint64_t(LCA_D) * 2, nbc * LCA_D * 2, 128};
+    cuuint32_t box[4] = {64, 1, 64, LCA_D / 64};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+                          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? LCA_OK : LCA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ timing / counting
 struct ProfRec {
     cudaEvent_t a, b;
@@ -793,15 +808,13 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
 
     CUtensorMap map_cache, map_rows, map_q, map_u, map_w;
     const uint64_t seq_bytes = uint64_t(cache_pitch(p, L)) * LCA_D * 2;
-    if ((rc = make_map3(&map_cache, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2, seq_bytes, 64, 64,
-                        1)))
+    if ((rc = make_map_rows(&map_cache, cache, uint64_t(L), uint64_t(B), uint64_t(cache_pitch(p, L)), 64)))
         return rc;
     // the condensation's history tiles: CP_ROWS rows
     if ((rc = make_map3(&map_rows, cache, LCA_D, uint64_t(L), uint64_t(B), uint64_t(LCA_D) * 2, seq_bytes, 64,
                         CP_ROWS, 1)))
         return rc;
-    if ((rc = make_map3(&map_q, q, LCA_D, uint64_t(L) * LCA_HEADS, uint64_t(B), uint64_t(LCA_D) * 2,
-                        uint64_t(L) * LCA_HEADS * LCA_D * 2, 64, 64, 1)))
+    if ((rc = make_map_rows(&map_q, q, uint64_t(L) * LCA_HEADS, uint64_t(B), uint64_t(L) * LCA_HEADS, 64)))
         return rc;
     if ((rc = make_map3(&map_u, w.uhl, LCA_D, 2, uint64_t(B) * uint64_t(nb), uint64_t(LCA_D) * 2,
                         uint64_t(LCA_D) * 4, 64, 1, 128)))
@@ -826,8 +839,7 @@ int lca_prefill_block(const void *cache, const void *q, const void *w_uv, int B,
             CUtensorMap map_rep = map_cache;
             if (n_gt > 0) {
                 // group-major [CP_G n_gt][nbc][576]; a box is 64 groups of one block
-                if ((rc = make_map3(&map_rep, w.rep, LCA_D, uint64_t(nbc), uint64_t(CP_G) * n_gt, uint64_t(LCA_D) * 2,
-                                    uint64_t(nbc) * LCA_D * 2, 64, 1, 64)))
+                if ((rc = make_map_reps(&map_rep, w.rep, uint64_t(nbc), uint64_t(CP_G) * n_gt)))
                     return rc;
                 CondPreArgs c{};
                 c.kc0 = kc0;

@@ -45,12 +45,23 @@
 
 namespace lca {
 
-// Prefetch a 3-D tensor box into L2 (no shared memory, no completion).
-__device__ __forceinline__ void pf_prefetch_3d(const CUtensorMap *map, int x, int y, int z)
+// 4-D tiled TMA load without an eviction hint, and its L2 prefetch form (a
+// box into L2 only: no shared memory, no completion).
+__device__ __forceinline__ void tma_load_4d_plain(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int y,
+                                                  int z, int w)
 {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void pf_prefetch_4d(const CUtensorMap *map, int x, int y, int z, int w)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y), "r"(z)
+                 "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
 }
 
@@ -492,9 +503,8 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
             prefetch_tensormap(&map_cache);
             if (n_rep > 0) prefetch_tensormap(&map_rep);
             mbar_expect_tx(qfull, AP_STAGE);
-#pragma unroll 1
-            for (int ch = 0; ch < 9; ++ch)
-                tma_load_3d_plain(qbase + ch * AP_CHUNK, &map_q, qfull, 64 * ch, int(16 * t_first), a.b);
+            // each of these copies brings 64 whole rows (nine 64-column blocks)
+            tma_load_4d_plain(qbase, &map_q, qfull, 0, int(16 * t_first), 0, a.b);
             int last[2] = {-1, -1};
 #pragma unroll 1
             for (int i = 0; i < n_tiles; ++i) {
@@ -503,20 +513,15 @@ __global__ void __launch_bounds__(AP_THREADS, 1)
                 mbar_expect_tx(full(s), AP_STAGE);
                 const uint32_t dst = stage_addr(i);
                 if (i < n_rep) {
-#pragma unroll 1
-                    for (int ch = 0; ch < 9; ++ch)
-                        tma_load_3d_plain(dst + ch * AP_CHUNK, &map_rep, full(s), 64 * ch, int(k - a.kc0), 64 * i);
+                    tma_load_4d_plain(dst, &map_rep, full(s), 0, int(k - a.kc0), 64 * i, 0);
                     // the block's first CTA warms L2 with the next representative
                     // tile for itself and the block's other three CTAs
                     if (qq == 0 && i + 1 < n_rep) {
-#pragma unroll 1
-                        for (int ch = 0; ch < 9; ++ch) pf_prefetch_3d(&map_rep, 64 * ch, int(k - a.kc0), 64 * (i + 1));
+                        pf_prefetch_4d(&map_rep, 0, int(k - a.kc0), 64 * (i + 1), 0);
                     }
                 } else {
                     const int row = int(win0 + 64 * (i - n_rep));
-#pragma unroll 1
-                    for (int ch = 0; ch < 9; ++ch)
-                        tma_load_3d_plain(dst + ch * AP_CHUNK, &map_cache, full(s), 64 * ch, row, a.b);
+                    tma_load_4d_plain(dst, &map_cache, full(s), 0, row, 0, a.b);
                 }
                 last[s] = i;
             }
