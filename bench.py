@@ -51,7 +51,9 @@ def parse(argv=None):
     ap.add_argument("--workload", default=None,
                     help=f"one workload only (default: the suite, headline {HEADLINE})")
     ap.add_argument("--no-suite", action="store_true", help="default run: the headline workload only")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="end-to-end steps (default: as many as the timed steps, so that both figures are "
+                         "taken in the same power state)")
     ap.add_argument("--e2e-full-copy", type=int, default=2,
                     help="decode: also time N steps that copy the whole cache in from the host")
     ap.add_argument("--no-e2e-graph", action="store_true",
@@ -104,6 +106,8 @@ def run_ours(args, rank, world, local_rank):
     single = args.workload is not None
     workload = args.workload or HEADLINE
     steps, warmup = defaults(args, workload)
+    if args.e2e_steps is None:
+        args.e2e_steps = steps
     kind = WORKLOADS[workload]["kind"]
     if args.stored or args.varlen or args.split_l:
         args.workload, args.steps, args.warmup = workload, steps, warmup
@@ -127,7 +131,7 @@ def run_ours(args, rank, world, local_rank):
     # 90% KV-cache reading (each step reads 7% of the rows)
     st_args = argparse.Namespace(**vars(args))
     st_args.workload, st_args.steps, st_args.warmup = HEADLINE, min(steps, 500), max(3, min(warmup, 20))
-    st_args.e2e_steps = min(args.e2e_steps, 5)
+    st_args.e2e_steps = st_args.steps
     sub = run_stored(st_args, rank, world, local_rank)
     if sub is not None:
         nested[HEADLINE + "_stored"] = suite_entry(sub)
